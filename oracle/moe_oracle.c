@@ -1,0 +1,665 @@
+/*
+ * moe_oracle.c -- the ORACLE for the MoE dispatch / combine path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is a plain, slow, single-threaded CPU
+ * statement of what every step of the path computes, written so that a
+ * reader can check it against the source pages by eye.  It exists to check
+ * the CUDA library, never to stand in for it: only the test suite, the smoke
+ * check and the benchmark's CPU-baseline leg may load it.  It shares no code,
+ * header, table or helper with the CUDA library.
+ *
+ * Sources (page title -- section):
+ *   [EC]  "Expert Coupling in MoE Pretraining: Reducing All-to-All Overhead
+ *          with Correlated Placement and Token Shuffling" (PicX summary)
+ *   [DD]  "DODOCO: MoE AlltoAll Traffic Matrices on Real Text" (dataset card)
+ *   [A2A] "AllToAllDispatchScenario" (mlsysim API page)
+ *
+ * Notation: T tokens, H hidden size, E experts, k = top-k, R = expert-parallel
+ * ranks, T_r = T / R tokens per source rank, src(t) = t / T_r, p[e] = rank
+ * holding expert e, S(t) = token t's selected experts in slot order.
+ *
+ * Floating point: gates are computed in double and rounded once to float.
+ * The combine accumulates in float with explicit fmaf, because that
+ * accumulation order and precision is part of the specified result.
+ *
+ * Every function returns 0 on success and a non-zero code on bad arguments.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* bf16 <-> float, round-to-nearest-even written out.                        */
+/* ------------------------------------------------------------------------ */
+
+static float bf16_to_float(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static uint16_t float_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u)      /* NaN: keep it a quiet NaN */
+        return (uint16_t)((u >> 16) | 0x0040u);
+    /* add half an ulp of the kept part, plus one if the kept part is odd */
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Router: top-k selection and gate weights.                                 */
+/* [EC] "Background": each token is routed to its top-k of E experts.        */
+/* [EC] "Method 1": routing probabilities travel with the dispatched rows.   */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    float logit;
+    int32_t expert;
+} cand_t;
+
+/* Larger logit first (IEEE comparison, so -0.0 equals +0.0); equal logits:
+ * lower expert index first. */
+static int cmp_cand(const void *a, const void *b)
+{
+    const cand_t *x = (const cand_t *)a, *y = (const cand_t *)b;
+    if (x->logit > y->logit) return -1;
+    if (x->logit < y->logit) return 1;
+    return (x->expert > y->expert) - (x->expert < y->expert);
+}
+
+/*
+ * idx[t*k + j] = the j-th expert of token t in (logit desc, expert asc) order.
+ * gate_mode 0: w_j = softmax over the k selected logits.
+ * gate_mode 1: w_j = softmax over all E logits, read at the selected experts.
+ * Both use the largest logit (slot 0) as the shift; the result is rounded to
+ * float once.
+ */
+int oracle_route_topk(const float *logits, int64_t T, int E, int k, int gate_mode,
+                      int32_t *idx, float *w)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E || (gate_mode != 0 && gate_mode != 1))
+        return 1;
+    cand_t *c = (cand_t *)malloc(sizeof(cand_t) * (size_t)E);
+    if (!c) return 2;
+    for (int64_t t = 0; t < T; ++t) {
+        const float *row = logits + t * E;
+        for (int e = 0; e < E; ++e) {
+            c[e].logit = row[e];
+            c[e].expert = e;
+        }
+        qsort(c, (size_t)E, sizeof(cand_t), cmp_cand);
+        for (int j = 0; j < k; ++j)
+            idx[t * k + j] = c[j].expert;
+
+        double m = (double)c[0].logit;
+        double denom = 0.0;
+        if (gate_mode == 0) {
+            for (int j = 0; j < k; ++j) denom += exp((double)c[j].logit - m);
+        } else {
+            for (int e = 0; e < E; ++e) denom += exp((double)row[e] - m);
+        }
+        for (int j = 0; j < k; ++j)
+            w[t * k + j] = (float)(exp((double)c[j].logit - m) / denom);
+    }
+    free(c);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dispatch layout.                                                          */
+/* [DD] "Reading the counts": counts are token-expert assignments, a token   */
+/*      sent to several experts on one rank is counted once per expert, and  */
+/*      each row of the send matrix sums to (tokens per rank) x top-k.       */
+/* [DD] "Setup": each rank routes a contiguous block of tokens; contiguous   */
+/*      placement puts experts r*E/R .. (r+1)*E/R-1 on rank r.               */
+/* [EC] "Method 1": the deduplicating dispatcher sends one row per distinct  */
+/*      (token, destination rank) pair, carrying every selected expert there.*/
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int64_t a, b, c;    /* sort key, compared in this order */
+    int64_t t;
+    int j;
+} lkey_t;
+
+static int cmp_lkey(const void *x_, const void *y_)
+{
+    const lkey_t *x = (const lkey_t *)x_, *y = (const lkey_t *)y_;
+    if (x->a != y->a) return x->a < y->a ? -1 : 1;
+    if (x->b != y->b) return x->b < y->b ? -1 : 1;
+    if (x->c != y->c) return x->c < y->c ? -1 : 1;
+    return 0;
+}
+
+/*
+ * Conventional rows: one per (t, j), ordered by (p[e], e, t) with e = S(t)_j,
+ * i.e. grouped by destination rank, then by expert, then by token.
+ * Dedup rows: one per distinct (t, d) with d in {p[e] : e in S(t)}, ordered
+ * by (d, t); bit j of the row's mask is set when p[S(t)_j] = d.
+ *
+ * Outputs (all sizes are the caller's):
+ *   assign_row[T*k]      conventional row of (t, j), in both modes
+ *   row_of_slot[T*k]     row of (t, j) in this mode's layout
+ *   row_token[n_rows]    token of each row
+ *   row_mask[n_rows]     slots of that token carried by the row
+ *   send_counts[R*R]     [s*R + d] rows from source rank s to rank d
+ *   expert_counts[E]     #{t : e in S(t)}
+ *   expert_offsets[E+1]  first conventional row of expert e; [E] = T*k
+ *   rank_offsets[R+1]    first row of rank d in this mode; [R] = n_rows
+ *   n_rows               number of rows in this mode
+ */
+int oracle_dispatch_layout(const int32_t *idx, int64_t T, int E, int k, int R,
+                           const int32_t *p, int mode,
+                           int32_t *row_of_slot, int32_t *assign_row,
+                           int32_t *row_token, uint32_t *row_mask,
+                           int64_t *send_counts, int64_t *expert_counts,
+                           int64_t *expert_offsets, int64_t *rank_offsets,
+                           int64_t *n_rows)
+{
+    if (T < 0 || E < 1 || k < 1 || k > E || k > 32 || R < 1 || T % R != 0 ||
+        (mode != 0 && mode != 1))
+        return 1;
+    for (int e = 0; e < E; ++e)
+        if (p[e] < 0 || p[e] >= R) return 1;
+    for (int64_t i = 0; i < T * k; ++i)
+        if (idx[i] < 0 || idx[i] >= E) return 1;
+    const int64_t Tr = T / R;
+    if (Tr == 0) {             /* no tokens: everything is empty */
+        for (int e = 0; e < E; ++e) { expert_counts[e] = 0; expert_offsets[e] = 0; }
+        expert_offsets[E] = 0;
+        for (int64_t i = 0; i < (int64_t)R * R; ++i) send_counts[i] = 0;
+        for (int d = 0; d <= R; ++d) rank_offsets[d] = 0;
+        *n_rows = 0;
+        return 0;
+    }
+
+    /* conventional positions: sort all (t, j) by (p[e], e, t) */
+    int64_t npairs = T * k;
+    lkey_t *keys = (lkey_t *)malloc(sizeof(lkey_t) * (size_t)(npairs > 0 ? npairs : 1));
+    if (!keys) return 2;
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int e = idx[t * k + j];
+            lkey_t *q = &keys[t * k + j];
+            q->a = p[e];
+            q->b = e;
+            q->c = t;
+            q->t = t;
+            q->j = j;
+        }
+    qsort(keys, (size_t)npairs, sizeof(lkey_t), cmp_lkey);
+    for (int64_t i = 0; i < npairs; ++i)
+        assign_row[keys[i].t * k + keys[i].j] = (int32_t)i;
+
+    for (int e = 0; e < E; ++e) expert_counts[e] = 0;
+    for (int64_t i = 0; i < npairs; ++i) expert_counts[idx[i]] += 1;
+
+    /* first conventional row of expert e = number of pairs whose (p, e')
+     * key sorts before (p[e], e) */
+    for (int e = 0; e < E; ++e) {
+        int64_t before = 0;
+        for (int e2 = 0; e2 < E; ++e2)
+            if (p[e2] < p[e] || (p[e2] == p[e] && e2 < e)) before += expert_counts[e2];
+        expert_offsets[e] = before;
+    }
+    expert_offsets[E] = npairs;
+
+    for (int64_t i = 0; i < (int64_t)R * R; ++i) send_counts[i] = 0;
+
+    if (mode == 0) {
+        for (int64_t i = 0; i < npairs; ++i) {
+            int64_t t = keys[i].t;
+            int j = keys[i].j;
+            row_of_slot[t * k + j] = (int32_t)i;
+            row_token[i] = (int32_t)t;
+            row_mask[i] = 1u << j;
+        }
+        for (int64_t t = 0; t < T; ++t)
+            for (int j = 0; j < k; ++j)
+                send_counts[(t / Tr) * R + p[idx[t * k + j]]] += 1;
+        for (int d = 0; d <= R; ++d) {
+            int64_t before = 0;
+            for (int e = 0; e < E; ++e)
+                if (p[e] < d) before += expert_counts[e];
+            rank_offsets[d] = before;
+        }
+        *n_rows = npairs;
+        free(keys);
+        return 0;
+    }
+
+    /* dedup: one entry per distinct (t, d), sorted by (d, t) */
+    int64_t nd = 0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int d = p[idx[t * k + j]];
+            int seen = 0;
+            for (int j2 = 0; j2 < j; ++j2)
+                if (p[idx[t * k + j2]] == d) seen = 1;
+            if (!seen) {
+                lkey_t *q = &keys[nd++];
+                q->a = d;
+                q->b = t;
+                q->c = 0;
+                q->t = t;
+                q->j = d; /* remember the rank */
+            }
+        }
+    qsort(keys, (size_t)nd, sizeof(lkey_t), cmp_lkey);
+    for (int64_t i = 0; i < nd; ++i) {
+        int64_t t = keys[i].t;
+        int d = keys[i].j;
+        uint32_t mask = 0;
+        for (int j = 0; j < k; ++j)
+            if (p[idx[t * k + j]] == d) {
+                mask |= 1u << j;
+                row_of_slot[t * k + j] = (int32_t)i;
+            }
+        row_token[i] = (int32_t)t;
+        row_mask[i] = mask;
+        send_counts[(t / Tr) * R + d] += 1;
+    }
+    for (int d = 0; d <= R; ++d) {
+        int64_t before = 0;
+        for (int64_t i = 0; i < nd; ++i)
+            if (keys[i].j < d) before += 1;
+        rank_offsets[d] = before;
+    }
+    *n_rows = nd;
+    free(keys);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Dispatch permute.  The dispatch buffer holds, in row order, the hidden    */
+/* state of each row's token ([DD] "Reading the counts": payload = count x   */
+/* hidden x bytes per element).                                              */
+/* ------------------------------------------------------------------------ */
+
+int oracle_dispatch_permute(const uint16_t *x, int64_t T, int64_t H,
+                            const int32_t *row_token, int64_t n_rows, uint16_t *out)
+{
+    if (T < 0 || H < 1 || n_rows < 0) return 1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t t = row_token[r];
+        if (t < 0 || t >= T) return 1;
+        memcpy(out + r * H, x + t * H, sizeof(uint16_t) * (size_t)H);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Combine.                                                                  */
+/* [DD] "Send matrices": combine returns the same volumes in reverse.        */
+/* [EC] "The Communication Bottleneck": dispatch and combine per MoE layer.  */
+/* The result is the gate-weighted sum of the token's expert outputs,        */
+/* accumulated in float in ascending expert order and rounded to bf16 once.  */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int64_t key1, key2;
+    int j;
+} slot_t;
+
+static int cmp_slot(const void *x_, const void *y_)
+{
+    const slot_t *x = (const slot_t *)x_, *y = (const slot_t *)y_;
+    if (x->key1 != y->key1) return x->key1 < y->key1 ? -1 : 1;
+    if (x->key2 != y->key2) return x->key2 < y->key2 ? -1 : 1;
+    return (x->j > y->j) - (x->j < y->j);
+}
+
+/*
+ * y: expert outputs, one row per (t, j) at row assign_row[t*k+j], bf16 [*, H].
+ * mode 0 (fused): out[t] = bf16( sum over slots by ascending expert of
+ *                 fmaf(w, y, acc) ), acc starting at +0.0f.
+ * mode 1 (wire):  for each destination rank d of t, ascending d:
+ *                   z(t,d) = bf16( same sum over the slots with p[e] = d );
+ *                   written to z at row row_of_slot of those slots;
+ *                 out[t] = bf16( sum over ascending d of float(z(t,d)) ).
+ */
+int oracle_combine(const uint16_t *y, int64_t y_rows, const int32_t *assign_row,
+                   const int32_t *idx, const float *w, int64_t T, int k, int64_t H,
+                   int mode, const int32_t *p, int R, const int32_t *row_of_slot,
+                   uint16_t *z, uint16_t *out)
+{
+    if (T < 0 || k < 1 || H < 1 || (mode != 0 && mode != 1)) return 1;
+    slot_t *s = (slot_t *)malloc(sizeof(slot_t) * (size_t)k);
+    if (!s) return 2;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int64_t r = assign_row[t * k + j];
+            if (r < 0 || r >= y_rows) { free(s); return 1; }
+            int e = idx[t * k + j];
+            s[j].key1 = mode == 0 ? e : p[e];
+            s[j].key2 = e;
+            s[j].j = j;
+        }
+        qsort(s, (size_t)k, sizeof(slot_t), cmp_slot);
+        for (int64_t h = 0; h < H; ++h) {
+            if (mode == 0) {
+                float acc = 0.0f;
+                for (int i = 0; i < k; ++i) {
+                    int j = s[i].j;
+                    float v = bf16_to_float(y[(int64_t)assign_row[t * k + j] * H + h]);
+                    acc = fmaf(w[t * k + j], v, acc);
+                }
+                out[t * H + h] = float_to_bf16(acc);
+            } else {
+                float total = 0.0f;
+                int i = 0;
+                while (i < k) {
+                    int64_t d = s[i].key1;
+                    int64_t zrow = row_of_slot[t * k + s[i].j];
+                    float acc = 0.0f;
+                    for (; i < k && s[i].key1 == d; ++i) {
+                        int j = s[i].j;
+                        float v = bf16_to_float(y[(int64_t)assign_row[t * k + j] * H + h]);
+                        acc = fmaf(w[t * k + j], v, acc);
+                    }
+                    uint16_t zb = float_to_bf16(acc);
+                    if (z) z[zrow * H + h] = zb;
+                    total = total + bf16_to_float(zb);
+                }
+                out[t * H + h] = float_to_bf16(total);
+            }
+        }
+    }
+    (void)R;
+    free(s);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Co-selection statistics.                                                  */
+/* [EC] "Correlated Placement": W[e,e'] counts tokens selecting both e, e'.  */
+/* [EC] "Cross-layer correlation": layer-l experts predict layer-l+1 ones.   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * W[e*E+e'] += #{t < T_fit : e in S(t) and e' in S(t)}  (diagonal = load)
+ * C[e*E+e'] += #{(t, i, j) : t < T_fit, S_l(t)_i = e, S_l+1(t)_j = e'}
+ * W or C may be NULL; accumulate = 0 clears them first.
+ */
+int oracle_coselect(const int32_t *idx_l, const int32_t *idx_next, int64_t T_fit,
+                    int E, int k, uint32_t *W, uint32_t *C, int accumulate)
+{
+    if (T_fit < 0 || E < 1 || k < 1) return 1;
+    if (!accumulate) {
+        if (W) memset(W, 0, sizeof(uint32_t) * (size_t)E * E);
+        if (C) memset(C, 0, sizeof(uint32_t) * (size_t)E * E);
+    }
+    for (int64_t t = 0; t < T_fit; ++t)
+        for (int i = 0; i < k; ++i)
+            for (int j = 0; j < k; ++j) {
+                int a = idx_l[t * k + i];
+                if (a < 0 || a >= E) return 1;
+                if (W) {
+                    int b = idx_l[t * k + j];
+                    W[(int64_t)a * E + b] += 1;
+                }
+                if (C && idx_next) {
+                    int b = idx_next[t * k + j];
+                    if (b < 0 || b >= E) return 1;
+                    C[(int64_t)a * E + b] += 1;
+                }
+            }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Correlated placement.                                                     */
+/* [EC] "Correlated Placement": a Kernighan-Lin-style local search starts    */
+/* from contiguous placement and swaps experts between GPUs to maximise the  */
+/* sum of W over pairs that share a GPU; every GPU keeps exactly E/EP        */
+/* experts.  The page does not print the search itself, so the steps below  */
+/* are the plainest reading: repeat the single best swap while it gains.     */
+/* ------------------------------------------------------------------------ */
+
+/* sum of W[e][e'] over unordered pairs e != e' on the same rank */
+long long oracle_placement_objective(const uint32_t *W, int E, const int32_t *p)
+{
+    long long s = 0;
+    for (int a = 0; a < E; ++a)
+        for (int b = a + 1; b < E; ++b)
+            if (p[a] == p[b]) s += (long long)W[(int64_t)a * E + b];
+    return s;
+}
+
+typedef struct {
+    uint32_t wv;
+    int a, b;
+} pair_t;
+
+static int cmp_pair(const void *x_, const void *y_)
+{
+    const pair_t *x = (const pair_t *)x_, *y = (const pair_t *)y_;
+    if (x->wv != y->wv) return x->wv > y->wv ? -1 : 1;
+    if (x->a != y->a) return x->a < y->a ? -1 : 1;
+    return (x->b > y->b) - (x->b < y->b);
+}
+
+/*
+ * seed_mode 0: start from contiguous placement (the page's starting point).
+ * seed_mode 1: greedy pair seed ("co-locate the top pairs first"): scan the
+ *   pairs e < e' with W[e][e'] > 0 by (W desc, e asc, e' asc);
+ *   both unplaced  -> both go to the rank with the most free slots (lowest
+ *                     rank on ties) if it has at least two;
+ *   one placed     -> the other joins it if its rank has a free slot;
+ *   then experts still unplaced go, in ascending order, to the lowest rank
+ *   with a free slot.
+ * refine != 0: repeat the swap (a on P, b on Q, P != Q, a < b) of largest
+ *   gain  A[a][Q] - A[a][P] + A[b][P] - A[b][Q] - 2 W[a][b]
+ *   (A[e][d] = sum of W[e][e'] over e' != e on rank d), lowest (a, b) on
+ *   ties, while that gain is > 0, at most E*E swaps.
+ * W must be symmetric, as the co-selection count is.
+ */
+int oracle_place_correlated(const uint32_t *W, int E, int R, int seed_mode, int refine,
+                            int32_t *p)
+{
+    if (E < 1 || R < 1 || E % R != 0 || (seed_mode != 0 && seed_mode != 1)) return 1;
+    const int cap = E / R;
+
+    if (seed_mode == 0) {
+        for (int e = 0; e < E; ++e) p[e] = e / cap;
+    } else {
+        int *fill = (int *)calloc((size_t)R, sizeof(int));
+        int64_t np = 0;
+        pair_t *pairs = (pair_t *)malloc(sizeof(pair_t) * ((size_t)E * (E - 1) / 2 + 1));
+        if (!fill || !pairs) { free(fill); free(pairs); return 2; }
+        for (int e = 0; e < E; ++e) p[e] = -1;
+        for (int a = 0; a < E; ++a)
+            for (int b = a + 1; b < E; ++b)
+                if (W[(int64_t)a * E + b] > 0) {
+                    pairs[np].wv = W[(int64_t)a * E + b];
+                    pairs[np].a = a;
+                    pairs[np].b = b;
+                    ++np;
+                }
+        qsort(pairs, (size_t)np, sizeof(pair_t), cmp_pair);
+        for (int64_t i = 0; i < np; ++i) {
+            int a = pairs[i].a, b = pairs[i].b;
+            if (p[a] < 0 && p[b] < 0) {
+                int best = 0;
+                for (int d = 1; d < R; ++d)
+                    if (cap - fill[d] > cap - fill[best]) best = d;
+                if (cap - fill[best] >= 2) {
+                    p[a] = best;
+                    p[b] = best;
+                    fill[best] += 2;
+                }
+            } else if (p[a] >= 0 && p[b] < 0) {
+                if (fill[p[a]] < cap) { p[b] = p[a]; fill[p[a]] += 1; }
+            } else if (p[a] < 0 && p[b] >= 0) {
+                if (fill[p[b]] < cap) { p[a] = p[b]; fill[p[b]] += 1; }
+            }
+        }
+        for (int e = 0; e < E; ++e)
+            if (p[e] < 0)
+                for (int d = 0; d < R; ++d)
+                    if (fill[d] < cap) { p[e] = d; fill[d] += 1; break; }
+        free(fill);
+        free(pairs);
+    }
+    if (!refine) return 0;
+
+    long long *A = (long long *)malloc(sizeof(long long) * (size_t)E * R);
+    if (!A) return 2;
+    for (long long iter = 0; iter < (long long)E * E; ++iter) {
+        /* A[e][d] = sum of W[e][e'] over e' != e with p[e'] = d */
+        for (int64_t i = 0; i < (int64_t)E * R; ++i) A[i] = 0;
+        for (int e = 0; e < E; ++e)
+            for (int e2 = 0; e2 < E; ++e2)
+                if (e2 != e) A[(int64_t)e * R + p[e2]] += W[(int64_t)e * E + e2];
+        long long best_gain = 0;
+        int ba = -1, bb = -1;
+        for (int a = 0; a < E; ++a)
+            for (int b = a + 1; b < E; ++b) {
+                int P = p[a], Q = p[b];
+                if (P == Q) continue;
+                long long g = A[(int64_t)a * R + Q] - A[(int64_t)a * R + P] +
+                              A[(int64_t)b * R + P] - A[(int64_t)b * R + Q] -
+                              2LL * (long long)W[(int64_t)a * E + b];
+                if (g > best_gain) { best_gain = g; ba = a; bb = b; }
+            }
+        if (ba < 0) break;
+        int P = p[ba];
+        p[ba] = p[bb];
+        p[bb] = P;
+    }
+    free(A);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Token shuffle.                                                            */
+/* [EC] "Method 2: Token Shuffling", Mechanism: predict each token's owner   */
+/* rank at the next layer; every rank owns exactly T/EP tokens, so tokens    */
+/* are assigned in decreasing confidence to their most preferred rank with   */
+/* capacity left.  The single-expert form of the prediction is used: the     */
+/* token's top-1 expert e1 at layer l predicts the next-layer expert         */
+/* argmax_e' C[e1][e'].                                                      */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    uint64_t num, den;   /* confidence = num / den; den = 0 means zero */
+    int64_t t;
+} conf_t;
+
+/* decreasing confidence, then increasing token; a zero-count row has
+ * confidence 0 */
+static int cmp_conf(const void *x_, const void *y_)
+{
+    const conf_t *x = (const conf_t *)x_, *y = (const conf_t *)y_;
+    /* compare x.num/x.den with y.num/y.den exactly; 0/0 counts as 0 */
+    uint64_t xn = x->den ? x->num : 0, xd = x->den ? x->den : 1;
+    uint64_t yn = y->den ? y->num : 0, yd = y->den ? y->den : 1;
+    unsigned __int128 l = (unsigned __int128)xn * yd, r = (unsigned __int128)yn * xd;
+    if (l != r) return l > r ? -1 : 1;
+    return (x->t > y->t) - (x->t < y->t);
+}
+
+/*
+ * For each token t with top-1 expert e1 = idx_l[t*k]:
+ *   e*   = argmax_e' C[e1][e'] (lowest e' on ties); first choice p_next[e*];
+ *   then the other ranks by sigma(d) = sum_{e' : p_next[e'] = d} C[e1][e']
+ *   descending, lowest d on ties;
+ *   confidence = C[e1][e*] / sum_e' C[e1][e'].
+ *   A row of C that is all zero gives confidence 0 and the preference order
+ *   src(t), then the other ranks ascending.
+ * Tokens are visited by (confidence desc, t asc); each takes its first
+ * preferred rank that still has fewer than T/R tokens.
+ * pred_rank[t] = the rank t was assigned; rank d's tokens take the new
+ * positions d*T_r .. (d+1)*T_r - 1 in ascending t; perm[t] = new position,
+ * inv[perm[t]] = t.
+ */
+int oracle_token_shuffle(const int32_t *idx_l, const uint32_t *C, const int32_t *p_next,
+                         int64_t T, int E, int k, int R,
+                         int32_t *pred_rank, int32_t *perm, int32_t *inv)
+{
+    if (T < 0 || E < 1 || k < 1 || R < 1 || T % R != 0) return 1;
+    const int64_t Tr = T / R;
+    int32_t *pref = (int32_t *)malloc(sizeof(int32_t) * (size_t)E * R);
+    uint64_t *num = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)E);
+    uint64_t *den = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)E);
+    uint64_t *sigma = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)R);
+    conf_t *order = (conf_t *)malloc(sizeof(conf_t) * (size_t)(T > 0 ? T : 1));
+    int64_t *load = (int64_t *)calloc((size_t)R, sizeof(int64_t));
+    int rc = 0;
+    if (!pref || !num || !den || !sigma || !order || !load) { rc = 2; goto done; }
+
+    for (int e1 = 0; e1 < E; ++e1) {
+        const uint32_t *row = C + (int64_t)e1 * E;
+        uint64_t total = 0;
+        int best = 0;
+        for (int e = 0; e < E; ++e) {
+            total += row[e];
+            if (row[e] > row[best]) best = e;
+        }
+        num[e1] = row[best];
+        den[e1] = total;
+        for (int d = 0; d < R; ++d) sigma[d] = 0;
+        for (int e = 0; e < E; ++e) sigma[p_next[e]] += row[e];
+        int32_t *pl = pref + (int64_t)e1 * R;
+        pl[0] = p_next[best];
+        int n = 1;
+        /* remaining ranks, sigma descending, lowest rank on ties:
+         * selection by repeated scan */
+        while (n < R) {
+            int pick = -1;
+            for (int d = 0; d < R; ++d) {
+                int used = 0;
+                for (int i = 0; i < n; ++i)
+                    if (pl[i] == d) used = 1;
+                if (used) continue;
+                if (pick < 0 || sigma[d] > sigma[pick]) pick = d;
+            }
+            pl[n++] = pick;
+        }
+    }
+
+    for (int64_t t = 0; t < T; ++t) {
+        int e1 = idx_l[t * k];
+        if (e1 < 0 || e1 >= E) { rc = 1; goto done; }
+        order[t].num = num[e1];
+        order[t].den = den[e1];
+        order[t].t = t;
+    }
+    qsort(order, (size_t)T, sizeof(conf_t), cmp_conf);
+
+    for (int64_t i = 0; i < T; ++i) {
+        int64_t t = order[i].t;
+        int e1 = idx_l[t * k];
+        int chosen = -1;
+        if (den[e1] == 0) {
+            int s = (int)(t / Tr);
+            if (load[s] < Tr) chosen = s;
+            for (int d = 0; chosen < 0 && d < R; ++d)
+                if (load[d] < Tr) chosen = d;
+        } else {
+            const int32_t *pl = pref + (int64_t)e1 * R;
+            for (int n = 0; chosen < 0 && n < R; ++n)
+                if (load[pl[n]] < Tr) chosen = pl[n];
+        }
+        pred_rank[t] = chosen;
+        load[chosen] += 1;
+    }
+
+    for (int d = 0; d < R; ++d) load[d] = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        int d = pred_rank[t];
+        int64_t pos = (int64_t)d * Tr + load[d];
+        load[d] += 1;
+        perm[t] = (int32_t)pos;
+        inv[pos] = (int32_t)t;
+    }
+done:
+    free(pref); free(num); free(den); free(sigma); free(order); free(load);
+    return rc;
+}
