@@ -1,0 +1,428 @@
+"""Benchmark: MoE dispatch + combine throughput on B200.
+
+One step = one pass of the per-layer hot path over one batch:
+    md_route_topk -> md_dispatch_layout (dedup) -> md_dispatch_permute -> md_combine
+on the workload "zipf_pairs_e128_k8" (T=65536 tokens, hidden 2048 bf16, E=128,
+top-8, 16 virtual EP ranks, correlated Zipf(1.1) pair logits, contiguous
+placement).  Inputs are synthetic, seeded, resident in HBM, and larger than L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Under torchrun each rank runs an independent replica on its own GPU (the
+virtual EP ranks live inside one GPU; nothing is sharded), times K steps with
+CUDA events, and rank 0 prints one JSON line with the max over ranks.
+--impl reference times the CPU oracle on the host instead (bounded samples).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "dispatch+combine Mtokens/s at 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
+UNIT = "Mtokens/s"
+WORKLOAD = "zipf_pairs_e128_k8"
+FALLBACK_HBM_GBS = 6650.0
+CPU_TOKENS_PER_S_GUESS = 16000.0  # oracle, one core, this workload's shape
+
+
+# ------------------------------------------------------------- environment
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(ws, backend):
+    if ws <= 1:
+        return None
+    import datetime
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(dist, value: float, device) -> float:
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        dist.barrier(device_ids=[device.index] if device.type == "cuda" else None)
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.gpu_index = gpu_index
+        self.period_ms = period_ms
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------ bytes model
+
+def algorithmic_bytes(T, H, k, E, n_rows):
+    """Bytes each kernel must move (inputs read once, outputs written once)."""
+    return {
+        "route_topk": T * (4 * E + 8 * k),
+        "dispatch_layout": T * k * (4 + 8) + n_rows * 8,
+        "dispatch_permute": T * (2 * H + 4 * k) + n_rows * 2 * H,
+        "combine": T * (2 * H * (k + 1) + 12 * k),
+    }
+
+
+def kernel_traffic(name, launches_units, units_per_launch):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current source of the kernel; else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(name)
+    except Exception:
+        return None
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "combine_warp_top_router_b200", "csrc", rec["source"])
+    try:
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except Exception:
+        return None
+    if digest != rec.get("source_sha256_16"):
+        return None
+    return rec["dram_bytes_per_unit"] * units_per_launch
+
+
+# -------------------------------------------------------------- native arm
+
+def run_native(args):
+    import combine_warp_top_router_b200 as md
+    from combine_warp_top_router_b200 import synth
+
+    ws, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(ws, "nccl")
+    md.lib()  # fail loudly if the library is missing
+
+    w = synth.make_workload(WORKLOAD, seed=args.seed, device=device)
+    T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
+    mode = md.MD_DEDUP if args.dispatch == "dedup" else md.MD_CONV
+    stream = torch.cuda.Stream(device)
+    cap = T * k if mode == md.MD_CONV else T * min(k, R)
+    idx = torch.empty(T, k, dtype=torch.int32, device=device)
+    gates = torch.empty(T, k, dtype=torch.float32, device=device)
+    L = md.alloc_layout(T, E, k, R, mode, device)
+    wsp = md.alloc_workspace(md.dispatch_layout_workspace_size(T, E, k, R, mode), device)
+    buf = torch.empty(cap, H, dtype=torch.bfloat16, device=device)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+    status = md.new_status(device)
+    torch.cuda.synchronize()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        md.md_route_topk(w.logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp,
+                              dev_status=status, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        md.md_dispatch_permute(w.x, L.row_of_slot, out=buf, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+        md.md_combine(w.y, L.assign_row, idx, gates, out=out, stream=stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    stream.synchronize()
+    md.check_status(status, "layout status after warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    launches0 = md.launch_count()
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                step(events[i])
+        stream.synchronize()
+    launches = md.launch_count() - launches0
+    torch.cuda.synchronize()
+    barrier(dist, device)
+
+    total_ms = events[0][0].elapsed_time(events[-1][4])
+    per = {n: 0.0 for n in ("route_topk", "dispatch_layout", "dispatch_permute", "combine")}
+    for ev in events:
+        for j, n in enumerate(per):
+            per[n] += ev[j].elapsed_time(ev[j + 1])
+    per = {n: v / args.steps for n, v in per.items()}  # ms per launch
+    total_ms_max = max_over_ranks(dist, total_ms, device)
+    n_rows = int(L.n_rows.item())
+    md.check_status(status, "layout status")
+
+    # end to end through host buffers: inputs copied in, the result copied out
+    e2e = run_e2e(args, md, w, mode, device, stream, idx, gates, L, wsp, buf, status, dist)
+
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    peak = float(peaks["hbm_gbs"]) if peaks and "hbm_gbs" in peaks else FALLBACK_HBM_GBS
+    peak_src = "of measured" if peaks and "hbm_gbs" in peaks else "of fallback"
+    ab = algorithmic_bytes(T, H, k, E, n_rows)
+    kernels = {n: {"us": round(per[n] * 1e3, 2), "bytes": ab[n],
+                   "GBps": round(ab[n] / (per[n] * 1e-3) / 1e9, 1),
+                   "frac": round(ab[n] / (per[n] * 1e-3) / 1e9 / peak, 3)} for n in per}
+    dom = max(("dispatch_permute", "combine"), key=lambda n: per[n])
+    achieved = ab[dom] / (per[dom] * 1e-3) / 1e9
+    traffic = kernel_traffic(dom, args.steps, T)
+    value = T * args.steps * ws / (total_ms_max * 1e-3) / 1e6
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "T": T, "H": H, "E": E, "top_k": k, "ep_ranks": R,
+                   "dispatch": args.dispatch, "combine": "fused", "gates": "topk_softmax",
+                   "placement": "contiguous", "parallelism": f"replicas x{ws}",
+                   "l2": "not flushed: every step moves >2.6 GB through HBM, 20x the 126 MB L2",
+                   "dedup_rows_per_token": round(n_rows / T, 4)},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "peak_source": peak_src,
+                     "traffic": None if traffic is None else int(traffic),
+                     "algorithmic_bytes_per_launch": ab[dom]},
+        "kernels": kernels,
+        "gpu_launches": int(launches),
+        "e2e": e2e,
+        "clocks": clk.summary(),
+    }
+    line["cpu_baseline"] = cpu_baseline(args)
+    return line
+
+
+def run_e2e(args, md, w, mode, device, stream, idx, gates, L, wsp, buf, status, dist):
+    """Same step through host buffers: pinned inputs -> HBM, path, result -> host."""
+    T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
+    h_logits = w.logits.cpu().pin_memory()
+    h_x = w.x.cpu().pin_memory()
+    h_y = w.y.cpu().pin_memory()
+    h_out = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    d_logits = torch.empty_like(w.logits)
+    d_x = torch.empty_like(w.x)
+    d_y = torch.empty_like(w.y)
+    d_out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+    steps = max(1, min(args.steps, args.e2e_steps))
+
+    def step():
+        d_logits.copy_(h_logits, non_blocking=True)
+        d_x.copy_(h_x, non_blocking=True)
+        d_y.copy_(h_y, non_blocking=True)
+        md.md_route_topk(d_logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream)
+        md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp,
+                              dev_status=status, stream=stream)
+        md.md_dispatch_permute(d_x, L.row_of_slot, out=buf, stream=stream)
+        md.md_combine(d_y, L.assign_row, idx, gates, out=d_out, stream=stream)
+        h_out.copy_(d_out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    barrier(dist, device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    ms = max_over_ranks(dist, e0.elapsed_time(e1), device)
+    ws = dist.get_world_size() if dist is not None else 1
+    h2d = (h_logits.numel() * 4 + h_x.numel() * 2 + h_y.numel() * 2)
+    return {"value": round(T * steps * ws / (ms * 1e-3) / 1e6, 4), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(h_out.numel() * 2),
+            "steps": steps, "note": "pinned host buffers; copies on the compute stream"}
+
+
+# -------------------------------------------------------- oracle (CPU) arm
+
+def oracle_sample(T_s, seed):
+    """Inputs for a T_s-token sample of the workload (same recipe, E, k, R, H)."""
+    from combine_warp_top_router_b200 import synth
+    w = synth.make_workload(WORKLOAD, seed=seed, device="cpu", T=T_s)
+    bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    return (w.logits.numpy(), bits(w.x), bits(w.y), w.expert_to_rank.numpy(), w.E, w.k, w.R)
+
+
+def oracle_step(oracle, inp, dedup=True):
+    lg, x, y, p, E, k, R = inp
+    idx, g = oracle.route_topk(lg, k)
+    L = oracle.dispatch_layout(idx, E, R, p, 1 if dedup else 0)
+    oracle.dispatch_permute(x, L["row_token"])
+    oracle.combine(y, L["assign_row"], idx, g)
+
+
+def cpu_baseline(args):
+    import oracle
+    oracle.build()
+    T_s = args.cpu_sample_tokens
+    inp = oracle_sample(T_s, args.seed)
+    oracle_step(oracle, oracle_sample(256, args.seed + 1))  # load the library
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle_step(oracle, inp, args.dispatch == "dedup")
+        reps += 1
+        if time.perf_counter() - t0 >= args.cpu_seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(T_s * reps / dt / 1e6, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{reps} x {T_s}-token sample of the same workload recipe "
+                      f"(E=128, top-8, 16 ranks, H=2048), single-threaded C oracle, "
+                      f"{dt:.1f} s", "host_cores": os.cpu_count()}
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    R = 16
+    # bound the run to about a minute of CPU for K + W steps
+    per_step = 60.0 / max(1, args.steps + args.warmup)
+    T_s = int(per_step * CPU_TOKENS_PER_S_GUESS) // R * R
+    T_s = max(R, min(65536, T_s))
+    inp = oracle_sample(T_s, args.seed)
+    for _ in range(args.warmup):
+        oracle_step(oracle, inp, args.dispatch == "dedup")
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(oracle, inp, args.dispatch == "dedup")
+    dt = time.perf_counter() - t0
+    value = T_s * args.steps / dt / 1e6
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT,
+        "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "T": T_s, "H": 2048, "E": 128, "top_k": 8, "ep_ranks": R,
+                   "dispatch": args.dispatch, "combine": "fused",
+                   "note": "each step is a bounded sample of the workload"},
+        "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"{T_s}-token sample per step"},
+        "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--dispatch", choices=["dedup", "conv"], default="dedup")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=32768)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    line = run_reference(args) if args.impl == "reference" else run_native(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    ws, _, _ = dist_env()
+    if ws > 1 and args.impl == "native":
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,12 @@
+"""B200-native MoE token dispatch / combine for expert parallelism.
+
+The compute lives in libmoedispatch.so (hand-written sm_100a CUDA kernels
+behind the C ABI in include/moedispatch.h).  `binding` is a thin ctypes layer
+with the same entry-point names; `synth` draws seeded synthetic inputs.
+"""
+from .binding import *  # noqa: F401,F403
+from .binding import Layout, MoeDispatchError, check_status, lib, new_status  # noqa: F401
+from . import synth  # noqa: F401
+
+__all__ = [n for n in dir() if n.startswith("md_") or n.startswith("MD_")] + [
+    "Layout", "MoeDispatchError", "check_status", "lib", "new_status", "synth"]

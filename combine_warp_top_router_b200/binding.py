@@ -1,0 +1,321 @@
+"""Thin ctypes binding of libmoedispatch (include/moedispatch.h).
+
+Argument marshalling only: every function checks tensor placement, dtype and
+contiguity, allocates outputs with torch when the caller passes none, and calls
+the C entry point of the same name on the current CUDA stream.  All arithmetic
+runs in the library's kernels.  If libmoedispatch.so is missing the first call
+raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoedispatch.so")
+
+MD_OK, MD_ERR_ARG, MD_ERR_UNSUPPORTED, MD_ERR_CUDA = 0, 1, 2, 3
+MD_ERR_WORKSPACE, MD_ERR_DATA, MD_ERR_TIMEOUT = 4, 5, 6
+MD_CONV, MD_DEDUP = 0, 1
+MD_GATE_TOPK_SOFTMAX, MD_GATE_FULL_SOFTMAX = 0, 1
+MD_COMBINE_FUSED, MD_COMBINE_WIRE = 0, 1
+MD_SEED_CONTIGUOUS, MD_SEED_GREEDY_PAIRS = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+_P, _I, _L, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+_SIGNATURES = {
+    "md_status_string": ([_I], ctypes.c_char_p),
+    "md_version": ([], _I),
+    "md_launch_count": ([], ctypes.c_uint64),
+    "md_route_topk": ([_P, _L, _I, _I, _I, _P, _P, _P], _I),
+    "md_dispatch_layout_workspace_size": ([_L, _I, _I, _I, _I], _S),
+    "md_dispatch_layout": ([_P, _L, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                            _P, _S, _P, _P], _I),
+    "md_dispatch_permute": ([_P, _L, _I, _I, _P, _L, _P, _P, _P], _I),
+    "md_combine": ([_P, _L, _P, _P, _P, _L, _I, _I, _I, _P, _L, _P, _P, _P, _P], _I),
+    "md_coselect_stats": ([_P, _P, _L, _I, _I, _P, _P, _I, _P, _P], _I),
+    "md_place_correlated_workspace_size": ([_I, _I], _S),
+    "md_place_correlated": ([_P, _I, _I, _I, _I, _P, _P, _S, _P, _P], _I),
+    "md_token_shuffle_workspace_size": ([_L, _I, _I], _S),
+    "md_token_shuffle": ([_P, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _S, _P, _P], _I),
+    "md_gather_rows": ([_P, _L, _L, _P, _L, _P, _P, _P], _I),
+}
+
+
+class MoeDispatchError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)}")
+        self.code = code
+
+
+def lib():
+    """The loaded libmoedispatch.so; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m combine_warp_top_router_b200.build` (there is no CPU fallback)")
+            h = ctypes.CDLL(LIB_PATH)
+            for name, (args, res) in _SIGNATURES.items():
+                fn = getattr(h, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = h
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().md_status_string(int(code)).decode()
+
+
+def launch_count() -> int:
+    return int(lib().md_launch_count())
+
+
+def _check(rc: int, what: str):
+    if rc != MD_OK:
+        raise MoeDispatchError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    return t
+
+
+def new_status(device) -> torch.Tensor:
+    """A device status word for the dev_status arguments."""
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check_status(dev_status: torch.Tensor, what: str = "device status"):
+    """Synchronise on the status word and raise if a kernel reported an error."""
+    code = int(dev_status.item())
+    if code != MD_OK:
+        raise MoeDispatchError(code, what)
+
+
+# ------------------------------------------------------------------ router
+
+def md_route_topk(logits, k, gate_mode=MD_GATE_TOPK_SOFTMAX, topk_idx=None, topk_w=None,
+                  stream=None):
+    _need(logits, "logits", torch.float32)
+    T, E = logits.shape
+    dev = logits.device
+    if topk_idx is None:
+        topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _need(topk_w, "topk_w", torch.float32, dev)
+    rc = lib().md_route_topk(_ptr(logits), T, E, k, gate_mode, _ptr(topk_idx), _ptr(topk_w),
+                             _stream(stream, dev))
+    _check(rc, "md_route_topk")
+    return topk_idx, topk_w
+
+
+# ------------------------------------------------------------------ layout
+
+@dataclass
+class Layout:
+    """Outputs of md_dispatch_layout (device tensors)."""
+    mode: int
+    row_of_slot: torch.Tensor   # int32 [T, k]
+    assign_row: torch.Tensor    # int32 [T, k]
+    row_token: torch.Tensor     # int32 [row capacity]
+    row_mask: torch.Tensor      # int32 [row capacity] (uint32 bit patterns)
+    send_counts: torch.Tensor   # int32 [R, R]
+    expert_counts: torch.Tensor  # int32 [E]
+    expert_offsets: torch.Tensor  # int32 [E+1]
+    rank_offsets: torch.Tensor  # int32 [R+1]
+    n_rows: torch.Tensor        # int32 [1]
+    row_capacity: int
+
+
+def dispatch_layout_workspace_size(T, E, k, R, mode) -> int:
+    return int(lib().md_dispatch_layout_workspace_size(T, E, k, R, mode))
+
+
+def alloc_layout(T, E, k, R, mode, device) -> Layout:
+    cap = T * k if mode == MD_CONV else T * min(k, R)
+    i32 = dict(dtype=torch.int32, device=device)
+    return Layout(mode=mode, row_of_slot=torch.empty(T, k, **i32),
+                  assign_row=torch.empty(T, k, **i32), row_token=torch.empty(max(cap, 1), **i32),
+                  row_mask=torch.empty(max(cap, 1), **i32), send_counts=torch.empty(R, R, **i32),
+                  expert_counts=torch.empty(E, **i32), expert_offsets=torch.empty(E + 1, **i32),
+                  rank_offsets=torch.empty(R + 1, **i32), n_rows=torch.empty(1, **i32),
+                  row_capacity=cap)
+
+
+def alloc_workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def md_dispatch_layout(topk_idx, E, R, expert_to_rank, mode, out: Layout | None = None,
+                       workspace=None, dev_status=None, stream=None) -> Layout:
+    _need(topk_idx, "topk_idx", torch.int32)
+    dev = topk_idx.device
+    _need(expert_to_rank, "expert_to_rank", torch.int32, dev)
+    T, k = topk_idx.shape
+    if out is None:
+        out = alloc_layout(T, E, k, R, mode, dev)
+    need = dispatch_layout_workspace_size(T, E, k, R, mode)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    rc = lib().md_dispatch_layout(
+        _ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), mode, _ptr(out.row_of_slot),
+        _ptr(out.assign_row), _ptr(out.row_token), _ptr(out.row_mask), _ptr(out.send_counts),
+        _ptr(out.expert_counts), _ptr(out.expert_offsets), _ptr(out.rank_offsets),
+        _ptr(out.n_rows), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+        _stream(stream, dev))
+    _check(rc, "md_dispatch_layout")
+    return out
+
+
+# --------------------------------------------------------- permute/combine
+
+def md_dispatch_permute(x, row_of_slot, out_rows=None, out=None, dev_status=None, stream=None):
+    _need(x, "x", torch.bfloat16)
+    dev = x.device
+    _need(row_of_slot, "row_of_slot", torch.int32, dev)
+    T, H = x.shape
+    k = row_of_slot.shape[1]
+    if out is None:
+        out = torch.empty(out_rows if out_rows is not None else T * k, H, dtype=torch.bfloat16,
+                          device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    rc = lib().md_dispatch_permute(_ptr(x), T, H, k, _ptr(row_of_slot), out.shape[0], _ptr(out),
+                                   _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_dispatch_permute")
+    return out
+
+
+def md_combine(y, assign_row, topk_idx, topk_w, mode=MD_COMBINE_FUSED, row_of_slot=None, z=None,
+               out=None, dev_status=None, stream=None):
+    _need(y, "y", torch.bfloat16)
+    dev = y.device
+    _need(assign_row, "assign_row", torch.int32, dev)
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    _need(topk_w, "topk_w", torch.float32, dev)
+    T, k = topk_idx.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    z_rows = 0
+    if mode == MD_COMBINE_WIRE:
+        _need(row_of_slot, "row_of_slot", torch.int32, dev)
+        _need(z, "z", torch.bfloat16, dev)
+        z_rows = z.shape[0]
+    rc = lib().md_combine(_ptr(y), y.shape[0], _ptr(assign_row), _ptr(topk_idx), _ptr(topk_w), T,
+                          k, H, mode, _ptr(row_of_slot), z_rows, _ptr(z), _ptr(out),
+                          _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_combine")
+    return out
+
+
+def md_gather_rows(src, index, out=None, dev_status=None, stream=None):
+    if not src.is_cuda or not src.is_contiguous():
+        raise ValueError("src must be a contiguous CUDA tensor")
+    dev = src.device
+    _need(index, "index", torch.int32, dev)
+    n = index.shape[0]
+    if out is None:
+        out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=dev)
+    if out.dtype != src.dtype or not out.is_contiguous():
+        raise ValueError("out must be contiguous and of src's dtype")
+    row_bytes = src[0].numel() * src.element_size() if src.shape[0] else \
+        out[0].numel() * out.element_size()
+    rc = lib().md_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out),
+                              _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_gather_rows")
+    return out
+
+
+# --------------------------------------------------- statistics / planning
+
+def md_coselect_stats(idx_l, idx_next, E, T_fit=None, W=None, C=None, accumulate=False,
+                      want_W=True, want_C=True, dev_status=None, stream=None):
+    _need(idx_l, "idx_l", torch.int32)
+    dev = idx_l.device
+    T, k = idx_l.shape
+    T_fit = T if T_fit is None else T_fit
+    if idx_next is not None:
+        _need(idx_next, "idx_next", torch.int32, dev)
+    if W is None and want_W:
+        W = torch.empty(E, E, dtype=torch.int32, device=dev)
+    if C is None and want_C and idx_next is not None:
+        C = torch.empty(E, E, dtype=torch.int32, device=dev)
+    for t, n in ((W, "W"), (C, "C")):
+        if t is not None:
+            _need(t, n, torch.int32, dev)
+    rc = lib().md_coselect_stats(_ptr(idx_l), _ptr(idx_next), T_fit, E, k, _ptr(W), _ptr(C),
+                                 1 if accumulate else 0, _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_coselect_stats")
+    return W, C
+
+
+def md_place_correlated(W, R, seed_mode=MD_SEED_CONTIGUOUS, refine=True, out=None,
+                        workspace=None, dev_status=None, stream=None):
+    _need(W, "W", torch.int32)
+    dev = W.device
+    E = W.shape[0]
+    if out is None:
+        out = torch.empty(E, dtype=torch.int32, device=dev)
+    need = int(lib().md_place_correlated_workspace_size(E, R))
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    rc = lib().md_place_correlated(_ptr(W), E, R, seed_mode, 1 if refine else 0, _ptr(out),
+                                   _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                   _stream(stream, dev))
+    _check(rc, "md_place_correlated")
+    return out
+
+
+def md_token_shuffle(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None, inv=None,
+                     workspace=None, dev_status=None, stream=None):
+    _need(idx_l, "idx_l", torch.int32)
+    dev = idx_l.device
+    _need(C, "C", torch.int32, dev)
+    _need(expert_to_rank_next, "expert_to_rank_next", torch.int32, dev)
+    T, k = idx_l.shape
+    E = C.shape[0]
+    i32 = dict(dtype=torch.int32, device=dev)
+    pred_rank = torch.empty(T, **i32) if pred_rank is None else pred_rank
+    perm = torch.empty(T, **i32) if perm is None else perm
+    inv = torch.empty(T, **i32) if inv is None else inv
+    need = int(lib().md_token_shuffle_workspace_size(T, E, R))
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    rc = lib().md_token_shuffle(_ptr(idx_l), k, _ptr(C), _ptr(expert_to_rank_next), T, E, R,
+                                _ptr(pred_rank), _ptr(perm), _ptr(inv), _ptr(workspace),
+                                workspace.numel(), _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_token_shuffle")
+    return pred_rank, perm, inv

@@ -1,0 +1,27 @@
+// api.cu -- status strings, version and launch accounting of libmoedispatch.
+#include <atomic>
+
+#include "common.cuh"
+
+namespace md {
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+}  // namespace md
+
+extern "C" const char *md_status_string(int status)
+{
+    switch (status) {
+    case MD_OK: return "MD_OK";
+    case MD_ERR_ARG: return "MD_ERR_ARG: invalid argument";
+    case MD_ERR_UNSUPPORTED: return "MD_ERR_UNSUPPORTED: size outside the supported limits";
+    case MD_ERR_CUDA: return "MD_ERR_CUDA: a CUDA launch or memset failed";
+    case MD_ERR_WORKSPACE: return "MD_ERR_WORKSPACE: workspace too small";
+    case MD_ERR_DATA: return "MD_ERR_DATA: invalid index, placement or row in the input data";
+    case MD_ERR_TIMEOUT: return "MD_ERR_TIMEOUT: a bounded device-side wait ran out";
+    default: return "unknown md_status";
+    }
+}
+
+extern "C" int md_version(void) { return 100; }
+
+extern "C" uint64_t md_launch_count(void) { return md::g_launches.load(std::memory_order_relaxed); }

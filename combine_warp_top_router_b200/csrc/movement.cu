@@ -1,0 +1,334 @@
+// movement.cu -- row movement on HBM: dispatch permute, combine, row gather
+// (md_dispatch_permute, md_combine, md_gather_rows).
+//
+// All three are bound by HBM bandwidth.  Rows are moved as 16-byte vectors,
+// one 16-byte column chunk per thread, so every warp reads or writes 512
+// contiguous bytes of a row.  A CTA works on a group of kGroup tokens at a
+// time: it first stages the group's row indices (and, for combine, the slot
+// order and gates) in shared memory, then each thread issues all loads of
+// its column chunk for the group before any store, so kGroup (permute) or k
+// (combine) 16-byte loads per thread are in flight.  Grids are a multiple of
+// the SM count and loop over token groups.
+#include <climits>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kGroup = 8;  // tokens per CTA iteration (one warp per token when sorting)
+
+int grid_for(int64_t units, int per_block)
+{
+    int64_t b = (units + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)md::sm_count() * 8;
+    if (b > cap) b = cap;
+    return b < 1 ? 1 : (int)b;
+}
+
+// ----------------------------------------------------------------- permute
+// out[row_of_slot[t][j]] = x[t] for every distinct row of token t.
+template <int KC>
+__global__ void __launch_bounds__(kThreads)
+    k_permute(const uint4 *__restrict__ x, int64_t T, int C, int k,
+              const int32_t *__restrict__ row_of_slot, int64_t out_rows, uint4 *__restrict__ out,
+              int32_t *status)
+{
+    __shared__ int s_row[kGroup][MD_MAX_TOPK];
+    const int K = KC ? KC : k;
+    for (int64_t g0 = (int64_t)blockIdx.x * kGroup; g0 < T; g0 += (int64_t)gridDim.x * kGroup) {
+        const int ng = (int)(T - g0 < kGroup ? T - g0 : kGroup);
+        for (int i = threadIdx.x; i < ng * K; i += kThreads) {
+            const int g = i / K, j = i - g * K;
+            const int32_t *rr = row_of_slot + (g0 + g) * K;
+            int r = rr[j];
+            bool dup = false;
+            for (int j2 = 0; j2 < j; ++j2)
+                if (__ldg(rr + j2) == r) dup = true;
+            if (!dup && (r < 0 || r >= out_rows)) {
+                md::report(status, MD_ERR_DATA);
+                r = -1;
+            }
+            s_row[g][j] = dup ? -1 : r;
+        }
+        __syncthreads();
+        for (int c = threadIdx.x; c < C; c += kThreads) {
+            uint4 v[kGroup];
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g)
+                if (g < ng) v[g] = md::ld_stream(x + (g0 + g) * C + c);
+#pragma unroll
+            for (int g = 0; g < kGroup; ++g) {
+                if (g < ng) {
+#pragma unroll 8
+                    for (int j = 0; j < K; ++j) {
+                        const int r = s_row[g][j];
+                        if (r >= 0) md::st_stream(out + (int64_t)r * C + c, v[g]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ----------------------------------------------------------------- combine
+__device__ __forceinline__ void fma_row(float (&acc)[8], float w, const uint4 &v)
+{
+    acc[0] = fmaf(w, md::bf16lo(v.x), acc[0]);
+    acc[1] = fmaf(w, md::bf16hi(v.x), acc[1]);
+    acc[2] = fmaf(w, md::bf16lo(v.y), acc[2]);
+    acc[3] = fmaf(w, md::bf16hi(v.y), acc[3]);
+    acc[4] = fmaf(w, md::bf16lo(v.z), acc[4]);
+    acc[5] = fmaf(w, md::bf16hi(v.z), acc[5]);
+    acc[6] = fmaf(w, md::bf16lo(v.w), acc[6]);
+    acc[7] = fmaf(w, md::bf16hi(v.w), acc[7]);
+}
+
+__device__ __forceinline__ uint4 pack_row(const float (&a)[8])
+{
+    return make_uint4(md::pack_bf16x2(a[0], a[1]), md::pack_bf16x2(a[2], a[3]),
+                      md::pack_bf16x2(a[4], a[5]), md::pack_bf16x2(a[6], a[7]));
+}
+
+// FUSED: out[t] = bf16(sum over slots by ascending expert of w * y), fp32 FMA.
+// WIRE:  slots sorted by (wire row, expert); each run of one wire row is
+//        summed, rounded to bf16 and stored in z; out[t] = bf16(fp32 sum of
+//        those bf16 partials in wire-row order).
+template <int KC, bool WIRE>
+__global__ void __launch_bounds__(kThreads)
+    k_combine(const uint4 *__restrict__ y, int64_t y_rows, const int32_t *__restrict__ assign_row,
+              const int32_t *__restrict__ idx, const float *__restrict__ w, int64_t T, int k, int C,
+              const int32_t *__restrict__ row_of_slot, int64_t z_rows, uint4 *__restrict__ z,
+              uint4 *__restrict__ out, int32_t *status)
+{
+    __shared__ int s_r[kGroup][MD_MAX_TOPK];
+    __shared__ float s_w[kGroup][MD_MAX_TOPK];
+    __shared__ int s_z[kGroup][WIRE ? MD_MAX_TOPK : 1];
+    const int K = KC ? KC : k;
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+
+    for (int64_t g0 = (int64_t)blockIdx.x * kGroup; g0 < T; g0 += (int64_t)gridDim.x * kGroup) {
+        const int ng = (int)(T - g0 < kGroup ? T - g0 : kGroup);
+        // warp wp orders the slots of token g0 + wp
+        if (wp < ng) {
+            const int64_t t = g0 + wp;
+            const bool live = lane < K;
+            const int e = live ? idx[t * K + lane] : INT_MAX;
+            int r = live ? assign_row[t * K + lane] : -1;
+            const float ww = live ? w[t * K + lane] : 0.0f;
+            int zr = (WIRE && live) ? row_of_slot[t * K + lane] : 0;
+            int rank = 0;
+            for (int j = 0; j < K; ++j) {
+                const int ej = __shfl_sync(0xffffffffu, e, j);
+                const int zj = WIRE ? __shfl_sync(0xffffffffu, zr, j) : 0;
+                bool before = ej < e || (ej == e && j < lane);
+                if (WIRE) before = zj < zr || (zj == zr && before);
+                rank += before ? 1 : 0;
+            }
+            if (live) {
+                if (r < 0 || r >= y_rows) {
+                    md::report(status, MD_ERR_DATA);
+                    r = -1;
+                }
+                if (WIRE && (zr < 0 || zr >= z_rows)) {
+                    md::report(status, MD_ERR_DATA);
+                    zr = -1;
+                }
+                s_r[wp][rank] = r;
+                s_w[wp][rank] = ww;
+                if (WIRE) s_z[wp][rank] = zr;
+            }
+        }
+        __syncthreads();
+        for (int g = 0; g < ng; ++g) {
+            const int64_t t = g0 + g;
+            for (int c = threadIdx.x; c < C; c += kThreads) {
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                float tot[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                constexpr int B = KC ? KC : 4;  // loads issued together
+                for (int j0 = 0; j0 < K; j0 += B) {
+                    uint4 v[B];
+#pragma unroll
+                    for (int q = 0; q < B; ++q) {
+                        const int j = j0 + q;
+                        const int r = j < K ? s_r[g][j] : -1;
+                        v[q] = r >= 0 ? md::ld_stream(y + (int64_t)r * C + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int q = 0; q < B; ++q) {
+                        const int j = j0 + q;
+                        if (j >= K) break;
+                        if (s_r[g][j] >= 0) fma_row(acc, s_w[g][j], v[q]);
+                        if (WIRE && (j == K - 1 || s_z[g][j + 1] != s_z[g][j])) {
+                            const uint4 zb = pack_row(acc);
+                            const int zr = s_z[g][j];
+                            if (zr >= 0) md::st_stream(z + (int64_t)zr * C + c, zb);
+                            tot[0] += md::bf16lo(zb.x);
+                            tot[1] += md::bf16hi(zb.x);
+                            tot[2] += md::bf16lo(zb.y);
+                            tot[3] += md::bf16hi(zb.y);
+                            tot[4] += md::bf16lo(zb.z);
+                            tot[5] += md::bf16hi(zb.z);
+                            tot[6] += md::bf16lo(zb.w);
+                            tot[7] += md::bf16hi(zb.w);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+                        }
+                    }
+                }
+                md::st_stream(out + t * C + c, pack_row(WIRE ? tot : acc));
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------ gather
+__global__ void __launch_bounds__(kThreads)
+    k_gather16(const uint4 *__restrict__ src, int64_t src_rows, int C,
+               const int32_t *__restrict__ index, int64_t n_out, uint4 *__restrict__ dst,
+               int32_t *status)
+{
+    const int64_t n = n_out * C;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * kThreads) {
+        const int64_t row = i / C;
+        const int c = (int)(i - row * C);
+        const int s = __ldg(index + row);
+        if (s < 0 || s >= src_rows) {
+            if (c == 0) md::report(status, MD_ERR_DATA);
+            continue;
+        }
+        md::st_stream(dst + i, md::ld_stream(src + (int64_t)s * C + c));
+    }
+}
+
+__global__ void __launch_bounds__(kThreads)
+    k_gather4(const uint32_t *__restrict__ src, int64_t src_rows, int C,
+              const int32_t *__restrict__ index, int64_t n_out, uint32_t *__restrict__ dst,
+              int32_t *status)
+{
+    const int64_t n = n_out * C;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * kThreads) {
+        const int64_t row = i / C;
+        const int c = (int)(i - row * C);
+        const int s = __ldg(index + row);
+        if (s < 0 || s >= src_rows) {
+            if (c == 0) md::report(status, MD_ERR_DATA);
+            continue;
+        }
+        dst[i] = __ldg(src + (int64_t)s * C + c);
+    }
+}
+
+template <int KC>
+void launch_permute(const void *x, int64_t T, int C, int k, const int32_t *rs, int64_t rows,
+                    void *out, int32_t *st, cudaStream_t s)
+{
+    k_permute<KC><<<grid_for(T, kGroup), kThreads, 0, s>>>(
+        static_cast<const uint4 *>(x), T, C, k, rs, rows, static_cast<uint4 *>(out), st);
+}
+
+template <int KC, bool WIRE>
+void launch_combine(const void *y, int64_t y_rows, const int32_t *ar, const int32_t *idx,
+                    const float *w, int64_t T, int k, int C, const int32_t *rs, int64_t z_rows,
+                    void *z, void *out, int32_t *st, cudaStream_t s)
+{
+    k_combine<KC, WIRE><<<grid_for(T, kGroup), kThreads, 0, s>>>(
+        static_cast<const uint4 *>(y), y_rows, ar, idx, w, T, k, C, rs, z_rows,
+        static_cast<uint4 *>(z), static_cast<uint4 *>(out), st);
+}
+
+template <bool WIRE>
+void dispatch_combine(const void *y, int64_t y_rows, const int32_t *ar, const int32_t *idx,
+                      const float *w, int64_t T, int k, int C, const int32_t *rs, int64_t z_rows,
+                      void *z, void *out, int32_t *st, cudaStream_t s)
+{
+    switch (k) {
+    case 1: launch_combine<1, WIRE>(y, y_rows, ar, idx, w, T, k, C, rs, z_rows, z, out, st, s); break;
+    case 2: launch_combine<2, WIRE>(y, y_rows, ar, idx, w, T, k, C, rs, z_rows, z, out, st, s); break;
+    case 4: launch_combine<4, WIRE>(y, y_rows, ar, idx, w, T, k, C, rs, z_rows, z, out, st, s); break;
+    case 6: launch_combine<6, WIRE>(y, y_rows, ar, idx, w, T, k, C, rs, z_rows, z, out, st, s); break;
+    case 8: launch_combine<8, WIRE>(y, y_rows, ar, idx, w, T, k, C, rs, z_rows, z, out, st, s); break;
+    default: launch_combine<0, WIRE>(y, y_rows, ar, idx, w, T, k, C, rs, z_rows, z, out, st, s); break;
+    }
+}
+
+}  // namespace
+
+extern "C" int md_dispatch_permute(const void *x, int64_t T, int H, int k,
+                                   const int32_t *row_of_slot, int64_t out_rows, void *out,
+                                   int32_t *dev_status, void *stream)
+{
+    if (T < 0 || H < 8 || H % 8 != 0 || k < 1 || k > MD_MAX_TOPK || out_rows < 0) return MD_ERR_ARG;
+    if (T > 0 && (!x || !row_of_slot || !md::aligned16(x))) return MD_ERR_ARG;
+    if (out_rows > 0 && (!out || !md::aligned16(out))) return MD_ERR_ARG;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK || T == 0) return rc;
+    const int C = H / 8;
+    switch (k) {
+    case 1: launch_permute<1>(x, T, C, k, row_of_slot, out_rows, out, dev_status, s); break;
+    case 2: launch_permute<2>(x, T, C, k, row_of_slot, out_rows, out, dev_status, s); break;
+    case 4: launch_permute<4>(x, T, C, k, row_of_slot, out_rows, out, dev_status, s); break;
+    case 6: launch_permute<6>(x, T, C, k, row_of_slot, out_rows, out, dev_status, s); break;
+    case 8: launch_permute<8>(x, T, C, k, row_of_slot, out_rows, out, dev_status, s); break;
+    default: launch_permute<0>(x, T, C, k, row_of_slot, out_rows, out, dev_status, s); break;
+    }
+    md::count_launches(1);
+    return md::launch_status();
+}
+
+extern "C" int md_combine(const void *y, int64_t y_rows, const int32_t *assign_row,
+                          const int32_t *topk_idx, const float *topk_w, int64_t T, int k, int H,
+                          int combine_mode, const int32_t *row_of_slot, int64_t z_rows, void *z,
+                          void *out, int32_t *dev_status, void *stream)
+{
+    if (T < 0 || H < 8 || H % 8 != 0 || k < 1 || k > MD_MAX_TOPK || y_rows < 0) return MD_ERR_ARG;
+    if (combine_mode != MD_COMBINE_FUSED && combine_mode != MD_COMBINE_WIRE) return MD_ERR_ARG;
+    if (T > 0 && (!assign_row || !topk_idx || !topk_w || !out || !md::aligned16(out)))
+        return MD_ERR_ARG;
+    if (y_rows > 0 && (!y || !md::aligned16(y))) return MD_ERR_ARG;
+    const bool wire = combine_mode == MD_COMBINE_WIRE;
+    if (wire && T > 0 && (!row_of_slot || z_rows < 0 || (z_rows > 0 && (!z || !md::aligned16(z)))))
+        return MD_ERR_ARG;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK || T == 0) return rc;
+    const int C = H / 8;
+    if (wire)
+        dispatch_combine<true>(y, y_rows, assign_row, topk_idx, topk_w, T, k, C, row_of_slot,
+                               z_rows, z, out, dev_status, s);
+    else
+        dispatch_combine<false>(y, y_rows, assign_row, topk_idx, topk_w, T, k, C, nullptr, 0,
+                                nullptr, out, dev_status, s);
+    md::count_launches(1);
+    return md::launch_status();
+}
+
+extern "C" int md_gather_rows(const void *src, int64_t src_rows, int64_t row_bytes,
+                              const int32_t *index, int64_t n_out, void *dst, int32_t *dev_status,
+                              void *stream)
+{
+    if (src_rows < 0 || n_out < 0 || row_bytes < 4 || row_bytes % 4 != 0) return MD_ERR_ARG;
+    if (n_out > 0 && (!index || !dst)) return MD_ERR_ARG;
+    if (src_rows > 0 && !src) return MD_ERR_ARG;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK || n_out == 0) return rc;
+    if (row_bytes % 16 == 0 && md::aligned16(src) && md::aligned16(dst)) {
+        const int C = (int)(row_bytes / 16);
+        k_gather16<<<grid_for(n_out * C, kThreads * 4), kThreads, 0, s>>>(
+            static_cast<const uint4 *>(src), src_rows, C, index, n_out, static_cast<uint4 *>(dst),
+            dev_status);
+    } else {
+        const int C = (int)(row_bytes / 4);
+        k_gather4<<<grid_for(n_out * C, kThreads * 4), kThreads, 0, s>>>(
+            static_cast<const uint32_t *>(src), src_rows, C, index, n_out,
+            static_cast<uint32_t *>(dst), dev_status);
+    }
+    md::count_launches(1);
+    return md::launch_status();
+}

@@ -1,0 +1,372 @@
+// shuffle.cu -- capacity-constrained token shuffle (md_token_shuffle).
+//
+// "Expert Coupling in MoE Pretraining" (PicX summary), Method 2 (Token
+// Shuffling), Mechanism: the planner predicts each token's owner rank at layer
+// l+1; every rank must own exactly T/EP tokens, so tokens are assigned in
+// decreasing confidence to their most preferred rank with capacity left.
+// Single-expert prediction from the layer-l top-1 expert e1: first choice
+// p_next[argmax_e' C[e1][e']], then the other ranks by their share of row e1.
+//
+// Everything a token needs depends only on e1, so it is computed per expert:
+//   k_shuf_prefs    one CTA per expert row: row sum, arg-max, per-rank sums,
+//                   preference list, confidence numerator / denominator.
+//   k_shuf_class    class[e] = number of experts with strictly larger
+//                   confidence (exact 128-bit cross products); empty rows
+//                   get class E.  Equal confidences share a class.
+//   bucket sort     stable counting sort of the tokens by class (so tokens
+//                   are visited by confidence desc, t asc): per-tile
+//                   histograms, a column scan, and a one-warp-per-tile
+//                   stable scatter using __match_any_sync.
+//   k_shuf_greedy   one CTA walks the sorted tokens 1024 at a time.  Each
+//                   token takes its first preferred rank that is not full.
+//                   Within a chunk the CTA finds the first position where a
+//                   rank reaches T/R, commits everything up to it, marks that
+//                   rank full and re-evaluates the rest of the chunk, which
+//                   gives exactly the sequential visit (at most R refills).
+//   bucket sort     stable partition by assigned rank gives perm / inv: rank
+//                   d's tokens take positions d*T/R .. in ascending t.
+#include <climits>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kTile = 1024;  // items per bucket-sort tile
+
+struct ShufWs {
+    int32_t *pref;                 // [E*R]
+    unsigned long long *num, *den; // [E]
+    int32_t *cls;                  // [E]
+    int32_t *order;                // [T]
+    int32_t *tile_hist;            // [n_tiles * max(E+1, R)]
+};
+
+size_t shuf_layout(int64_t T, int E, int R, ShufWs *w, void *base)
+{
+    char *b = static_cast<char *>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        char *p = b ? b + o : nullptr;
+        o += md::align_up(bytes, 256);
+        return p;
+    };
+    const int64_t n_tiles = (T + kTile - 1) / kTile;
+    ShufWs x;
+    x.pref = reinterpret_cast<int32_t *>(take((size_t)E * R * 4));
+    x.num = reinterpret_cast<unsigned long long *>(take((size_t)E * 8));
+    x.den = reinterpret_cast<unsigned long long *>(take((size_t)E * 8));
+    x.cls = reinterpret_cast<int32_t *>(take((size_t)E * 4));
+    x.order = reinterpret_cast<int32_t *>(take((size_t)(T > 0 ? T : 1) * 4));
+    const int nbk = E + 1 > R ? E + 1 : R;
+    x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)(n_tiles > 0 ? n_tiles : 1) * nbk * 4));
+    if (w) *w = x;
+    return o;
+}
+
+// ------------------------------------------------------ per-expert tables
+__global__ void __launch_bounds__(256)
+    k_shuf_prefs(const uint32_t *__restrict__ C, const int32_t *__restrict__ p_next, int E, int R,
+                 ShufWs ws, int32_t *status)
+{
+    __shared__ unsigned long long s_sig[MD_MAX_RANKS];
+    __shared__ unsigned long long s_tot[8];
+    __shared__ uint32_t s_bv[8];
+    __shared__ int s_be[8];
+    __shared__ int s_first;
+    const int e1 = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    for (int d = tid; d < R; d += 256) s_sig[d] = 0ull;
+    __syncthreads();
+    const uint32_t *row = C + (int64_t)e1 * E;
+    unsigned long long tot = 0;
+    uint32_t bv = 0;
+    int be = INT_MAX;
+    for (int e = tid; e < E; e += 256) {
+        const uint32_t v = row[e];
+        tot += v;
+        if (v > bv || (v == bv && e < be)) { bv = v; be = e; }
+        const int d = p_next[e];
+        if (d < 0 || d >= R) {
+            if (e1 == 0) md::report(status, MD_ERR_DATA);
+            continue;
+        }
+        if (v) atomicAdd(&s_sig[d], (unsigned long long)v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        const uint32_t v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int e2 = __shfl_xor_sync(0xffffffffu, be, o);
+        if (v2 > bv || (v2 == bv && e2 < be)) { bv = v2; be = e2; }
+    }
+    if (lane == 0) { s_tot[w] = tot; s_bv[w] = bv; s_be[w] = be; }
+    __syncthreads();
+    if (tid == 0) {
+        for (int i = 1; i < 8; ++i) {
+            s_tot[0] += s_tot[i];
+            if (s_bv[i] > s_bv[0] || (s_bv[i] == s_bv[0] && s_be[i] < s_be[0])) {
+                s_bv[0] = s_bv[i];
+                s_be[0] = s_be[i];
+            }
+        }
+        int d0 = p_next[s_be[0]];
+        if (d0 < 0 || d0 >= R) d0 = 0;
+        s_first = d0;
+        ws.num[e1] = s_bv[0];
+        ws.den[e1] = s_tot[0];
+    }
+    __syncthreads();
+    const int first = s_first;
+    for (int d = tid; d < R; d += 256) {
+        int pos = 0;
+        if (d != first) {
+            pos = 1;
+            for (int d2 = 0; d2 < R; ++d2)
+                if (d2 != first && d2 != d &&
+                    (s_sig[d2] > s_sig[d] || (s_sig[d2] == s_sig[d] && d2 < d)))
+                    ++pos;
+        }
+        ws.pref[(int64_t)e1 * R + pos] = d;
+    }
+}
+
+__global__ void __launch_bounds__(256) k_shuf_class(int E, ShufWs ws)
+{
+    const int e = blockIdx.x * 256 + threadIdx.x;
+    if (e >= E) return;
+    const unsigned long long n = ws.num[e], d = ws.den[e];
+    if (d == 0) { ws.cls[e] = E; return; }
+    int c = 0;
+    for (int e2 = 0; e2 < E; ++e2) {
+        const unsigned long long d2 = ws.den[e2];
+        if (d2 == 0) continue;
+        // conf(e2) > conf(e)  <=>  num2 * d > n * d2
+        if ((unsigned __int128)ws.num[e2] * d > (unsigned __int128)n * d2) ++c;
+    }
+    ws.cls[e] = c;
+}
+
+// ------------------------------------------------------------ bucket sort
+// key source 0: confidence class of the token's top-1 expert (E+1 buckets);
+// key source 1: assigned rank (R buckets).
+__device__ __forceinline__ int bucket_key(int src, int64_t t, const int32_t *idx_l, int k,
+                                          const int32_t *cls, int E, const int32_t *pred, int nbk)
+{
+    if (src == 0) {
+        const int e1 = idx_l[t * k];
+        return (e1 >= 0 && e1 < E) ? cls[e1] : E;
+    }
+    const int d = pred[t];
+    return d >= 0 && d < nbk ? d : 0;  // every token is assigned; keep bounds anyway
+}
+
+__global__ void __launch_bounds__(256)
+    k_bucket_hist(int src, int64_t T, const int32_t *__restrict__ idx_l, int k,
+                  const int32_t *__restrict__ cls, int E, const int32_t *__restrict__ pred, int nbk,
+                  int32_t *__restrict__ tile_hist)
+{
+    extern __shared__ int h[];
+    for (int b = threadIdx.x; b < nbk; b += 256) h[b] = 0;
+    __syncthreads();
+    const int64_t t0 = (int64_t)blockIdx.x * kTile;
+    for (int i = threadIdx.x; i < kTile; i += 256) {
+        const int64_t t = t0 + i;
+        if (t < T) atomicAdd(&h[bucket_key(src, t, idx_l, k, cls, E, pred, nbk)], 1);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < nbk; b += 256) tile_hist[(int64_t)blockIdx.x * nbk + b] = h[b];
+}
+
+// tile_hist[tile][b] <- first output position of bucket b's items in tile
+__global__ void __launch_bounds__(1024)
+    k_bucket_scan(int32_t *__restrict__ tile_hist, int n_tiles, int nbk)
+{
+    extern __shared__ int tot[];
+    for (int b = threadIdx.x; b < nbk; b += 1024) {
+        int run = 0;
+        for (int i = 0; i < n_tiles; ++i) {
+            const int v = tile_hist[(int64_t)i * nbk + b];
+            tile_hist[(int64_t)i * nbk + b] = run;
+            run += v;
+        }
+        tot[b] = run;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int b = 0; b < nbk; ++b) {
+            const int v = tot[b];
+            tot[b] = run;
+            run += v;
+        }
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < nbk; b += 1024) {
+        const int base = tot[b];
+        for (int i = 0; i < n_tiles; ++i) tile_hist[(int64_t)i * nbk + b] += base;
+    }
+}
+
+// One warp per tile: items in ascending t, stable within each bucket.
+__global__ void __launch_bounds__(32)
+    k_bucket_scatter(int src, int64_t T, const int32_t *__restrict__ idx_l, int k,
+                     const int32_t *__restrict__ cls, int E, const int32_t *__restrict__ pred,
+                     int nbk, const int32_t *__restrict__ tile_hist, int32_t *__restrict__ order,
+                     int32_t *__restrict__ perm, int32_t *__restrict__ inv)
+{
+    extern __shared__ int cnt[];
+    const int lane = threadIdx.x;
+    for (int b = lane; b < nbk; b += 32) cnt[b] = tile_hist[(int64_t)blockIdx.x * nbk + b];
+    __syncwarp();
+    const int64_t t0 = (int64_t)blockIdx.x * kTile;
+    for (int c = 0; c < kTile; c += 32) {
+        const int64_t t = t0 + c + lane;
+        const bool in = t < T;
+        const int key = in ? bucket_key(src, t, idx_l, k, cls, E, pred, nbk) : -1;
+        const unsigned g = __match_any_sync(0xffffffffu, in ? (unsigned)key : (0x80000000u | lane));
+        int pos = 0;
+        if (in) pos = cnt[key] + __popc(g & md::lanemask_lt());
+        __syncwarp();
+        if (in && (g >> lane) == 1u) cnt[key] += __popc(g);
+        __syncwarp();
+        if (in) {
+            if (src == 0) {
+                order[pos] = (int32_t)t;
+            } else {
+                perm[t] = pos;
+                inv[pos] = (int32_t)t;
+            }
+        }
+    }
+}
+
+// ----------------------------------------------------------------- greedy
+__global__ void __launch_bounds__(1024)
+    k_shuf_greedy(const int32_t *__restrict__ order, const int32_t *__restrict__ idx_l, int k,
+                  ShufWs ws, int64_t T, int E, int R, int64_t Tr, int32_t *__restrict__ pred,
+                  int32_t *status)
+{
+    __shared__ long long s_load[MD_MAX_RANKS];
+    __shared__ unsigned long long s_full;
+    __shared__ int s_cnt[32][MD_MAX_RANKS];
+    __shared__ int s_pmin;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    for (int d = tid; d < R; d += 1024) s_load[d] = 0;
+    if (tid == 0) s_full = 0ull;
+    __syncthreads();
+
+    for (int64_t base = 0; base < T; base += 1024) {
+        const int64_t pos = base + tid;
+        const bool have = pos < T;
+        const int64_t t = have ? order[pos] : 0;
+        int e1 = have ? idx_l[t * k] : 0;
+        bool empty_row = true;
+        if (have) {
+            if (e1 < 0 || e1 >= E) {
+                md::report(status, MD_ERR_DATA);
+                e1 = 0;
+            } else {
+                empty_row = ws.den[e1] == 0ull;
+            }
+        }
+        const int src_rank = (int)(t / Tr);
+        int start = 0;
+        while (true) {
+            const unsigned long long full = s_full;
+            int ch = -1;
+            if (have && tid >= start) {
+                if (empty_row) {
+                    if (!((full >> src_rank) & 1ull)) {
+                        ch = src_rank;
+                    } else {
+                        for (int d = 0; d < R; ++d)
+                            if (!((full >> d) & 1ull)) { ch = d; break; }
+                    }
+                } else {
+                    const int32_t *pl = ws.pref + (int64_t)e1 * R;
+                    for (int n = 0; n < R; ++n) {
+                        const int d = pl[n];
+                        if (!((full >> d) & 1ull)) { ch = d; break; }
+                    }
+                }
+            }
+            const unsigned g =
+                __match_any_sync(0xffffffffu, ch >= 0 ? (unsigned)ch : (0x80000000u | lane));
+            const int r_in = __popc(g & md::lanemask_lt());
+            for (int i = tid; i < 32 * MD_MAX_RANKS; i += 1024) (&s_cnt[0][0])[i] = 0;
+            if (tid == 0) s_pmin = INT_MAX;
+            __syncthreads();
+            if (ch >= 0 && (g >> lane) == 1u) s_cnt[wp][ch] = __popc(g);
+            __syncthreads();
+            for (int d = tid; d < R; d += 1024) {
+                int run = 0;
+                for (int w2 = 0; w2 < 32; ++w2) {
+                    const int c = s_cnt[w2][d];
+                    s_cnt[w2][d] = run;
+                    run += c;
+                }
+            }
+            __syncthreads();
+            if (ch >= 0 && s_load[ch] + s_cnt[wp][ch] + r_in + 1 == Tr) atomicMin(&s_pmin, tid);
+            __syncthreads();
+            const int pmin = s_pmin;
+            if (ch >= 0 && tid <= pmin) {
+                pred[t] = ch;
+                atomicAdd(reinterpret_cast<unsigned long long *>(&s_load[ch]), 1ull);
+            }
+            if (tid == pmin) s_full |= 1ull << ch;
+            __syncthreads();
+            if (pmin == INT_MAX || pmin >= 1023) break;
+            start = pmin + 1;
+        }
+    }
+}
+
+}  // namespace
+
+extern "C" size_t md_token_shuffle_workspace_size(int64_t T, int E, int R)
+{
+    if (T < 0 || E < 1 || R < 1) return 0;
+    return shuf_layout(T, E, R, nullptr, nullptr);
+}
+
+extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
+                                const int32_t *expert_to_rank_next, int64_t T, int E, int R,
+                                int32_t *pred_rank, int32_t *perm, int32_t *inv, void *workspace,
+                                size_t workspace_bytes, int32_t *dev_status, void *stream)
+{
+    if (T < 0 || E < 1 || R < 1 || k < 1 || k > MD_MAX_TOPK) return MD_ERR_ARG;
+    if (E > MD_MAX_EXPERTS || R > MD_MAX_RANKS || T >= ((int64_t)1 << 31)) return MD_ERR_UNSUPPORTED;
+    if (T % R != 0) return MD_ERR_ARG;
+    if (!C || !expert_to_rank_next) return MD_ERR_ARG;
+    if (T > 0 && (!idx_l || !pred_rank || !perm || !inv)) return MD_ERR_ARG;
+    const size_t need = shuf_layout(T, E, R, nullptr, nullptr);
+    if (!workspace || workspace_bytes < need) return MD_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MD_ERR_ARG;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK || T == 0) return rc;
+    ShufWs ws;
+    shuf_layout(T, E, R, &ws, workspace);
+    const int n_tiles = (int)((T + kTile - 1) / kTile);
+    const int64_t Tr = T / R;
+
+    k_shuf_prefs<<<E, 256, 0, s>>>(C, expert_to_rank_next, E, R, ws, dev_status);
+    k_shuf_class<<<(E + 255) / 256, 256, 0, s>>>(E, ws);
+    // visit order: by confidence class, then t
+    const int nbk0 = E + 1;
+    k_bucket_hist<<<n_tiles, 256, nbk0 * sizeof(int), s>>>(0, T, idx_l, k, ws.cls, E, nullptr, nbk0,
+                                                          ws.tile_hist);
+    k_bucket_scan<<<1, 1024, nbk0 * sizeof(int), s>>>(ws.tile_hist, n_tiles, nbk0);
+    k_bucket_scatter<<<n_tiles, 32, nbk0 * sizeof(int), s>>>(0, T, idx_l, k, ws.cls, E, nullptr,
+                                                            nbk0, ws.tile_hist, ws.order, nullptr,
+                                                            nullptr);
+    k_shuf_greedy<<<1, 1024, 0, s>>>(ws.order, idx_l, k, ws, T, E, R, Tr, pred_rank, dev_status);
+    // new positions: stable partition by assigned rank
+    k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
+                                                       ws.tile_hist);
+    k_bucket_scan<<<1, 1024, R * sizeof(int), s>>>(ws.tile_hist, n_tiles, R);
+    k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
+                                                         ws.tile_hist, nullptr, perm, inv);
+    md::count_launches(9);
+    return md::launch_status();
+}

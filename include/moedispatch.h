@@ -1,0 +1,268 @@
+/*
+ * moedispatch.h -- C ABI of libmoedispatch, the B200 (sm_100a) MoE token
+ * dispatch / combine path for expert parallelism.
+ *
+ * The problem follows the pages' statement of one expert-parallel dispatch
+ * ("AllToAllDispatchScenario", mlsysim API page: total_tokens of hidden_dim
+ * values over n_devices holding n_experts):
+ *   T tokens (total_tokens), H hidden values each (hidden_dim, bf16),
+ *   E experts (n_experts) placed on R ranks (n_devices) by expert_to_rank,
+ *   each token routed to its top-k experts.
+ * The R ranks are virtual: they are partitions of one GPU's memory, so every
+ * "send" is a row copy inside HBM and there are no collectives.  Source rank
+ * of token t is src(t) = t / (T / R): each rank routes a contiguous block of
+ * T/R tokens ("DODOCO: MoE AlltoAll Traffic Matrices on Real Text", Setup).
+ *
+ * Conventions for every entry point below:
+ *   - Pointers are DEVICE pointers unless marked host; the caller allocates
+ *     and owns all memory.  The library never allocates or frees.
+ *   - Arrays are dense, row-major, without padding.  bf16 is the IEEE
+ *     bfloat16 bit pattern (__nv_bfloat16).  x, y, out, z must be 16-byte
+ *     aligned and H must be a multiple of 8 (16-byte rows).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Each call
+ *     only enqueues work on it and returns; results are ready when the
+ *     stream reaches that point.
+ *   - The return value reports what can be checked on the host: MD_ERR_ARG
+ *     for bad sizes or pointers, MD_ERR_WORKSPACE for a short workspace,
+ *     MD_ERR_CUDA when a launch fails.  Nothing is enqueued on an error.
+ *   - `dev_status` (device int32, may be NULL) receives what only the data
+ *     can show: an expert index outside [0, E), an expert twice in one
+ *     token's list, a placement that does not give every rank E/R experts,
+ *     a row index outside its buffer (MD_ERR_DATA), or a bounded wait that
+ *     ran out (MD_ERR_TIMEOUT).  Each call that takes it sets it to MD_OK
+ *     first; read it after synchronising.  Offending entries are skipped,
+ *     never written out of bounds; the other outputs are then unspecified.
+ *   - Calls that share a workspace, or write the same outputs, must not run
+ *     concurrently.
+ */
+#ifndef MOEDISPATCH_H
+#define MOEDISPATCH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum md_status {
+    MD_OK = 0,
+    MD_ERR_ARG = 1,
+    MD_ERR_UNSUPPORTED = 2,
+    MD_ERR_CUDA = 3,
+    MD_ERR_WORKSPACE = 4,
+    MD_ERR_DATA = 5,
+    MD_ERR_TIMEOUT = 6
+} md_status;
+
+#define MD_CONV 0              /* one row per (token, expert) assignment   */
+#define MD_DEDUP 1             /* one row per distinct (token, rank) pair  */
+#define MD_GATE_TOPK_SOFTMAX 0 /* softmax over the k selected logits       */
+#define MD_GATE_FULL_SOFTMAX 1 /* softmax over all E logits, then gathered */
+#define MD_COMBINE_FUSED 0     /* one weighted sum per token               */
+#define MD_COMBINE_WIRE 1      /* per-rank partial sums (bf16), then sum   */
+#define MD_SEED_CONTIGUOUS 0   /* placement search starts contiguous       */
+#define MD_SEED_GREEDY_PAIRS 1 /* placement search starts from greedy pairs*/
+
+#define MD_MAX_TOPK 32
+#define MD_MAX_EXPERTS 1024
+#define MD_MAX_RANKS 64
+
+/* Name of a status code; never NULL. */
+const char *md_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int md_version(void);
+
+/* Number of kernels (and device memsets) this library has enqueued in this
+ * process so far; a host-side counter for launch accounting. */
+uint64_t md_launch_count(void);
+
+/*
+ * md_route_topk -- router top-k selection and gate weights.
+ * "Expert Coupling in MoE Pretraining" (PicX summary), Background: each token
+ * is routed to its top-k of E experts; Method 1: the routing probabilities
+ * travel with the dispatched rows.
+ *
+ *   logits    float32 [T, E]   raw router logits (no NaN; -inf allowed)
+ *   topk_idx  int32   [T, k]   out: experts by logit descending; equal
+ *                              logits (-0.0 == +0.0) by lower expert index
+ *   topk_w    float32 [T, k]   out: gate weights.  MD_GATE_TOPK_SOFTMAX:
+ *                              softmax over the k selected logits;
+ *                              MD_GATE_FULL_SOFTMAX: softmax over all E,
+ *                              read at the selected experts.  Computed in
+ *                              double from exact logit differences, rounded
+ *                              to float once.
+ *   Limits: 1 <= k <= min(E, 32), E <= 1024, T >= 0.
+ */
+int md_route_topk(const float *logits, int64_t T, int E, int k, int gate_mode,
+                  int32_t *topk_idx, float *topk_w, void *stream);
+
+/*
+ * md_dispatch_layout -- rows, positions and the rank-by-rank send matrix.
+ * "DODOCO: MoE AlltoAll Traffic Matrices on Real Text", send_matrices.csv and
+ * Reading the counts: send_counts[s][d] counts what source rank s sends to
+ * rank d; conventional counts are token-expert assignments (a row sums to
+ * T/R x k); combine returns the transposed volumes.
+ * "Expert Coupling in MoE Pretraining", Method 1: the deduplicating
+ * dispatcher sends one row per distinct (token, destination rank) pair.
+ *
+ *   topk_idx        int32 [T, k]   experts per token (from md_route_topk)
+ *   expert_to_rank  int32 [E]      p[e] in [0, R), exactly E/R experts per rank
+ *   mode            MD_CONV or MD_DEDUP
+ * Outputs:
+ *   assign_row      int32 [T, k]   conventional row of (t, j): rows ordered by
+ *                                  (p[e], e, t), e = topk_idx[t][j].  This is
+ *                                  the expert-grouped order of the expert
+ *                                  outputs md_combine reads, in both modes.
+ *   row_of_slot     int32 [T, k]   row of (t, j) in this mode's layout; in
+ *                                  MD_DEDUP rows are ordered by (d, t) and all
+ *                                  slots of t on rank d share one row.
+ *   row_token       int32 [T*k]    token of each row (first n_rows valid)
+ *   row_mask        uint32 [T*k]   bit j set: the row carries slot j of its token
+ *   send_counts     int32 [R, R]   rows from source rank s to rank d
+ *   expert_counts   int32 [E]      tokens selecting expert e
+ *   expert_offsets  int32 [E+1]    first conventional row of expert e; [E] = T*k
+ *   rank_offsets    int32 [R+1]    first row of rank d in this mode; [R] = n_rows
+ *   n_rows          int32 [1]      rows in this mode (T*k for MD_CONV)
+ *   workspace       >= md_dispatch_layout_workspace_size(...) bytes, 256-B
+ *                   aligned; contents on entry do not matter.
+ *   Limits: T % R == 0, E % R == 0, 1 <= k <= min(E, 32), E <= 1024,
+ *   R <= 64, T*k < 2^31.
+ */
+size_t md_dispatch_layout_workspace_size(int64_t T, int E, int k, int R, int mode);
+
+int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int k, int R,
+                       const int32_t *expert_to_rank, int mode,
+                       int32_t *row_of_slot, int32_t *assign_row,
+                       int32_t *row_token, uint32_t *row_mask,
+                       int32_t *send_counts, int32_t *expert_counts,
+                       int32_t *expert_offsets, int32_t *rank_offsets, int32_t *n_rows,
+                       void *workspace, size_t workspace_bytes,
+                       int32_t *dev_status, void *stream);
+
+/*
+ * md_dispatch_permute -- build the dispatch buffer: out[row] = x[token(row)]
+ * bit for bit.  "DODOCO ...", Reading the counts: the payload of a count is
+ * hidden_size x bytes per element (bf16 here).
+ * Token-major scatter: each x row is read once and written to every distinct
+ * row named in row_of_slot[t][*] (slots sharing a row are written once).
+ *
+ *   x            bf16  [T, H]
+ *   row_of_slot  int32 [T, k]   from md_dispatch_layout (either mode)
+ *   out          bf16  [out_rows, H]; rows nobody names are left untouched
+ *   A row index outside [0, out_rows) is skipped and reported (MD_ERR_DATA).
+ */
+int md_dispatch_permute(const void *x, int64_t T, int H, int k,
+                        const int32_t *row_of_slot, int64_t out_rows, void *out,
+                        int32_t *dev_status, void *stream);
+
+/*
+ * md_combine -- gate-weighted combine of the expert outputs.
+ * "DODOCO ...", send_matrices.csv: combine, the second AlltoAll of each MoE
+ * layer, returns the volumes of dispatch in reverse.  "Expert Coupling ...",
+ * The Communication Bottleneck: dispatch and combine per MoE layer.
+ *
+ *   y            bf16  [y_rows, H]  expert outputs, row assign_row[t][j] holds
+ *                                   expert topk_idx[t][j]'s output for token t
+ *   assign_row, topk_idx int32 [T, k];  topk_w float32 [T, k]
+ *   MD_COMBINE_FUSED: out[t] = bf16( sum over t's slots by ascending expert
+ *                     of w * y, fp32 fused multiply-add from +0.0f ).
+ *   MD_COMBINE_WIRE:  with row_of_slot from an MD_DEDUP layout: for each wire
+ *                     row of t (ascending, i.e. ascending destination rank)
+ *                     z[row] = bf16( same sum over the slots on that row );
+ *                     out[t] = bf16( fp32 sum of the z rows in that order ).
+ *                     z is bf16 [z_rows, H] (the return rows of the wire).
+ *   out          bf16 [T, H]
+ *   Row indices outside y_rows / z_rows are skipped and reported.
+ */
+int md_combine(const void *y, int64_t y_rows, const int32_t *assign_row,
+               const int32_t *topk_idx, const float *topk_w, int64_t T, int k, int H,
+               int combine_mode, const int32_t *row_of_slot, int64_t z_rows, void *z,
+               void *out, int32_t *dev_status, void *stream);
+
+/*
+ * md_coselect_stats -- within-layer co-selection and cross-layer counts.
+ * "Expert Coupling ...", Correlated Placement: W[e, e'] counts tokens
+ * selecting both e and e' (diagonal: tokens selecting e); Cross-layer
+ * correlation: experts chosen at layer l predict those at layer l+1.
+ *
+ *   idx_l     int32 [>= T_fit, k]  layer-l top-k
+ *   idx_next  int32 [>= T_fit, k]  layer-l+1 top-k, or NULL (then C unused)
+ *   W         uint32 [E, E] or NULL: W[e][e'] += #{t < T_fit : e, e' in S_l(t)}
+ *   C         uint32 [E, E] or NULL: C[e][e'] += #{(t,i,j) : S_l(t)_i = e,
+ *                                                     S_l+1(t)_j = e'}
+ *   accumulate  0: W and C are cleared first; 1: counts are added.
+ *   Limits: E <= 1024, k <= 32.
+ */
+int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, int64_t T_fit, int E,
+                      int k, uint32_t *W, uint32_t *C, int accumulate, int32_t *dev_status,
+                      void *stream);
+
+/*
+ * md_place_correlated -- correlated expert placement on the GPU.
+ * "Expert Coupling ...", Correlated Placement: a Kernighan-Lin-style local
+ * search from contiguous placement swaps experts between GPUs to maximise
+ * the sum of W over co-located pairs; every GPU holds exactly E/EP experts.
+ *
+ *   W               uint32 [E, E], symmetric (from md_coselect_stats)
+ *   seed_mode       MD_SEED_CONTIGUOUS or MD_SEED_GREEDY_PAIRS (pairs with
+ *                   W > 0 by weight: both unplaced -> the rank with most free
+ *                   slots if >= 2; one placed -> join it if room; leftovers
+ *                   ascending into the lowest rank with room)
+ *   refine          non-zero: repeat the best single swap (largest gain,
+ *                   lowest expert pair on ties) while it gains, at most E*E
+ *   expert_to_rank  int32 [E] out
+ *   Limits: E % R == 0, E <= 1024, R <= 64.
+ */
+size_t md_place_correlated_workspace_size(int E, int R);
+
+int md_place_correlated(const uint32_t *W, int E, int R, int seed_mode, int refine,
+                        int32_t *expert_to_rank, void *workspace, size_t workspace_bytes,
+                        int32_t *dev_status, void *stream);
+
+/*
+ * md_token_shuffle -- capacity-constrained token shuffle to predicted owners.
+ * "Expert Coupling ...", Method 2 (Token Shuffling), Mechanism: predict each
+ * token's owner rank at layer l+1; every rank owns exactly T/EP tokens, so
+ * tokens are assigned in decreasing confidence to their most preferred rank
+ * with capacity left.  Single-expert prediction: token t with layer-l top-1
+ * expert e1 prefers p_next[argmax_e' C[e1][e']] (lowest e' on ties), then
+ * the other ranks by sum_{e' on d} C[e1][e'] descending (lowest d on ties);
+ * confidence = max / sum of C's row e1 (exact rational comparison; an empty
+ * row has confidence 0 and prefers src(t), then ascending ranks).  Tokens
+ * are visited by (confidence desc, t asc).
+ *
+ *   idx_l                int32 [T, k]  layer-l top-k (column 0 is the top-1)
+ *   C                    uint32 [E, E] layer l -> l+1 counts
+ *   expert_to_rank_next  int32 [E]     layer-l+1 placement
+ *   pred_rank  int32 [T]  out: rank each token is assigned to
+ *   perm       int32 [T]  out: new position of token t; rank d's tokens take
+ *                         d*T/R .. (d+1)*T/R-1 in ascending t
+ *   inv        int32 [T]  out: inv[perm[t]] = t
+ *   Limits: T % R == 0, E <= 1024, R <= 64, T < 2^31.
+ */
+size_t md_token_shuffle_workspace_size(int64_t T, int E, int R);
+
+int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
+                     const int32_t *expert_to_rank_next, int64_t T, int E, int R,
+                     int32_t *pred_rank, int32_t *perm, int32_t *inv,
+                     void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                     void *stream);
+
+/*
+ * md_gather_rows -- dst[i] = src[index[i]] for i < n_out, rows of row_bytes.
+ * Moves tokens into (index = inv) or out of (index = perm) the shuffled order
+ * of md_token_shuffle ("Expert Coupling ...", Method 2: the all-gather
+ * restores canonical order).  row_bytes must be a multiple of 4; src and dst
+ * 16-byte aligned when row_bytes is a multiple of 16.  An index outside
+ * [0, src_rows) leaves its row untouched and is reported (MD_ERR_DATA).
+ */
+int md_gather_rows(const void *src, int64_t src_rows, int64_t row_bytes, const int32_t *index,
+                   int64_t n_out, void *dst, int32_t *dev_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEDISPATCH_H */

@@ -1,0 +1,139 @@
+"""md_dispatch_layout on the GPU against the oracle: every output bit-exact.
+
+Inputs (top-k lists, placements) come from the seeded generator and the
+oracle; the GPU and the oracle see the same arrays."""
+import numpy as np
+import pytest
+import torch
+
+import combine_warp_top_router_b200 as md
+import oracle
+from combine_warp_top_router_b200 import synth
+
+from _util import DEV, i32, shuffled_placement
+
+pytestmark = pytest.mark.gpu
+
+POISON = -7
+
+
+def gpu_layout(idx_np, E, R, p_np, mode):
+    idx = i32(idx_np)
+    T, k = idx_np.shape
+    L = md.alloc_layout(T, E, k, R, mode, DEV)
+    L.row_token.fill_(POISON)
+    L.row_mask.fill_(POISON)
+    st = md.new_status(DEV)
+    md.md_dispatch_layout(idx, E, R, i32(p_np), mode, out=L, dev_status=st)
+    torch.cuda.synchronize()
+    return L, int(st.item())
+
+
+def assert_layout_equal(L, O, T, k):
+    n = O["n_rows"]
+    assert int(L.n_rows.item()) == n
+    assert np.array_equal(L.assign_row.cpu().numpy(), O["assign_row"])
+    assert np.array_equal(L.row_of_slot.cpu().numpy(), O["row_of_slot"])
+    rt = L.row_token.cpu().numpy()
+    rm = L.row_mask.cpu().numpy().view(np.uint32)
+    assert np.array_equal(rt[:n], O["row_token"])
+    assert np.array_equal(rm[:n], O["row_mask"])
+    assert np.all(rt[n:] == POISON)  # rows past n_rows are never written
+    assert np.array_equal(L.send_counts.cpu().numpy(), O["send_counts"])
+    assert np.array_equal(L.expert_counts.cpu().numpy(), O["expert_counts"])
+    assert np.array_equal(L.expert_offsets.cpu().numpy(), O["expert_offsets"])
+    assert np.array_equal(L.rank_offsets.cpu().numpy(), O["rank_offsets"])
+
+
+def _routes(name, T, seed=0):
+    w = synth.make_workload(name, seed=seed, T=T, with_rows=False)
+    return oracle.route_topk(w.logits.numpy(), synth.SPECS[name]["k"])[0]
+
+
+CASES = [
+    # (workload, T, R, placement)
+    ("iid_e64_k6", 4096, 16, "contiguous"),
+    ("zipf_pairs_e128_k8", 8192, 16, "contiguous"),
+    ("boost_pairs_e128_k2", 8192, 8, "shuffled"),
+    ("boost_pairs_e128_k2", 8192, 32, "shuffled"),
+    ("two_layer_e128_k6", 8192, 16, "shuffled"),
+    ("full_e256_k8", 8192, 64, "contiguous"),
+    ("zipf_pairs_e128_k8", 16 * 37, 16, "contiguous"),   # ragged last tile
+    ("iid_e64_k6", 64 * 3, 64, "shuffled"),              # 3 tokens per rank
+]
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("name,T,R,pl", CASES)
+def test_layout_matches_oracle(name, T, R, pl, mode):
+    idx = _routes(name, T)
+    E = synth.SPECS[name]["E"]
+    p = synth.contiguous_placement(E, R).numpy() if pl == "contiguous" else shuffled_placement(E, R, 3)
+    L, st = gpu_layout(idx, E, R, p, mode)
+    assert st == md.MD_OK
+    assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), *idx.shape)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("E,k,R,T", [(8, 1, 2, 100), (8, 8, 8, 64), (16, 3, 1, 48), (12, 5, 3, 99),
+                                     (1024, 32, 64, 128), (256, 16, 4, 256), (64, 6, 64, 4096)])
+def test_layout_edge_shapes(E, k, R, T, mode):
+    lg = synth.normal_f32(T, E, 11, 1).numpy()
+    idx = oracle.route_topk(lg, k)[0]
+    p = shuffled_placement(E, R, 5)
+    L, st = gpu_layout(idx, E, R, p, mode)
+    assert st == md.MD_OK
+    assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), T, k)
+
+
+def test_layout_empty():
+    E, k, R = 16, 2, 4
+    L, st = gpu_layout(np.zeros((0, k), np.int32), E, R, synth.contiguous_placement(E, R).numpy(), 1)
+    assert st == md.MD_OK and int(L.n_rows.item()) == 0
+    assert int(L.send_counts.sum().item()) == 0
+    assert L.rank_offsets.cpu().tolist() == [0] * (R + 1)
+
+
+def test_layout_reports_bad_data():
+    E, k, R, T = 16, 3, 4, 64
+    idx = oracle.route_topk(synth.normal_f32(T, E, 1, 1).numpy(), k)[0]
+    p = synth.contiguous_placement(E, R).numpy()
+    bad = idx.copy()
+    bad[5, 1] = E + 3                 # out of range
+    _, st = gpu_layout(bad, E, R, p, 1)
+    assert st == md.MD_ERR_DATA
+    dup = idx.copy()
+    dup[7, 2] = dup[7, 0]             # same expert twice
+    _, st = gpu_layout(dup, E, R, p, 0)
+    assert st == md.MD_ERR_DATA
+    q = p.copy()
+    q[0] = 1                          # rank 0 has E/R - 1 experts
+    _, st = gpu_layout(idx, E, R, q, 0)
+    assert st == md.MD_ERR_DATA
+    _, st = gpu_layout(idx, E, R, p, 1)  # and a clean call resets the status
+    assert st == md.MD_OK
+
+
+def test_layout_rejects_bad_arguments():
+    idx = torch.zeros(10, 2, dtype=torch.int32, device=DEV)
+    p = torch.zeros(8, dtype=torch.int32, device=DEV)
+    with pytest.raises(md.MoeDispatchError):
+        md.md_dispatch_layout(idx, 8, 4, p, 0)           # T % R != 0
+    with pytest.raises(md.MoeDispatchError):
+        md.md_dispatch_layout(idx, 8, 2, p, 0, workspace=torch.empty(256, dtype=torch.uint8,
+                                                                    device=DEV))
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_layout_full_size(mode):
+    # the full-pipeline workload at full size: T=262144, E=256, k=8, R=64
+    w = synth.make_workload("full_e256_k8", device=DEV, with_rows=False)
+    idx_g, _ = md.md_route_topk(w.logits, 8)
+    idx = idx_g.cpu().numpy()
+    # the layout's input is the oracle's own top-k of the same logits
+    oi = oracle.route_topk(w.logits.cpu().numpy(), 8)[0]
+    assert np.array_equal(idx, oi)
+    p = synth.contiguous_placement(256, 64).numpy()
+    L, st = gpu_layout(oi, 256, 64, p, mode)
+    assert st == md.MD_OK
+    assert_layout_equal(L, oracle.dispatch_layout(oi, 256, 64, p, mode), *oi.shape)

@@ -1,0 +1,78 @@
+"""md_route_topk on the GPU against the oracle.
+
+Expert indices must match bit for bit; gate weights within 1e-6 relative."""
+import numpy as np
+import pytest
+import torch
+
+import combine_warp_top_router_b200 as md
+import oracle
+from combine_warp_top_router_b200 import synth
+
+from _util import DEV
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(lg_np, k, mode):
+    lg = torch.from_numpy(np.ascontiguousarray(lg_np, np.float32)).to(DEV)
+    idx, w = md.md_route_topk(lg, k, mode)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), w.cpu().numpy()
+
+
+def _compare(lg_np, k, mode):
+    gi, gw = _run(lg_np, k, mode)
+    oi, ow = oracle.route_topk(lg_np, k, mode)
+    assert np.array_equal(gi, oi)
+    rel = np.abs(gw.astype(np.float64) - ow) / np.maximum(np.abs(ow.astype(np.float64)), 1e-300)
+    assert rel.max() <= 1e-6, rel.max()
+    return gi, gw
+
+
+@pytest.mark.parametrize("E,k,T", [(64, 6, 4096), (128, 8, 1000), (128, 2, 777), (256, 8, 3000),
+                                   (40, 5, 300), (384, 8, 257), (1024, 32, 64), (8, 8, 50),
+                                   (1, 1, 33), (96, 3, 129)])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_iid_shapes(E, k, T, mode):
+    lg = synth.normal_f32(T, E, 7, 1).numpy() * 2.0
+    _compare(lg, k, mode)
+
+
+@pytest.mark.parametrize("name", ["iid_e64_k6", "zipf_pairs_e128_k8", "boost_pairs_e128_k2",
+                                  "full_e256_k8"])
+def test_workload_logits(name):
+    w = synth.make_workload(name, T=4096 if name != "full_e256_k8" else 8192, with_rows=False)
+    _compare(w.logits.numpy(), synth.SPECS[name]["k"], 0)
+
+
+@pytest.mark.parametrize("E", [16, 128, 256])
+def test_ties_and_signed_zero(E):
+    rng = np.random.default_rng(E)
+    lg = rng.integers(-2, 3, size=(512, E)).astype(np.float32)
+    lg[rng.random(lg.shape) < 0.2] = -0.0
+    lg[rng.random(lg.shape) < 0.05] = -np.inf
+    lg[0] = 0.0
+    lg[0, ::2] = -0.0
+    for k in (1, 4, min(E, 32)):
+        _compare(lg, k, 0)
+
+
+def test_k1_gate_is_one_and_empty_batch():
+    lg = synth.normal_f32(100, 64, 3, 1).numpy()
+    _, w = _compare(lg, 1, 0)
+    assert np.all(w == 1.0)
+    idx, w = md.md_route_topk(torch.empty(0, 64, device=DEV), 4)
+    assert idx.shape == (0, 4)
+
+
+def test_full_size_sampled():
+    # the benchmark's router shape: T=65536, E=128, k=8; every row checked
+    w = synth.make_workload("zipf_pairs_e128_k8", device=DEV, with_rows=False)
+    idx, gw = md.md_route_topk(w.logits, 8)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(0).choice(w.T, 4096, replace=False)
+    lg = w.logits.cpu().numpy()
+    oi, ow = oracle.route_topk(lg[rows], 8)
+    assert np.array_equal(idx.cpu().numpy()[rows], oi)
+    assert np.allclose(gw.cpu().numpy()[rows], ow, rtol=1e-6, atol=0)
