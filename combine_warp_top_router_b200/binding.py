@@ -37,6 +37,9 @@ _SIGNATURES = {
     "md_dispatch_layout_workspace_size": ([_L, _I, _I, _I, _I], _S),
     "md_dispatch_layout": ([_P, _L, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                             _P, _S, _P, _P], _I),
+    "md_dispatch_layout_noalloc_max_scratch": ([], _S),
+    "md_dispatch_layout_noalloc": ([_P, _L, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                                    _P, _P, _P], _I),
     "md_dispatch_permute": ([_P, _L, _I, _I, _P, _L, _P, _P, _P], _I),
     "md_combine": ([_P, _L, _P, _P, _P, _L, _I, _I, _I, _P, _L, _P, _P, _P, _P], _I),
     "md_coselect_stats": ([_P, _P, _L, _I, _I, _P, _P, _I, _P, _P], _I),
@@ -196,6 +199,26 @@ def md_dispatch_layout(topk_idx, E, R, expert_to_rank, mode, out: Layout | None 
         _ptr(out.n_rows), _ptr(workspace), workspace.numel(), _ptr(dev_status),
         _stream(stream, dev))
     _check(rc, "md_dispatch_layout")
+    return out
+
+
+def md_dispatch_layout_noalloc(topk_idx, E, R, expert_to_rank, mode, out: Layout | None = None,
+                               dev_status=None, stream=None) -> Layout:
+    """md_dispatch_layout without a workspace, for callers that cannot allocate
+    device memory: the library uses its own fixed 4 MiB per-GPU scratch array.
+    Calls that overlap on one GPU share that array and must be serialised."""
+    _need(topk_idx, "topk_idx", torch.int32)
+    dev = topk_idx.device
+    _need(expert_to_rank, "expert_to_rank", torch.int32, dev)
+    T, k = topk_idx.shape
+    if out is None:
+        out = alloc_layout(T, E, k, R, mode, dev)
+    rc = lib().md_dispatch_layout_noalloc(
+        _ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), mode, _ptr(out.row_of_slot),
+        _ptr(out.assign_row), _ptr(out.row_token), _ptr(out.row_mask), _ptr(out.send_counts),
+        _ptr(out.expert_counts), _ptr(out.expert_offsets), _ptr(out.rank_offsets),
+        _ptr(out.n_rows), _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_dispatch_layout_noalloc")
     return out
 
 

@@ -459,3 +459,66 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
     md::count_launches(1);
     return md::launch_status();
 }
+
+// ------------------------------------------------------------------------
+// md_dispatch_layout_noalloc: the same layout for callers that cannot
+// allocate device memory.  Its scratch is the file-scope array below, so the
+// library itself allocates nothing at call time.
+// ------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // MD_NOALLOC_LAYOUT_SCRATCH_BYTES
+
+// Resident on every GPU that loads the library, for the life of the process.
+static __device__ __align__(256) unsigned char g_layout_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 256;
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_layout_scratch on the current device.  In host code the
+// symbol names a host-side stand-in, so the address must be looked up with
+// cudaGetSymbolAddress while that device is current; it is cached per device.
+int scratch_for_current_device(void **addr)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MD_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_addr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_layout_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return MD_ERR_CUDA;
+        }
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return MD_OK;
+}
+
+}  // namespace
+
+extern "C" size_t md_dispatch_layout_noalloc_max_scratch(void) { return kNoAllocScratchBytes; }
+
+extern "C" int md_dispatch_layout_noalloc(const int32_t *topk_idx, int64_t T, int E, int k, int R,
+                                          const int32_t *expert_to_rank, int mode,
+                                          int32_t *row_of_slot, int32_t *assign_row,
+                                          int32_t *row_token, uint32_t *row_mask,
+                                          int32_t *send_counts, int32_t *expert_counts,
+                                          int32_t *expert_offsets, int32_t *rank_offsets,
+                                          int32_t *n_rows, int32_t *dev_status, void *stream)
+{
+    int rc = check_layout_args(T, E, k, R, mode);
+    if (rc != MD_OK) return rc;
+    if (plan(T, E, k, R, mode).total > kNoAllocScratchBytes) return MD_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((rc = scratch_for_current_device(&scratch)) != MD_OK) return rc;
+    // The shared array keeps the previous call's contents; md_dispatch_layout
+    // clears the part that must start at zero on the stream before using it.
+    return md_dispatch_layout(topk_idx, T, E, k, R, expert_to_rank, mode, row_of_slot, assign_row,
+                              row_token, row_mask, send_counts, expert_counts, expert_offsets,
+                              rank_offsets, n_rows, scratch, kNoAllocScratchBytes, dev_status,
+                              stream);
+}

@@ -142,6 +142,42 @@ int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int k, int R,
                        int32_t *dev_status, void *stream);
 
 /*
+ * md_dispatch_layout_noalloc -- md_dispatch_layout without a caller workspace.
+ * No counterpart in the source pages: this is a calling convenience, not a
+ * step of the method.  Some callers cannot allocate device memory at all --
+ * for example a plug-in running inside a host framework that owns every byte
+ * of GPU memory through its own pool, or a process that has handed all free
+ * HBM to a caching allocator -- so they cannot size and cudaMalloc the
+ * workspace md_dispatch_layout needs.  This entry point takes the same
+ * arguments minus the workspace and allocates nothing: its scratch is a
+ * fixed array of MD_NOALLOC_LAYOUT_SCRATCH_BYTES (4 MiB) compiled into the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  The caller still passes all inputs and outputs.
+ *   - Problems whose workspace would exceed that size return
+ *     MD_ERR_UNSUPPORTED (md_dispatch_layout_workspace_size tells the need;
+ *     T=262144, E=256, k=8, R=64 dedup needs about 2.6 MiB).
+ *   - The first call on each device looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Every call on a device shares the one array, which keeps the previous
+ *     call's contents; each call clears what must start at zero on its
+ *     stream.  Calls that overlap on the GPU (other streams, other threads)
+ *     race on it and must be serialised by the caller.
+ *   - Results are identical to md_dispatch_layout's.
+ */
+#define MD_NOALLOC_LAYOUT_SCRATCH_BYTES ((size_t)4 << 20)
+
+size_t md_dispatch_layout_noalloc_max_scratch(void);
+
+int md_dispatch_layout_noalloc(const int32_t *topk_idx, int64_t T, int E, int k, int R,
+                               const int32_t *expert_to_rank, int mode,
+                               int32_t *row_of_slot, int32_t *assign_row,
+                               int32_t *row_token, uint32_t *row_mask,
+                               int32_t *send_counts, int32_t *expert_counts,
+                               int32_t *expert_offsets, int32_t *rank_offsets, int32_t *n_rows,
+                               int32_t *dev_status, void *stream);
+
+/*
  * md_dispatch_permute -- build the dispatch buffer: out[row] = x[token(row)]
  * bit for bit.  "DODOCO ...", Reading the counts: the payload of a count is
  * hidden_size x bytes per element (bf16 here).
