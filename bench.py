@@ -376,7 +376,7 @@ def run_reference(args):
     # bound the run to about a minute of CPU for K + W steps
     per_step = 60.0 / max(1, args.steps + args.warmup)
     T_s = int(per_step * CPU_TOKENS_PER_S_GUESS) // R * R
-    T_s = max(R, min(65536, T_s))
+    T_s = max(R, min(16384, T_s))
     inp = oracle_sample(T_s, args.seed)
     for _ in range(args.warmup):
         oracle_step(oracle, inp, args.dispatch == "dedup")

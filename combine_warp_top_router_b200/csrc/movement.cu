@@ -1,14 +1,17 @@
 // movement.cu -- row movement on HBM: dispatch permute, combine, row gather
 // (md_dispatch_permute, md_combine, md_gather_rows).
 //
-// All three are bound by HBM bandwidth.  Rows are moved as 16-byte vectors,
-// one 16-byte column chunk per thread, so every warp reads or writes 512
-// contiguous bytes of a row.  A CTA works on a group of kGroup tokens at a
-// time: it first stages the group's row indices (and, for combine, the slot
-// order and gates) in shared memory, then each thread issues all loads of
-// its column chunk for the group before any store, so kGroup (permute) or k
-// (combine) 16-byte loads per thread are in flight.  Grids are a multiple of
-// the SM count and loop over token groups.
+// All three are bound by HBM bandwidth and move rows as 16-byte vectors, so
+// every warp instruction reads or writes 512 contiguous bytes of a row.
+//   permute  one warp per token, no block barriers; the next token's x row
+//            and row indices are loaded while the current token's stores
+//            drain.
+//   combine  a CTA takes kGroup tokens at a time: one warp per token orders
+//            its slots and stages (row, gate) in shared memory, then each
+//            thread issues the k 16-byte loads of its column chunk before the
+//            FMAs, so k loads per thread are in flight.
+//   gather   one 16-byte (or 4-byte) chunk per thread, grid-stride.
+// Grids are sized from the SM count and loop over their work.
 #include <climits>
 
 #include "common.cuh"
@@ -28,47 +31,65 @@ int grid_for(int64_t units, int per_block)
 
 // ----------------------------------------------------------------- permute
 // out[row_of_slot[t][j]] = x[t] for every distinct row of token t.
+// One warp per token, no block barriers.  A pass moves kPermU 16-byte chunks
+// per lane (4 KiB per warp); while the stores of token t drain, the x chunks
+// and row indices of the warp's next token are already in flight.
+constexpr int kPermU = 8;
+
 template <int KC>
 __global__ void __launch_bounds__(kThreads)
     k_permute(const uint4 *__restrict__ x, int64_t T, int C, int k,
               const int32_t *__restrict__ row_of_slot, int64_t out_rows, uint4 *__restrict__ out,
               int32_t *status)
 {
-    __shared__ int s_row[kGroup][MD_MAX_TOPK];
     const int K = KC ? KC : k;
-    for (int64_t g0 = (int64_t)blockIdx.x * kGroup; g0 < T; g0 += (int64_t)gridDim.x * kGroup) {
-        const int ng = (int)(T - g0 < kGroup ? T - g0 : kGroup);
-        for (int i = threadIdx.x; i < ng * K; i += kThreads) {
-            const int g = i / K, j = i - g * K;
-            const int32_t *rr = row_of_slot + (g0 + g) * K;
-            int r = rr[j];
-            bool dup = false;
-            for (int j2 = 0; j2 < j; ++j2)
-                if (__ldg(rr + j2) == r) dup = true;
-            if (!dup && (r < 0 || r >= out_rows)) {
-                md::report(status, MD_ERR_DATA);
-                r = -1;
-            }
-            s_row[g][j] = dup ? -1 : r;
+    const int lane = threadIdx.x & 31;
+    const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
+    if (w0 >= T) return;
+    for (int c0 = 0; c0 < C; c0 += 32 * kPermU) {
+        int64_t t = w0;
+        uint4 cur[kPermU];
+        int rows = -1;
+#pragma unroll
+        for (int u = 0; u < kPermU; ++u) {
+            const int c = c0 + u * 32 + lane;
+            if (c < C) cur[u] = md::ld_stream(x + t * C + c);
         }
-        __syncthreads();
-        for (int c = threadIdx.x; c < C; c += kThreads) {
-            uint4 v[kGroup];
+        if (lane < K) rows = __ldg(row_of_slot + t * K + lane);
+        for (; t < T; t += nw) {
+            const int64_t tn = t + nw;
+            uint4 nxt[kPermU];
+            int nrows = -1;
+            if (tn < T) {
 #pragma unroll
-            for (int g = 0; g < kGroup; ++g)
-                if (g < ng) v[g] = md::ld_stream(x + (g0 + g) * C + c);
+                for (int u = 0; u < kPermU; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < C) nxt[u] = md::ld_stream(x + tn * C + c);
+                }
+                if (lane < K) nrows = __ldg(row_of_slot + tn * K + lane);
+            }
+            // distinct, in-range rows of this token (slots sharing a row write once)
+            const unsigned g = __match_any_sync(0xffffffffu, lane < K ? (unsigned)rows : (0x80000000u | lane));
+            const bool first = lane < K && (g & md::lanemask_lt()) == 0u;
+            const bool ok = rows >= 0 && rows < out_rows;
+            if (first && !ok && c0 == 0) md::report(status, MD_ERR_DATA);
+            unsigned todo = __ballot_sync(0xffffffffu, first && ok);
+            while (todo) {
+                const int j = __ffs(todo) - 1;
+                todo &= todo - 1;
+                const int64_t r = __shfl_sync(0xffffffffu, rows, j);
+                uint4 *dst = out + r * C;
 #pragma unroll
-            for (int g = 0; g < kGroup; ++g) {
-                if (g < ng) {
-#pragma unroll 8
-                    for (int j = 0; j < K; ++j) {
-                        const int r = s_row[g][j];
-                        if (r >= 0) md::st_stream(out + (int64_t)r * C + c, v[g]);
-                    }
+                for (int u = 0; u < kPermU; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < C) md::st_stream(dst + c, cur[u]);
                 }
             }
+#pragma unroll
+            for (int u = 0; u < kPermU; ++u) cur[u] = nxt[u];
+            rows = nrows;
         }
-        __syncthreads();
     }
 }
 
@@ -227,7 +248,15 @@ template <int KC>
 void launch_permute(const void *x, int64_t T, int C, int k, const int32_t *rs, int64_t rows,
                     void *out, int32_t *st, cudaStream_t s)
 {
-    k_permute<KC><<<grid_for(T, kGroup), kThreads, 0, s>>>(
+    static int per_sm = 0;
+    if (per_sm == 0) {
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_permute<KC>, kThreads, 0);
+        if (per_sm < 1) per_sm = 1;
+    }
+    int64_t blocks = (T + kThreads / 32 - 1) / (kThreads / 32);
+    const int64_t cap = (int64_t)md::sm_count() * per_sm;
+    if (blocks > cap) blocks = cap;
+    k_permute<KC><<<(unsigned)(blocks < 1 ? 1 : blocks), kThreads, 0, s>>>(
         static_cast<const uint4 *>(x), T, C, k, rs, rows, static_cast<uint4 *>(out), st);
 }
 

@@ -5,18 +5,28 @@
 // ride with the dispatched rows.
 //
 // One warp per token.  Lane L holds M of the token's E logits as order-
-// preserving 32-bit keys (element index increases with the register slot).
-// k rounds of a warp arg-max pick the experts: __reduce_max_sync finds the
-// largest key, __reduce_min_sync the lowest expert holding it, and only the
-// winning lane replaces its local best.  Keys compare exactly like the fp32
-// logits with -0.0 folded onto +0.0, so ties go to the lower expert index.
-// The gates are computed in double from exact logit differences and rounded
-// to float once.
+// preserving 32-bit keys (element index increases with the register slot);
+// keys compare exactly like the fp32 logits with -0.0 folded onto +0.0, and
+// equal keys go to the lower expert index.
+//
+// Fast path: the k-th largest of the 32 lane maxima is a lower bound on the
+// k-th largest logit (k lane maxima are k distinct logits at or above it), so
+// every top-k element is at or above it.  The few candidates that pass
+// (typically k to 2k) are compacted one per lane, and k rounds of
+// __reduce_max_sync / __reduce_min_sync pick them in order.  If more than 32
+// pass (heavy ties), the exact slow path runs instead: k rounds of the same
+// warp arg-max over all elements, with the winning lane rescanning its own.
+//
+// A warp handles G = floor(32/k) tokens back to back and keeps token g's slot
+// r in lane g*k + r, so the gates of the whole group are computed at once:
+// exp of exact (double) logit differences to the token's largest logit, a
+// double sum in slot order, one rounding to float.
 #include "common.cuh"
 
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
 
 __device__ __forceinline__ uint32_t float_key(float f)
 {
@@ -32,7 +42,7 @@ __device__ __forceinline__ float key_float(uint32_t k)
 }
 
 // Element held in register slot s of `lane`.
-template <int M, bool VEC>
+template <bool VEC>
 __device__ __forceinline__ int elem_of(int lane, int s)
 {
     return VEC ? (s >> 2) * 128 + lane * 4 + (s & 3) : s * 32 + lane;
@@ -46,77 +56,150 @@ __device__ __forceinline__ double warp_sum_d(double v)
 }
 
 template <int M, bool VEC>
+__device__ __forceinline__ void load_row(float (&v)[M], const float *row, int E, int lane)
+{
+    if (VEC) {
+#pragma unroll
+        for (int c = 0; c < M / 4; ++c) {
+            float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c * 128 < E) q = __ldcs(reinterpret_cast<const float4 *>(row + c * 128 + lane * 4));
+            v[4 * c + 0] = q.x;
+            v[4 * c + 1] = q.y;
+            v[4 * c + 2] = q.z;
+            v[4 * c + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int s = 0; s < M; ++s) {
+            const int e = s * 32 + lane;
+            v[s] = e < E ? __ldcs(row + e) : 0.0f;
+        }
+    }
+}
+
+template <int M, bool VEC>
 __global__ void __launch_bounds__(kThreads)
     k_route_topk(const float *__restrict__ logits, int64_t T, int E, int k, int gate_mode,
                  int32_t *__restrict__ out_idx, float *__restrict__ out_w)
 {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * kThreads) >> 5;
+    __shared__ uint32_t s_ck[kWarps][32];
+    __shared__ int s_ce[kWarps][32];
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+    const int G = 32 / k;  // tokens per warp group
+    const int64_t warp0 = (int64_t)blockIdx.x * kWarps + wl;
+    const int64_t nwarps = (int64_t)gridDim.x * kWarps;
 
-    for (int64_t t = warp0; t < T; t += nwarps) {
-        const float *row = logits + t * (int64_t)E;
-        float val[M];
-        uint32_t key[M];
-        if (VEC) {
+    // token sequence of this warp: groups tg = (warp0 + i*nwarps)*G, tokens tg .. tg+G-1;
+    // the next token's logits are loaded while the current one is processed
+    float cur[M];
+    const int64_t first = warp0 * G;
+    if (first < T) load_row<M, VEC>(cur, logits + first * (int64_t)E, E, lane);
+    for (int64_t tg = first; tg < T; tg += nwarps * G) {
+        int my_e = -1;          // lane g*k + r: expert of token tg+g, slot r
+        uint32_t my_key = 0;
+        double my_den = 1.0;    // full-softmax denominator of that token
+        const int ng = (int)(T - tg < G ? T - tg : G);
+        for (int g = 0; g < ng; ++g) {
+            const int64_t tn = g + 1 < ng ? tg + g + 1 : tg + nwarps * G;
+            float val[M];
 #pragma unroll
-            for (int c = 0; c < M / 4; ++c) {
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (c * 128 < E) v = __ldcs(reinterpret_cast<const float4 *>(row + c * 128 + lane * 4));
-                val[4 * c + 0] = v.x;
-                val[4 * c + 1] = v.y;
-                val[4 * c + 2] = v.z;
-                val[4 * c + 3] = v.w;
-            }
-        } else {
+            for (int s = 0; s < M; ++s) val[s] = cur[s];
+            if (tn < T) load_row<M, VEC>(cur, logits + tn * (int64_t)E, E, lane);
+            uint32_t key[M];
+            uint32_t best = 0;
+            int bs = 0;
 #pragma unroll
             for (int s = 0; s < M; ++s) {
-                int e = s * 32 + lane;
-                val[s] = e < E ? __ldcs(row + e) : 0.0f;
+                key[s] = elem_of<VEC>(lane, s) < E ? float_key(val[s]) : 0u;
+                if (key[s] > best) { best = key[s]; bs = s; }
             }
-        }
-        uint32_t best = 0;
-        int bs = 0;
-#pragma unroll
-        for (int s = 0; s < M; ++s) {
-            key[s] = elem_of<M, VEC>(lane, s) < E ? float_key(val[s]) : 0u;
-            if (key[s] > best) { best = key[s]; bs = s; }
-        }
-
-        int my_e = -1;
-        uint32_t my_key = 0;
-        double denom_full = 0.0;
-        for (int r = 0; r < k; ++r) {
-            const uint32_t kmax = __reduce_max_sync(0xffffffffu, best);
-            const uint32_t cand = best == kmax ? (uint32_t)elem_of<M, VEC>(lane, bs) : 0xffffffffu;
-            const uint32_t emin = __reduce_min_sync(0xffffffffu, cand);
-            if (r == 0 && gate_mode == MD_GATE_FULL_SOFTMAX) {
-                const double m = (double)key_float(kmax);
+            if (gate_mode == MD_GATE_FULL_SOFTMAX) {
+                const double m = (double)key_float(__reduce_max_sync(0xffffffffu, best));
                 double s = 0.0;
 #pragma unroll
                 for (int q = 0; q < M; ++q)
-                    if (elem_of<M, VEC>(lane, q) < E) s += exp((double)val[q] - m);
-                denom_full = warp_sum_d(s);
+                    if (elem_of<VEC>(lane, q) < E) s += exp((double)val[q] - m);
+                s = warp_sum_d(s);
+                if (lane >= g * k && lane < (g + 1) * k) my_den = s;
             }
-            if (lane == r) { my_e = (int)emin; my_key = kmax; }
-            if (cand == emin) {  // winning lane: drop the taken element, find the next best
-                best = 0;
-                bs = 0;
+
+            // threshold: the k-th largest lane maximum
+            uint32_t act = best, th = 0;
+            for (int r = 0; r < k; ++r) {
+                th = __reduce_max_sync(0xffffffffu, act);
+                const unsigned b = __ballot_sync(0xffffffffu, act == th);
+                if (lane == __ffs(b) - 1) act = 0u;
+            }
+            int c = 0;
 #pragma unroll
-                for (int s = 0; s < M; ++s) {
-                    if (elem_of<M, VEC>(lane, s) == (int)emin) key[s] = 0u;
-                    if (key[s] > best) { best = key[s]; bs = s; }
+            for (int s = 0; s < M; ++s) c += key[s] >= th ? 1 : 0;
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int ncand = __shfl_sync(0xffffffffu, incl, 31);
+
+            if (ncand <= 32) {
+                int pos = incl - c;
+#pragma unroll
+                for (int s = 0; s < M; ++s)
+                    if (key[s] >= th) {
+                        s_ck[wl][pos] = key[s];
+                        s_ce[wl][pos] = elem_of<VEC>(lane, s);
+                        ++pos;
+                    }
+                __syncwarp();
+                uint32_t ck = lane < ncand ? s_ck[wl][lane] : 0u;
+                const uint32_t ce = lane < ncand ? (uint32_t)s_ce[wl][lane] : 0xffffffffu;
+                __syncwarp();
+                for (int r = 0; r < k; ++r) {
+                    const uint32_t kmax = __reduce_max_sync(0xffffffffu, ck);
+                    const uint32_t cand = ck == kmax ? ce : 0xffffffffu;
+                    const uint32_t emin = __reduce_min_sync(0xffffffffu, cand);
+                    if (cand == emin) ck = 0u;
+                    if (lane == g * k + r) { my_e = (int)emin; my_key = kmax; }
+                }
+            } else {
+                // exact fallback over all elements
+                for (int r = 0; r < k; ++r) {
+                    const uint32_t kmax = __reduce_max_sync(0xffffffffu, best);
+                    const uint32_t cand = best == kmax ? (uint32_t)elem_of<VEC>(lane, bs) : 0xffffffffu;
+                    const uint32_t emin = __reduce_min_sync(0xffffffffu, cand);
+                    if (lane == g * k + r) { my_e = (int)emin; my_key = kmax; }
+                    if (cand == emin) {
+                        best = 0;
+                        bs = 0;
+#pragma unroll
+                        for (int s = 0; s < M; ++s) {
+                            if (elem_of<VEC>(lane, s) == (int)emin) key[s] = 0u;
+                            if (key[s] > best) { best = key[s]; bs = s; }
+                        }
+                    }
                 }
             }
         }
 
-        // gates: exp of exact (double) differences to the largest logit
-        const float m = __shfl_sync(0xffffffffu, key_float(my_key), 0);
-        const double ex = lane < k ? exp((double)key_float(my_key) - (double)m) : 0.0;
-        const double denom = gate_mode == MD_GATE_FULL_SOFTMAX ? denom_full : warp_sum_d(ex);
-        if (lane < k) {
-            out_idx[t * k + lane] = my_e;
-            out_w[t * k + lane] = (float)(ex / denom);
+        // gates of the whole group: lane g*k + r holds token g's slot r
+        const int base = (lane / k) * k;
+        const bool live = lane < ng * k;
+        const float v = key_float(my_key);
+        const float m = __shfl_sync(0xffffffffu, v, base < 32 ? base : 0);
+        const double ex = live ? exp((double)v - (double)m) : 0.0;
+        double den;
+        if (gate_mode == MD_GATE_FULL_SOFTMAX) {
+            den = my_den;
+        } else {
+            den = 0.0;
+            for (int r = 0; r < k; ++r) {
+                const int src = base + r;
+                den += __shfl_sync(0xffffffffu, ex, src < 32 ? src : 0);
+            }
+        }
+        if (live) {
+            out_idx[tg * k + lane] = my_e;
+            out_w[tg * k + lane] = (float)(ex / den);
         }
     }
 }
@@ -125,8 +208,9 @@ template <int M, bool VEC>
 void launch(const float *logits, int64_t T, int E, int k, int gate_mode, int32_t *idx, float *w,
             cudaStream_t s)
 {
-    int64_t blocks = (T + kThreads / 32 - 1) / (kThreads / 32);
-    int64_t cap = (int64_t)md::sm_count() * 16;
+    const int64_t G = 32 / k;
+    int64_t blocks = (T + kWarps * G - 1) / (kWarps * G);
+    const int64_t cap = (int64_t)md::sm_count() * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     k_route_topk<M, VEC><<<(unsigned)blocks, kThreads, 0, s>>>(logits, T, E, k, gate_mode, idx, w);

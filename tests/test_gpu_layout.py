@@ -137,3 +137,21 @@ def test_layout_full_size(mode):
     L, st = gpu_layout(oi, 256, 64, p, mode)
     assert st == md.MD_OK
     assert_layout_equal(L, oracle.dispatch_layout(oi, 256, 64, p, mode), *oi.shape)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_layout_unaligned_outputs(mode):
+    # outputs that are not 16-byte aligned take the scalar-store kernel
+    name, T, R = "zipf_pairs_e128_k8", 2048, 16
+    idx = _routes(name, T)
+    E, k = 128, 8
+    p = synth.contiguous_placement(E, R).numpy()
+    L = md.alloc_layout(T, E, k, R, mode, DEV)
+    raw_a = torch.full((T * k + 1,), -5, dtype=torch.int32, device=DEV)
+    raw_r = torch.full((T * k + 1,), -5, dtype=torch.int32, device=DEV)
+    L.assign_row = raw_a[1:].view(T, k)
+    L.row_of_slot = raw_r[1:].view(T, k)
+    L.row_token.fill_(POISON)
+    md.md_dispatch_layout(i32(idx), E, R, i32(p), mode, out=L)
+    torch.cuda.synchronize()
+    assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), T, k)
