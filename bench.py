@@ -280,8 +280,174 @@ def run_native(args):
         "e2e": e2e,
         "clocks": clk.summary(),
     }
+    if args.rows:
+        del w, buf, out
+        torch.cuda.empty_cache()
+        line["rows"] = run_rows(args, md, device, stream, peak)
     line["cpu_baseline"] = cpu_baseline(args)
     return line
+
+
+def _time(fn, stream, reps):
+    """Average device time (ms) of fn() over reps launches on `stream`, after a warm-up.
+    Inputs are produced on the default stream, which the (non-blocking) timing
+    stream does not wait for: synchronise the device first."""
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        fn()
+    stream.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+    stream.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_rows(args, md, device, stream, peak):
+    """Every step of the path on the workload it belongs to (one GPU)."""
+    from combine_warp_top_router_b200 import synth
+    rows = {}
+    reps = args.row_reps
+
+    def gbps(nbytes, ms):
+        return {"GBps": round(nbytes / (ms * 1e-3) / 1e9, 1), "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 3)}
+
+    # conventional dispatch and the two-stage (wire) combine, same workload as the headline
+    w = synth.make_workload(WORKLOAD, seed=args.seed, device=device)
+    T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
+    idx, gates = md.md_route_topk(w.logits, k)
+    for name, mode in (("conv", md.MD_CONV), ("dedup", md.MD_DEDUP)):
+        L = md.alloc_layout(T, E, k, R, mode, device)
+        wsp = md.alloc_workspace(md.dispatch_layout_workspace_size(T, E, k, R, mode), device)
+        buf = torch.empty(L.row_capacity, H, dtype=torch.bfloat16, device=device)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+        t_lay = _time(lambda: md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L,
+                                                      workspace=wsp, stream=stream), stream, reps)
+        n = int(L.n_rows.item())
+        t_perm = _time(lambda: md.md_dispatch_permute(w.x, L.row_of_slot, out=buf, stream=stream),
+                       stream, reps)
+        t_comb = _time(lambda: md.md_combine(w.y, L.assign_row, idx, gates, out=out, stream=stream),
+                       stream, reps)
+        pb = T * (2 * H + 4 * k) + n * 2 * H
+        cb = T * (2 * H * (k + 1) + 12 * k)
+        r = {"rows_per_token": round(n / T, 4), "layout_us": round(t_lay * 1e3, 2),
+             "permute_us": round(t_perm * 1e3, 2), "permute": gbps(pb, t_perm),
+             "combine_us": round(t_comb * 1e3, 2), "combine": gbps(cb, t_comb),
+             "dispatch_combine_Mtokens_per_s": round(T / ((t_lay + t_perm + t_comb) * 1e-3) / 1e6, 2)}
+        if mode == md.MD_DEDUP:
+            z = torch.empty(L.row_capacity, H, dtype=torch.bfloat16, device=device)
+            t_wire = _time(lambda: md.md_combine(w.y, L.assign_row, idx, gates, md.MD_COMBINE_WIRE,
+                                                 row_of_slot=L.row_of_slot, z=z, out=out,
+                                                 stream=stream), stream, reps)
+            wb = T * (2 * H * k + 2 * H + 16 * k) + n * 2 * H
+            r["combine_wire_us"] = round(t_wire * 1e3, 2)
+            r["combine_wire"] = gbps(wb, t_wire)
+            del z
+        rows[f"zipf_pairs_e128_k8_{name}"] = r
+        del L, wsp, buf, out
+    t_topk = _time(lambda: md.md_route_topk(w.logits, k, topk_idx=idx, topk_w=gates, stream=stream),
+                   stream, reps)
+    rows["route_topk_e128_k8"] = {"us": round(t_topk * 1e3, 2), **gbps(T * (4 * E + 8 * k), t_topk)}
+    del w, idx, gates
+    torch.cuda.empty_cache()
+
+    # token shuffle on the two-layer workload (C fitted on the first 4096 tokens)
+    w = synth.make_workload("two_layer_e128_k6", seed=args.seed, device=device)
+    a, _ = md.md_route_topk(w.logits, w.k)
+    b, _ = md.md_route_topk(w.logits_next, w.k)
+    _, C = md.md_coselect_stats(a, b, w.E, T_fit=w.fit_tokens, want_W=False)
+    sws = md.alloc_workspace(int(md.lib().md_token_shuffle_workspace_size(w.T, w.E, w.R)), device)
+    pred = torch.empty(w.T, dtype=torch.int32, device=device)
+    perm = torch.empty_like(pred)
+    inv = torch.empty_like(pred)
+    t_sh = _time(lambda: md.md_token_shuffle(a, C, w.expert_to_rank, w.R, pred, perm, inv,
+                                             workspace=sws, stream=stream), stream, reps)
+    xs = torch.empty_like(w.x)
+    t_g = _time(lambda: md.md_gather_rows(w.x, inv, out=xs, stream=stream), stream, reps)
+    loc_before = float((torch.arange(w.T, device=device) // (w.T // w.R)).eq(
+        w.expert_to_rank[b.long()].T).float().mean())
+    bs = b[inv.long()]
+    loc_after = float((torch.arange(w.T, device=device) // (w.T // w.R)).eq(
+        w.expert_to_rank[bs.long()].T).float().mean())
+    rows["token_shuffle_e128_k6"] = {
+        "T": w.T, "shuffle_us": round(t_sh * 1e3, 2), "gather_x_us": round(t_g * 1e3, 2),
+        "gather": gbps(2 * w.T * 2 * w.H + 4 * w.T, t_g),
+        "locality_before": round(loc_before, 4), "locality_after": round(loc_after, 4)}
+    del w, a, b, C, sws, xs
+    torch.cuda.empty_cache()
+
+    # the full pipeline at full size: T=262144, E=256, k=8, R=64
+    w = synth.make_workload("full_e256_k8", seed=args.seed, device=device)
+    T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
+    a = torch.empty(T, k, dtype=torch.int32, device=device)
+    g = torch.empty(T, k, dtype=torch.float32, device=device)
+    b = torch.empty_like(a)
+    gb = torch.empty_like(g)
+    W = torch.empty(E, E, dtype=torch.int32, device=device)
+    C = torch.empty_like(W)
+    p = torch.empty(E, dtype=torch.int32, device=device)
+    pws = md.alloc_workspace(int(md.lib().md_place_correlated_workspace_size(E, R)), device)
+    L = md.alloc_layout(T, E, k, R, md.MD_DEDUP, device)
+    lws = md.alloc_workspace(md.dispatch_layout_workspace_size(T, E, k, R, md.MD_DEDUP), device)
+    buf = torch.empty(L.row_capacity, H, dtype=torch.bfloat16, device=device)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+    parts = {}
+
+    def pipeline(ev=None):
+        steps = [
+            ("route_topk_x2", lambda: (md.md_route_topk(w.logits, k, topk_idx=a, topk_w=g, stream=stream),
+                                       md.md_route_topk(w.logits_next, k, topk_idx=b, topk_w=gb,
+                                                        stream=stream))),
+            ("coselect_W_C", lambda: md.md_coselect_stats(a, b, E, W=W, C=C, stream=stream)),
+            ("place_correlated", lambda: md.md_place_correlated(W, R, out=p, workspace=pws,
+                                                                stream=stream)),
+            ("dispatch_layout", lambda: md.md_dispatch_layout(a, E, R, p, md.MD_DEDUP, out=L,
+                                                              workspace=lws, stream=stream)),
+            ("dispatch_permute", lambda: md.md_dispatch_permute(w.x, L.row_of_slot, out=buf,
+                                                                stream=stream)),
+            ("combine", lambda: md.md_combine(w.y, L.assign_row, a, g, out=out, stream=stream)),
+        ]
+        for name, fn in steps:
+            if ev is None:
+                fn()
+                continue
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            ev.append((name, e0, e1))
+
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        pipeline()
+    stream.synchronize()
+    evs = []
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, reps // 5)):
+            pipeline(evs)
+    stream.synchronize()
+    for name, e0, e1 in evs:
+        parts[name] = parts.get(name, 0.0) + e0.elapsed_time(e1) / max(1, reps // 5)
+    total = sum(parts.values())
+    n = int(L.n_rows.item())
+    contiguous = synth.contiguous_placement(E, R, device)
+    torch.cuda.synchronize()
+    Lc = md.md_dispatch_layout(a, E, R, contiguous, md.MD_DEDUP)
+    rows["full_e256_k8_pipeline"] = {
+        "T": T, "ms": round(total, 3), "Mtokens_per_s": round(T / (total * 1e-3) / 1e6, 2),
+        "parts_us": {kk: round(v * 1e3, 1) for kk, v in parts.items()},
+        "rows_per_token_correlated": round(n / T, 4),
+        "rows_per_token_contiguous": round(int(Lc.n_rows.item()) / T, 4),
+        "permute": gbps(T * (2 * H + 4 * k) + n * 2 * H, parts["dispatch_permute"]),
+        "combine": gbps(T * (2 * H * (k + 1) + 12 * k), parts["combine"])}
+    del w, buf, out
+    torch.cuda.empty_cache()
+    return rows
 
 
 def run_e2e(args, md, w, mode, device, stream, idx, gates, L, wsp, buf, status, dist):
@@ -411,6 +577,9 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-sample-tokens", type=int, default=32768)
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
+    ap.add_argument("--rows", action=argparse.BooleanOptionalAction, default=True,
+                    help="also time every step of the path on its own workload")
+    ap.add_argument("--row-reps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
