@@ -3,9 +3,11 @@
 //
 // All three are bound by HBM bandwidth and move rows as 16-byte vectors, so
 // every warp instruction reads or writes 512 contiguous bytes of a row.
-//   permute  one warp per token, no block barriers; the next token's x row
-//            and row indices are loaded while the current token's stores
-//            drain.
+//   permute  rows of 1 KiB and more: TMA bulk copies through a per-warp
+//            ring of shared-memory slots (one bulk load per row piece, one
+//            bulk store per destination row).  Shorter rows: one warp per
+//            token, 16-byte vectors, the next token's x row and row indices
+//            loaded while the current token's stores drain.
 //   combine  a CTA takes kGroup tokens at a time: one warp per token orders
 //            its slots and stages (row, gate) in shared memory, then each
 //            thread issues the k 16-byte loads of its column chunk before the
@@ -91,6 +93,109 @@ __global__ void __launch_bounds__(kThreads)
             rows = nrows;
         }
     }
+}
+
+// Rows of 1 KiB and more move by TMA bulk copies instead: each warp runs its
+// own ring of kTmaStages 4 KiB shared-memory slots.  Lane 0 loads a piece of
+// x (up to 4 KiB of one row) into a slot with one bulk copy, kTmaAhead pieces
+// ahead, and writes it to each distinct destination row with one bulk store
+// per row; the other lanes resolve the token's distinct rows.  A slot is
+// reloaded only after the stores that read it have finished reading.
+constexpr int kTmaWarps = 4;
+constexpr int kTmaStages = 4;
+constexpr int kTmaAhead = 2;
+constexpr int kTmaPiece = 4096;
+constexpr int kTmaMinRowBytes = 1024;
+constexpr long long kTmaPolls = 1ll << 22;
+
+template <int KC>
+__global__ void __launch_bounds__(kTmaWarps * 32)
+    k_permute_tma(const char *__restrict__ x, int64_t T, int rowbytes, int pieces, int k,
+                  const int32_t *__restrict__ row_of_slot, int64_t out_rows, char *__restrict__ out,
+                  int32_t *status)
+{
+    extern __shared__ __align__(128) unsigned char tma_ring[];
+    __shared__ uint64_t bars[kTmaWarps][kTmaStages];
+    const int K = KC ? KC : k;
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+    unsigned char *ring = tma_ring + (size_t)wl * kTmaStages * kTmaPiece;
+    uint64_t *bar = bars[wl];
+    const int64_t U = T * pieces;  // units: (token, piece)
+    const int64_t gw = (int64_t)blockIdx.x * kTmaWarps + wl;
+    const int64_t nw = (int64_t)gridDim.x * kTmaWarps;
+    if (lane == 0) {
+        for (int st = 0; st < kTmaStages; ++st) md::mbar_init(&bar[st], 1);
+        md::fence_mbar_init();
+    }
+    __syncwarp();
+    if (gw >= U) return;
+
+    auto token_of = [&](int64_t u) { return pieces == 1 ? u : u / pieces; };
+    auto piece_of = [&](int64_t u) { return pieces == 1 ? 0 : (int)(u - (u / pieces) * pieces); };
+    auto bytes_of = [&](int64_t u) {
+        const int b = rowbytes - piece_of(u) * kTmaPiece;
+        return (uint32_t)(b < kTmaPiece ? b : kTmaPiece);
+    };
+    auto issue_load = [&](int64_t u, int st) {
+        const uint32_t nb = bytes_of(u);
+        md::mbar_expect_tx(&bar[st], nb);
+        md::bulk_load(ring + (size_t)st * kTmaPiece,
+                      x + token_of(u) * (int64_t)rowbytes + (int64_t)piece_of(u) * kTmaPiece, nb,
+                      &bar[st]);
+    };
+
+    if (lane == 0)
+        for (int j = 0; j < kTmaAhead; ++j)
+            if (gw + j * nw < U) issue_load(gw + j * nw, j % kTmaStages);
+    int rows = lane < K ? __ldg(row_of_slot + token_of(gw) * K + lane) : -1;
+
+    int64_t i = 0;
+    for (int64_t u = gw; u < U; u += nw, ++i) {
+        const int st = (int)(i % kTmaStages);
+        const int64_t ua = u + (int64_t)kTmaAhead * nw;
+        if (lane == 0 && ua < U) {
+            // slot of unit i + kTmaAhead was last read by the stores of unit
+            // i + kTmaAhead - kTmaStages
+            md::bulk_wait_read<kTmaStages - kTmaAhead - 1>();
+            issue_load(ua, (int)((i + kTmaAhead) % kTmaStages));
+        }
+        const int64_t un = u + nw;
+        const int nrows = (un < U && lane < K) ? __ldg(row_of_slot + token_of(un) * K + lane) : -1;
+
+        int ok = 1;
+        if (lane == 0) ok = md::mbar_wait_bounded(&bar[st], (uint32_t)((i / kTmaStages) & 1), kTmaPolls);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+            md::report(status, MD_ERR_TIMEOUT);
+            if (lane == 0) {
+                // wait, again bounded, for the loads still in flight
+                for (int j = 1; j <= kTmaAhead; ++j)
+                    if (u + j * nw < U)
+                        md::mbar_wait_bounded(&bar[(i + j) % kTmaStages],
+                                              (uint32_t)(((i + j) / kTmaStages) & 1), kTmaPolls);
+            }
+            break;
+        }
+        // distinct, in-range rows of this token (slots sharing a row write once)
+        const unsigned g = __match_any_sync(0xffffffffu, lane < K ? (unsigned)rows : (0x80000000u | lane));
+        const bool first = lane < K && (g & md::lanemask_lt()) == 0u;
+        const bool valid = rows >= 0 && rows < out_rows;
+        const int pc = piece_of(u);
+        if (first && !valid && pc == 0) md::report(status, MD_ERR_DATA);
+        unsigned todo = __ballot_sync(0xffffffffu, first && valid);
+        const uint32_t nb = bytes_of(u);
+        while (todo) {
+            const int j = __ffs(todo) - 1;
+            todo &= todo - 1;
+            const int64_t r = __shfl_sync(0xffffffffu, rows, j);
+            if (lane == 0)
+                md::bulk_store(out + r * rowbytes + (int64_t)pc * kTmaPiece,
+                               ring + (size_t)st * kTmaPiece, nb);
+        }
+        if (lane == 0) md::bulk_commit();
+        rows = nrows;
+    }
+    if (lane == 0) md::bulk_wait_all();
 }
 
 // ----------------------------------------------------------------- combine
@@ -248,6 +353,21 @@ template <int KC>
 void launch_permute(const void *x, int64_t T, int C, int k, const int32_t *rs, int64_t rows,
                     void *out, int32_t *st, cudaStream_t s)
 {
+    const int rowbytes = C * 16;
+    if (rowbytes >= kTmaMinRowBytes) {
+        const int pieces = (rowbytes + kTmaPiece - 1) / kTmaPiece;
+        const size_t smem = (size_t)kTmaWarps * kTmaStages * kTmaPiece;
+        cudaFuncSetAttribute(k_permute_tma<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        const int64_t units = T * pieces;
+        int64_t blocks = (units + kTmaWarps - 1) / kTmaWarps;
+        const int64_t cap = md::sm_count();
+        if (blocks > cap) blocks = cap;
+        k_permute_tma<KC><<<(unsigned)(blocks < 1 ? 1 : blocks), kTmaWarps * 32, smem, s>>>(
+            static_cast<const char *>(x), T, rowbytes, pieces, k, rs, rows, static_cast<char *>(out),
+            st);
+        return;
+    }
     static int per_sm = 0;
     if (per_sm == 0) {
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_permute<KC>, kThreads, 0);

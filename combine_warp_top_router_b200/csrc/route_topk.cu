@@ -77,13 +77,14 @@ __device__ __forceinline__ void load_row(float (&v)[M], const float *row, int E,
     }
 }
 
-template <int M, bool VEC>
+template <int M, bool VEC, int KC>
 __global__ void __launch_bounds__(kThreads)
-    k_route_topk(const float *__restrict__ logits, int64_t T, int E, int k, int gate_mode,
+    k_route_topk(const float *__restrict__ logits, int64_t T, int E, int k_rt, int gate_mode,
                  int32_t *__restrict__ out_idx, float *__restrict__ out_w)
 {
     __shared__ uint32_t s_ck[kWarps][32];
     __shared__ int s_ce[kWarps][32];
+    const int k = KC ? KC : k_rt;  // compile-time for the common k
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     const int G = 32 / k;  // tokens per warp group
     const int64_t warp0 = (int64_t)blockIdx.x * kWarps + wl;
@@ -125,7 +126,9 @@ __global__ void __launch_bounds__(kThreads)
 
             // threshold: the k-th largest lane maximum
             uint32_t act = best, th = 0;
-            for (int r = 0; r < k; ++r) {
+#pragma unroll
+            for (int r = 0; r < (KC ? KC : MD_MAX_TOPK); ++r) {
+                if (!KC && r >= k) break;
                 th = __reduce_max_sync(0xffffffffu, act);
                 const unsigned b = __ballot_sync(0xffffffffu, act == th);
                 if (lane == __ffs(b) - 1) act = 0u;
@@ -154,7 +157,9 @@ __global__ void __launch_bounds__(kThreads)
                 uint32_t ck = lane < ncand ? s_ck[wl][lane] : 0u;
                 const uint32_t ce = lane < ncand ? (uint32_t)s_ce[wl][lane] : 0xffffffffu;
                 __syncwarp();
-                for (int r = 0; r < k; ++r) {
+#pragma unroll
+                for (int r = 0; r < (KC ? KC : MD_MAX_TOPK); ++r) {
+                    if (!KC && r >= k) break;
                     const uint32_t kmax = __reduce_max_sync(0xffffffffu, ck);
                     const uint32_t cand = ck == kmax ? ce : 0xffffffffu;
                     const uint32_t emin = __reduce_min_sync(0xffffffffu, cand);
@@ -192,7 +197,9 @@ __global__ void __launch_bounds__(kThreads)
             den = my_den;
         } else {
             den = 0.0;
-            for (int r = 0; r < k; ++r) {
+#pragma unroll
+            for (int r = 0; r < (KC ? KC : MD_MAX_TOPK); ++r) {
+                if (!KC && r >= k) break;
                 const int src = base + r;
                 den += __shfl_sync(0xffffffffu, ex, src < 32 ? src : 0);
             }
@@ -204,7 +211,7 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
-template <int M, bool VEC>
+template <int M, bool VEC, int KC>
 void launch(const float *logits, int64_t T, int E, int k, int gate_mode, int32_t *idx, float *w,
             cudaStream_t s)
 {
@@ -213,8 +220,23 @@ void launch(const float *logits, int64_t T, int E, int k, int gate_mode, int32_t
     const int64_t cap = (int64_t)md::sm_count() * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
-    k_route_topk<M, VEC><<<(unsigned)blocks, kThreads, 0, s>>>(logits, T, E, k, gate_mode, idx, w);
+    k_route_topk<M, VEC, KC><<<(unsigned)blocks, kThreads, 0, s>>>(logits, T, E, k, gate_mode, idx, w);
     md::count_launches(1);
+}
+
+// 16-byte loads; the common k are compile-time constants
+template <int M>
+void launch_k(const float *logits, int64_t T, int E, int k, int gate_mode, int32_t *idx, float *w,
+              cudaStream_t s)
+{
+    switch (k) {
+    case 1: launch<M, true, 1>(logits, T, E, k, gate_mode, idx, w, s); break;
+    case 2: launch<M, true, 2>(logits, T, E, k, gate_mode, idx, w, s); break;
+    case 4: launch<M, true, 4>(logits, T, E, k, gate_mode, idx, w, s); break;
+    case 6: launch<M, true, 6>(logits, T, E, k, gate_mode, idx, w, s); break;
+    case 8: launch<M, true, 8>(logits, T, E, k, gate_mode, idx, w, s); break;
+    default: launch<M, true, 0>(logits, T, E, k, gate_mode, idx, w, s); break;
+    }
 }
 
 }  // namespace
@@ -231,20 +253,20 @@ extern "C" int md_route_topk(const float *logits, int64_t T, int E, int k, int g
     const bool vec = (E % 128 == 0) && md::aligned16(logits);
     if (vec) {
         switch (E / 128) {
-        case 1: launch<4, true>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
-        case 2: launch<8, true>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
+        case 1: launch_k<4>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
+        case 2: launch_k<8>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
         case 3:
-        case 4: launch<16, true>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
-        default: launch<32, true>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
+        case 4: launch_k<16>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
+        default: launch_k<32>(logits, T, E, k, gate_mode, topk_idx, topk_w, s); break;
         }
     } else {
         const int m = (E + 31) / 32;
-        if (m <= 1) launch<1, false>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
-        else if (m <= 2) launch<2, false>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
-        else if (m <= 4) launch<4, false>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
-        else if (m <= 8) launch<8, false>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
-        else if (m <= 16) launch<16, false>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
-        else launch<32, false>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
+        if (m <= 1) launch<1, false, 0>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
+        else if (m <= 2) launch<2, false, 0>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
+        else if (m <= 4) launch<4, false, 0>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
+        else if (m <= 8) launch<8, false, 0>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
+        else if (m <= 16) launch<16, false, 0>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
+        else launch<32, false, 0>(logits, T, E, k, gate_mode, topk_idx, topk_w, s);
     }
     return md::launch_status();
 }

@@ -18,11 +18,13 @@
 //                   histograms, a column scan, and a one-warp-per-tile
 //                   stable scatter using __match_any_sync.
 //   k_shuf_greedy   one CTA walks the sorted tokens 1024 at a time.  Each
-//                   token takes its first preferred rank that is not full.
-//                   Within a chunk the CTA finds the first position where a
-//                   rank reaches T/R, commits everything up to it, marks that
-//                   rank full and re-evaluates the rest of the chunk, which
-//                   gives exactly the sequential visit (at most R refills).
+//                   token takes its first preferred rank that is not full,
+//                   looked up per expert.  A chunk in which no rank reaches
+//                   T/R is committed at once; otherwise the CTA finds the
+//                   first position where a rank fills, commits up to it,
+//                   marks that rank full and re-evaluates the rest of the
+//                   chunk, which gives exactly the sequential visit (at most
+//                   R refills in all).
 //   bucket sort     stable partition by assigned rank gives perm / inv: rank
 //                   d's tokens take positions d*T/R .. in ascending t.
 #include <climits>
@@ -38,6 +40,7 @@ struct ShufWs {
     unsigned long long *num, *den; // [E]
     int32_t *cls;                  // [E]
     int32_t *order;                // [T]
+    int32_t *keys;                 // [T] bucket of each token in the current sort
     int32_t *tile_hist;            // [n_tiles * max(E+1, R)]
 };
 
@@ -57,6 +60,7 @@ size_t shuf_layout(int64_t T, int E, int R, ShufWs *w, void *base)
     x.den = reinterpret_cast<unsigned long long *>(take((size_t)E * 8));
     x.cls = reinterpret_cast<int32_t *>(take((size_t)E * 4));
     x.order = reinterpret_cast<int32_t *>(take((size_t)(T > 0 ? T : 1) * 4));
+    x.keys = reinterpret_cast<int32_t *>(take((size_t)(T > 0 ? T : 1) * 4));
     const int nbk = E + 1 > R ? E + 1 : R;
     x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)(n_tiles > 0 ? n_tiles : 1) * nbk * 4));
     if (w) *w = x;
@@ -159,10 +163,11 @@ __device__ __forceinline__ int bucket_key(int src, int64_t t, const int32_t *idx
     return d >= 0 && d < nbk ? d : 0;  // every token is assigned; keep bounds anyway
 }
 
+// Per-tile histograms; each token's bucket is also stored for the scatter.
 __global__ void __launch_bounds__(256)
     k_bucket_hist(int src, int64_t T, const int32_t *__restrict__ idx_l, int k,
                   const int32_t *__restrict__ cls, int E, const int32_t *__restrict__ pred, int nbk,
-                  int32_t *__restrict__ tile_hist)
+                  int32_t *__restrict__ keys, int32_t *__restrict__ tile_hist)
 {
     extern __shared__ int h[];
     for (int b = threadIdx.x; b < nbk; b += 256) h[b] = 0;
@@ -170,58 +175,90 @@ __global__ void __launch_bounds__(256)
     const int64_t t0 = (int64_t)blockIdx.x * kTile;
     for (int i = threadIdx.x; i < kTile; i += 256) {
         const int64_t t = t0 + i;
-        if (t < T) atomicAdd(&h[bucket_key(src, t, idx_l, k, cls, E, pred, nbk)], 1);
+        if (t < T) {
+            const int key = bucket_key(src, t, idx_l, k, cls, E, pred, nbk);
+            keys[t] = key;
+            atomicAdd(&h[key], 1);
+        }
     }
     __syncthreads();
     for (int b = threadIdx.x; b < nbk; b += 256) tile_hist[(int64_t)blockIdx.x * nbk + b] = h[b];
 }
 
-// tile_hist[tile][b] <- first output position of bucket b's items in tile
+// tile_hist[tile][b] <- first output position of bucket b's items in tile.
+// A warp scans one bucket's column over the tiles; then the bucket totals are
+// scanned and added.
 __global__ void __launch_bounds__(1024)
     k_bucket_scan(int32_t *__restrict__ tile_hist, int n_tiles, int nbk)
 {
     extern __shared__ int tot[];
-    for (int b = threadIdx.x; b < nbk; b += 1024) {
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+    for (int b = wp; b < nbk; b += 32) {
         int run = 0;
-        for (int i = 0; i < n_tiles; ++i) {
-            const int v = tile_hist[(int64_t)i * nbk + b];
-            tile_hist[(int64_t)i * nbk + b] = run;
-            run += v;
+        for (int i0 = 0; i0 < n_tiles; i0 += 32) {
+            const int i = i0 + lane;
+            const int v = i < n_tiles ? tile_hist[(int64_t)i * nbk + b] : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (i < n_tiles) tile_hist[(int64_t)i * nbk + b] = run + incl - v;
+            run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        tot[b] = run;
+        if (lane == 0) tot[b] = run;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int run = 0;
-        for (int b = 0; b < nbk; ++b) {
+    if (wp == 0) {
+        // exclusive scan of the bucket totals: lane L takes a contiguous run
+        const int per = (nbk + 31) / 32;
+        const int lo = lane * per, hi = min(nbk, lo + per);
+        int sum = 0;
+        for (int b = lo; b < hi; ++b) sum += tot[b];
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int run = incl - sum;
+        for (int b = lo; b < hi; ++b) {
             const int v = tot[b];
             tot[b] = run;
             run += v;
         }
     }
     __syncthreads();
-    for (int b = threadIdx.x; b < nbk; b += 1024) {
+    for (int b = wp; b < nbk; b += 32) {
         const int base = tot[b];
-        for (int i = 0; i < n_tiles; ++i) tile_hist[(int64_t)i * nbk + b] += base;
+        for (int i = lane; i < n_tiles; i += 32) tile_hist[(int64_t)i * nbk + b] += base;
     }
 }
 
-// One warp per tile: items in ascending t, stable within each bucket.
+// One warp per tile: items in ascending t, stable within each bucket.  The
+// tile's 1024 keys are loaded up front (32 per lane).
 __global__ void __launch_bounds__(32)
-    k_bucket_scatter(int src, int64_t T, const int32_t *__restrict__ idx_l, int k,
-                     const int32_t *__restrict__ cls, int E, const int32_t *__restrict__ pred,
-                     int nbk, const int32_t *__restrict__ tile_hist, int32_t *__restrict__ order,
+    k_bucket_scatter(int src, int64_t T, int nbk, const int32_t *__restrict__ keys,
+                     const int32_t *__restrict__ tile_hist, int32_t *__restrict__ order,
                      int32_t *__restrict__ perm, int32_t *__restrict__ inv)
 {
     extern __shared__ int cnt[];
     const int lane = threadIdx.x;
     for (int b = lane; b < nbk; b += 32) cnt[b] = tile_hist[(int64_t)blockIdx.x * nbk + b];
-    __syncwarp();
     const int64_t t0 = (int64_t)blockIdx.x * kTile;
-    for (int c = 0; c < kTile; c += 32) {
-        const int64_t t = t0 + c + lane;
-        const bool in = t < T;
-        const int key = in ? bucket_key(src, t, idx_l, k, cls, E, pred, nbk) : -1;
+    int kv[kTile / 32];
+#pragma unroll
+    for (int c = 0; c < kTile / 32; ++c) {
+        const int64_t t = t0 + c * 32 + lane;
+        kv[c] = t < T ? keys[t] : -1;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < kTile / 32; ++c) {
+        const int64_t t = t0 + c * 32 + lane;
+        const int key = kv[c];
+        const bool in = key >= 0;
         const unsigned g = __match_any_sync(0xffffffffu, in ? (unsigned)key : (0x80000000u | lane));
         int pos = 0;
         if (in) pos = cnt[key] + __popc(g & md::lanemask_lt());
@@ -240,82 +277,184 @@ __global__ void __launch_bounds__(32)
 }
 
 // ----------------------------------------------------------------- greedy
-__global__ void __launch_bounds__(1024)
+// A token's choice depends only on its top-1 expert and on which ranks are
+// full, and the set of full ranks changes at most R times.  So the CTA keeps
+// first[e] = the first rank in e's preference list that is not full (-1 for
+// an empty row), and walks the sorted tokens 1024 at a time:
+//   every token looks up its choice; the chunk's per-rank totals are added
+//   up (one shared atomic per warp and rank); if no rank goes past T/R the
+//   whole chunk is committed at once.  Otherwise the first position where a
+//   rank reaches T/R is found from per-warp counts, the chunk is committed up
+//   to it, that rank is marked full, first[] is recomputed and the rest of
+//   the chunk is re-evaluated: exactly the sequential visit.
+constexpr int kGreedyThreads = 1024;
+constexpr int kGreedyWarps = kGreedyThreads / 32;
+
+__global__ void __launch_bounds__(kGreedyThreads, 1)
     k_shuf_greedy(const int32_t *__restrict__ order, const int32_t *__restrict__ idx_l, int k,
                   ShufWs ws, int64_t T, int E, int R, int64_t Tr, int32_t *__restrict__ pred,
                   int32_t *status)
 {
+    extern __shared__ __align__(16) unsigned char g_raw[];
+    int *s_first = reinterpret_cast<int *>(g_raw);                    // [E]
+    unsigned char *s_pref = g_raw + (size_t)E * sizeof(int);          // [E*R]
     __shared__ long long s_load[MD_MAX_RANKS];
+    __shared__ int s_tot[MD_MAX_RANKS];
+    __shared__ int s_cnt[kGreedyWarps][MD_MAX_RANKS];
+    __shared__ unsigned s_msk[kGreedyWarps][MD_MAX_RANKS];
     __shared__ unsigned long long s_full;
-    __shared__ int s_cnt[32][MD_MAX_RANKS];
-    __shared__ int s_pmin;
+    __shared__ int s_first_any, s_over, s_pmin;
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
-    for (int d = tid; d < R; d += 1024) s_load[d] = 0;
-    if (tid == 0) s_full = 0ull;
+
+    for (int i = tid; i < E * R; i += kGreedyThreads) s_pref[i] = (unsigned char)ws.pref[i];
+    for (int d = tid; d < R; d += kGreedyThreads) {
+        s_load[d] = 0;
+        s_tot[d] = 0;
+    }
+    if (tid == 0) {
+        s_full = 0ull;
+        s_first_any = 0;
+    }
+    __syncthreads();
+    for (int e = tid; e < E; e += kGreedyThreads)
+        s_first[e] = ws.den[e] == 0ull ? -1 : (int)s_pref[(size_t)e * R];
     __syncthreads();
 
-    for (int64_t base = 0; base < T; base += 1024) {
+    // token ids are fetched two chunks ahead and their top-1 experts one chunk
+    // ahead, so neither load is waited on in the chunk that uses it
+    auto token_at = [&](int64_t base) -> int64_t {
         const int64_t pos = base + tid;
-        const bool have = pos < T;
-        const int64_t t = have ? order[pos] : 0;
-        int e1 = have ? idx_l[t * k] : 0;
-        bool empty_row = true;
-        if (have) {
-            if (e1 < 0 || e1 >= E) {
-                md::report(status, MD_ERR_DATA);
-                e1 = 0;
-            } else {
-                empty_row = ws.den[e1] == 0ull;
-            }
+        return pos < T ? (int64_t)order[pos] : -1;
+    };
+    int64_t t_n1 = token_at(0);
+    int e_n1 = t_n1 >= 0 ? idx_l[t_n1 * k] : 0;
+    int64_t t_n2 = token_at(kGreedyThreads);
+
+    for (int64_t base = 0; base < T; base += kGreedyThreads) {
+        const int64_t t = t_n1;
+        int e1 = e_n1;
+        t_n1 = t_n2;
+        e_n1 = t_n1 >= 0 ? idx_l[t_n1 * k] : 0;
+        t_n2 = token_at(base + 2 * kGreedyThreads);
+        const bool have = t >= 0;
+        if (have && (e1 < 0 || e1 >= E)) {
+            md::report(status, MD_ERR_DATA);
+            e1 = 0;
         }
-        const int src_rank = (int)(t / Tr);
+        const int src_rank = have ? (int)(t / Tr) : 0;
         int start = 0;
         while (true) {
-            const unsigned long long full = s_full;
+            // choice under the current set of full ranks
             int ch = -1;
             if (have && tid >= start) {
-                if (empty_row) {
-                    if (!((full >> src_rank) & 1ull)) {
-                        ch = src_rank;
-                    } else {
-                        for (int d = 0; d < R; ++d)
-                            if (!((full >> d) & 1ull)) { ch = d; break; }
-                    }
-                } else {
-                    const int32_t *pl = ws.pref + (int64_t)e1 * R;
-                    for (int n = 0; n < R; ++n) {
-                        const int d = pl[n];
-                        if (!((full >> d) & 1ull)) { ch = d; break; }
-                    }
-                }
+                const int f = s_first[e1];
+                ch = f >= 0 ? f : (((s_full >> src_rank) & 1ull) ? s_first_any : src_rank);
             }
             const unsigned g =
                 __match_any_sync(0xffffffffu, ch >= 0 ? (unsigned)ch : (0x80000000u | lane));
-            const int r_in = __popc(g & md::lanemask_lt());
-            for (int i = tid; i < 32 * MD_MAX_RANKS; i += 1024) (&s_cnt[0][0])[i] = 0;
+            const bool leader = ch >= 0 && (g & md::lanemask_lt()) == 0u;
+            if (leader) atomicAdd(&s_tot[ch], __popc(g));
+            if (tid == 0) s_over = 0;
+            __syncthreads();
+            for (int d = tid; d < R; d += kGreedyThreads)
+                if (s_load[d] + s_tot[d] > Tr) s_over = 1;
+            __syncthreads();
+            if (!s_over) {
+                // no rank goes past T/R: commit the whole chunk
+                if (ch >= 0) pred[t] = ch;
+                int newly_full = 0;
+                for (int d = tid; d < R; d += kGreedyThreads) {
+                    s_load[d] += s_tot[d];
+                    s_tot[d] = 0;
+                    if (s_load[d] == Tr && !((s_full >> d) & 1ull)) newly_full = 1;
+                }
+                if (__syncthreads_or(newly_full)) {
+                    if (tid == 0) {
+                        unsigned long long f = s_full;
+                        for (int d = 0; d < R; ++d)
+                            if (s_load[d] == Tr) f |= 1ull << d;
+                        s_full = f;
+                    }
+                    __syncthreads();
+                    for (int e = tid; e < E; e += kGreedyThreads) {
+                        if (s_first[e] < 0) continue;
+                        const unsigned char *pl = s_pref + (size_t)e * R;
+                        int n = 0;
+                        while (n < R && ((s_full >> pl[n]) & 1ull)) ++n;
+                        s_first[e] = n < R ? (int)pl[n] : 0;
+                    }
+                    if (tid == 0) {
+                        int d = 0;
+                        while (d < R && ((s_full >> d) & 1ull)) ++d;
+                        s_first_any = d < R ? d : 0;
+                    }
+                    __syncthreads();
+                }
+                break;
+            }
+            // some rank goes past T/R: find the first position where a rank fills
+            for (int i = tid; i < kGreedyWarps * MD_MAX_RANKS; i += kGreedyThreads)
+                (&s_cnt[0][0])[i] = 0;
             if (tid == 0) s_pmin = INT_MAX;
             __syncthreads();
-            if (ch >= 0 && (g >> lane) == 1u) s_cnt[wp][ch] = __popc(g);
+            if (leader) {
+                s_cnt[wp][ch] = __popc(g);
+                s_msk[wp][ch] = g;
+            }
             __syncthreads();
-            for (int d = tid; d < R; d += 1024) {
-                int run = 0;
-                for (int w2 = 0; w2 < 32; ++w2) {
-                    const int c = s_cnt[w2][d];
-                    s_cnt[w2][d] = run;
-                    run += c;
+            for (int d = wp; d < R; d += kGreedyWarps) {
+                // ranks that fill inside this chunk (full ranks get no tokens)
+                if (s_tot[d] == 0 || s_load[d] + s_tot[d] < Tr) continue;
+                const long long need = Tr - s_load[d];  // tokens rank d still takes
+                int c = s_cnt[lane][d];
+                int incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+                const int w = __ffs(hit) - 1;  // the warp holding the filling token
+                if (lane == w) {
+                    // the nth (1-based) token of warp w that chose d fills it
+                    const int nth = (int)(need - (incl - c));
+                    unsigned m = s_msk[w][d];
+                    for (int i = 1; i < nth; ++i) m &= m - 1u;
+                    atomicMin(&s_pmin, w * 32 + __ffs(m) - 1);
                 }
             }
             __syncthreads();
-            if (ch >= 0 && s_load[ch] + s_cnt[wp][ch] + r_in + 1 == Tr) atomicMin(&s_pmin, tid);
-            __syncthreads();
             const int pmin = s_pmin;
-            if (ch >= 0 && tid <= pmin) {
-                pred[t] = ch;
-                atomicAdd(reinterpret_cast<unsigned long long *>(&s_load[ch]), 1ull);
-            }
-            if (tid == pmin) s_full |= 1ull << ch;
+            const bool commit = ch >= 0 && tid <= pmin;
+            if (commit) pred[t] = ch;
+            const unsigned g2 =
+                __match_any_sync(0xffffffffu, commit ? (unsigned)ch : (0x80000000u | lane));
+            if (commit && (g2 & md::lanemask_lt()) == 0u)
+                atomicAdd(reinterpret_cast<unsigned long long *>(&s_load[ch]),
+                          (unsigned long long)__popc(g2));
+            for (int d = tid; d < R; d += kGreedyThreads) s_tot[d] = 0;
             __syncthreads();
-            if (pmin == INT_MAX || pmin >= 1023) break;
+            if (tid == 0) {
+                unsigned long long f = s_full;
+                for (int d = 0; d < R; ++d)
+                    if (s_load[d] == Tr) f |= 1ull << d;
+                s_full = f;
+            }
+            __syncthreads();
+            for (int e = tid; e < E; e += kGreedyThreads) {
+                if (s_first[e] < 0) continue;
+                const unsigned char *pl = s_pref + (size_t)e * R;
+                int n = 0;
+                while (n < R && ((s_full >> pl[n]) & 1ull)) ++n;
+                s_first[e] = n < R ? (int)pl[n] : 0;
+            }
+            if (tid == 0) {
+                int d = 0;
+                while (d < R && ((s_full >> d) & 1ull)) ++d;
+                s_first_any = d < R ? d : 0;
+            }
+            __syncthreads();
+            if (pmin >= kGreedyThreads - 1) break;
             start = pmin + 1;
         }
     }
@@ -355,18 +494,22 @@ extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
     // visit order: by confidence class, then t
     const int nbk0 = E + 1;
     k_bucket_hist<<<n_tiles, 256, nbk0 * sizeof(int), s>>>(0, T, idx_l, k, ws.cls, E, nullptr, nbk0,
-                                                          ws.tile_hist);
+                                                          ws.keys, ws.tile_hist);
     k_bucket_scan<<<1, 1024, nbk0 * sizeof(int), s>>>(ws.tile_hist, n_tiles, nbk0);
-    k_bucket_scatter<<<n_tiles, 32, nbk0 * sizeof(int), s>>>(0, T, idx_l, k, ws.cls, E, nullptr,
-                                                            nbk0, ws.tile_hist, ws.order, nullptr,
-                                                            nullptr);
-    k_shuf_greedy<<<1, 1024, 0, s>>>(ws.order, idx_l, k, ws, T, E, R, Tr, pred_rank, dev_status);
+    k_bucket_scatter<<<n_tiles, 32, nbk0 * sizeof(int), s>>>(0, T, nbk0, ws.keys, ws.tile_hist,
+                                                            ws.order, nullptr, nullptr);
+    const size_t gsm = (size_t)E * sizeof(int) + (size_t)E * R;
+    if (cudaFuncSetAttribute(k_shuf_greedy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm) !=
+        cudaSuccess)
+        return MD_ERR_CUDA;
+    k_shuf_greedy<<<1, kGreedyThreads, gsm, s>>>(ws.order, idx_l, k, ws, T, E, R, Tr, pred_rank,
+                                                 dev_status);
     // new positions: stable partition by assigned rank
     k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
-                                                       ws.tile_hist);
+                                                       ws.keys, ws.tile_hist);
     k_bucket_scan<<<1, 1024, R * sizeof(int), s>>>(ws.tile_hist, n_tiles, R);
-    k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
-                                                         ws.tile_hist, nullptr, perm, inv);
+    k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, R, ws.keys, ws.tile_hist, nullptr,
+                                                         perm, inv);
     md::count_launches(9);
     return md::launch_status();
 }

@@ -108,8 +108,30 @@ def test_generic_k(k):
     assert np.array_equal(bits(z), wz)
 
 
-def test_bad_rows_are_skipped_and_reported():
-    T, H, k = 64, 16, 2
+# rows of 1 KiB and more move by bulk copies in pieces of at most 4 KiB:
+# just under and at that size, a 16-byte last piece, three pieces; several k
+# (5 has no specialised kernel)
+@pytest.mark.parametrize("H", [504, 512, 2056, 4104])
+@pytest.mark.parametrize("k", [2, 5, 8, 32])
+def test_permute_row_pieces(H, k):
+    T, E, R = 300, 64, 4
+    idx = oracle.route_topk(synth.normal_f32(T, E, H + k, 1).numpy(), k)[0]
+    L = oracle.dispatch_layout(idx, E, R, shuffled_placement(E, R, 6), 1)
+    x = synth.normal_bf16(T, H, k, 3)
+    n = L["n_rows"]
+    out = from_bits(np.full((n + 3, H), POISON_BITS, np.uint16))
+    st = md.new_status(DEV)
+    md.md_dispatch_permute(x.to(DEV), i32(L["row_of_slot"]), out=out, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == md.MD_OK
+    got = bits(out)
+    assert np.array_equal(got[:n], oracle.dispatch_permute(bits(x), L["row_token"]))
+    assert np.all(got[n:] == POISON_BITS)
+
+
+@pytest.mark.parametrize("H", [16, 1024])
+def test_bad_rows_are_skipped_and_reported(H):
+    T, k = 64, 2
     x = synth.normal_bf16(T, H, 0, 3).to(DEV)
     rows = torch.arange(T * k, dtype=torch.int32, device=DEV).view(T, k)
     rows[3, 1] = 10_000

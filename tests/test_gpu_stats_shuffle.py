@@ -86,6 +86,29 @@ def test_placement_small_and_unrefined():
             assert np.array_equal(p.cpu().numpy(), oracle.place_correlated(W, 3, seed_mode, refine))
 
 
+def _random_w(E, seed, hi):
+    rng = np.random.default_rng(seed)
+    W = np.triu(rng.integers(0, hi, size=(E, E)), 1).astype(np.uint32)
+    W = W + W.T
+    W[np.arange(E), np.arange(E)] = rng.integers(0, 4 * hi, size=E).astype(np.uint32)
+    return W
+
+
+# small value ranges force many equal weights and gains (tie rules); E=1024
+# covers the largest tables, R=16 keeps A (E x R) in shared memory and R=64
+# puts it in the workspace; E/R=1 and R=1 leave nothing to swap
+@pytest.mark.parametrize("E,R,hi", [(8, 2, 3), (16, 4, 2), (64, 64, 5), (64, 8, 1000),
+                                    (256, 2, 7), (256, 64, 4), (1024, 16, 9), (1024, 64, 50),
+                                    (128, 1, 5)])
+@pytest.mark.parametrize("seed_mode", [0, 1])
+def test_placement_random_weights(E, R, hi, seed_mode):
+    W = _random_w(E, E * 7 + R, hi)
+    p = md.md_place_correlated(torch.from_numpy(W.view(np.int32)).to(DEV), R, seed_mode)
+    torch.cuda.synchronize()
+    want = oracle.place_correlated(W, R, seed_mode)
+    assert np.array_equal(p.cpu().numpy(), want)
+
+
 def _shuffle_both(a, C, p, R):
     pred, perm, inv = md.md_token_shuffle(i32(a), torch.from_numpy(C.view(np.int32)).to(DEV), i32(p), R)
     torch.cuda.synchronize()
@@ -100,6 +123,23 @@ def test_shuffle_matches_oracle(name, T, R):
     _, C = oracle.coselect(a, b, w.E, T_fit=min(T, 4096))
     C[5, :] = 0  # an empty row
     p = shuffled_placement(w.E, R, 4)
+    got, want = _shuffle_both(a, C, p, R)
+    for g, o in zip(got, want):
+        assert np.array_equal(g, o)
+
+
+# counts skewed toward a few ranks, so that ranks fill one after another in
+# the middle of chunks and most tokens fall back down their preference lists
+@pytest.mark.parametrize("E,k,R,T", [(64, 2, 64, 64 * 40), (128, 6, 16, 16 * 700), (1024, 8, 64, 64 * 80),
+                                     (32, 1, 4, 4 * 1000), (16, 3, 2, 2 * 2500)])
+def test_shuffle_skewed_counts(E, k, R, T):
+    rng = np.random.default_rng(E + R)
+    C = rng.integers(0, 3, size=(E, E)).astype(np.uint32)
+    hot = rng.choice(E, size=max(1, E // 16), replace=False)
+    C[:, hot] += 40
+    C[rng.choice(E, size=max(1, E // 10), replace=False), :] = 0  # empty rows
+    a = oracle.route_topk(synth.normal_f32(T, E, 3, 7).numpy(), k)[0]
+    p = shuffled_placement(E, R, 9)
     got, want = _shuffle_both(a, C, p, R)
     for g, o in zip(got, want):
         assert np.array_equal(g, o)
