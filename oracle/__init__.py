@@ -58,6 +58,7 @@ def _load():
             lib.oracle_dispatch_layout.argtypes = [P, I64, I32, I32, I32, P, I32,
                                                    P, P, P, P, P, P, P, P, P]
             lib.oracle_dispatch_permute.argtypes = [P, I64, I64, P, I64, P]
+            lib.oracle_dedup_expand.argtypes = [P, I64, I64, P, P, I64, I32, I64, P]
             lib.oracle_combine.argtypes = [P, I64, P, P, P, I64, I32, I64, I32, P, I32, P, P, P]
             lib.oracle_coselect.argtypes = [P, P, I64, I32, I32, P, P, I32]
             lib.oracle_placement_objective.argtypes = [P, I32, P]
@@ -65,6 +66,7 @@ def _load():
             lib.oracle_place_correlated.argtypes = [P, I32, I32, I32, I32, P]
             lib.oracle_token_shuffle.argtypes = [P, P, P, I64, I32, I32, I32, P, P, P]
             for name in ("oracle_route_topk", "oracle_dispatch_layout", "oracle_dispatch_permute",
+                         "oracle_dedup_expand",
                          "oracle_combine", "oracle_coselect", "oracle_place_correlated",
                          "oracle_token_shuffle"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -134,6 +136,24 @@ def dispatch_permute(x_bits, row_token):
     rt = _c(row_token, np.int32)
     out = np.empty((rt.shape[0], H), np.uint16)
     _check(lib.oracle_dispatch_permute(_ptr(x), T, H, _ptr(rt), rt.shape[0], _ptr(out)), "permute")
+    return out
+
+
+def dedup_expand(wire_bits, row_of_slot, assign_row, n_out=None):
+    """Receiver-side expand: out[assign_row[t, j]] = wire[row_of_slot[t, j]].
+
+    wire_bits uint16 [n_wire, H]; row_of_slot, assign_row int32 [T, k] ->
+    out uint16 [n_out, H] (n_out defaults to T * k)."""
+    lib = _load()
+    wire = _c(wire_bits, np.uint16)
+    n_wire, H = wire.shape
+    rs = _c(row_of_slot, np.int32)
+    ar = _c(assign_row, np.int32)
+    T, k = rs.shape
+    n_out = T * k if n_out is None else int(n_out)
+    out = np.zeros((n_out, H), np.uint16)
+    _check(lib.oracle_dedup_expand(_ptr(wire), n_wire, H, _ptr(rs), _ptr(ar), T, k, n_out, _ptr(out)),
+           "dedup_expand")
     return out
 
 

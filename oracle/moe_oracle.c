@@ -295,6 +295,29 @@ int oracle_dispatch_permute(const uint16_t *x, int64_t T, int64_t H,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Receiver-side expand of deduplicated rows.                                */
+/* [EC] Method 1, Deduplicating Dispatcher: a rank receives one row per      */
+/* (token, rank) carrying all of the token's experts on that rank; each of   */
+/* those experts needs its own copy of the row.  Slot j of token t goes to   */
+/* its conventional (expert-grouped) position assign_row[t][j], copied from  */
+/* the deduplicated row row_of_slot[t][j] that carried it.                   */
+/* ------------------------------------------------------------------------ */
+
+int oracle_dedup_expand(const uint16_t *wire, int64_t n_wire, int64_t H,
+                        const int32_t *row_of_slot, const int32_t *assign_row, int64_t T, int k,
+                        int64_t n_out, uint16_t *out)
+{
+    if (T < 0 || H < 1 || k < 1 || n_wire < 0 || n_out < 0) return 1;
+    for (int64_t t = 0; t < T; ++t)
+        for (int j = 0; j < k; ++j) {
+            int64_t src = row_of_slot[t * k + j], dst = assign_row[t * k + j];
+            if (src < 0 || src >= n_wire || dst < 0 || dst >= n_out) return 1;
+            memcpy(out + dst * H, wire + src * H, sizeof(uint16_t) * (size_t)H);
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Combine.                                                                  */
 /* [DD] "Send matrices": combine returns the same volumes in reverse.        */
 /* [EC] "The Communication Bottleneck": dispatch and combine per MoE layer.  */

@@ -135,3 +135,43 @@ def test_wire_with_one_expert_per_rank():
     for i in range(k):
         acc = acc + zb[torch.arange(T), torch.from_numpy(order[:, i])].float()
     assert np.array_equal(wire, _bits(acc.to(torch.bfloat16)))
+
+
+# ---------------------------------------------------------------- dedup expand
+# "Expert Coupling in MoE Pretraining", Method 1: the deduplicating dispatcher
+# delivers the same rows as the conventional one, once per (token, rank); the
+# receiver copies each into one row per selected expert.  So expanding the
+# dedup dispatch buffer must give the conventional dispatch buffer exactly.
+
+@pytest.mark.parametrize("T,E,k,R", [(256, 32, 4, 8), (160, 64, 6, 16), (64, 16, 8, 2), (96, 8, 1, 4)])
+def test_expand_of_dedup_dispatch_is_conventional_dispatch(T, E, k, R):
+    lg = synth.group_boost_logits(T, E, 2, 3.0, 1, 1, 5, 6).numpy()
+    idx, _ = oracle.route_topk(lg, k)
+    p = np.random.default_rng(T + E).permutation(synth.contiguous_placement(E, R).numpy()).astype(np.int32)
+    Ld = oracle.dispatch_layout(idx, E, R, p, 1)
+    Lc = oracle.dispatch_layout(idx, E, R, p, 0)
+    x = _bits(synth.normal_bf16(T, 24, 2, 3))
+    wire = oracle.dispatch_permute(x, Ld["row_token"])
+    conv = oracle.dispatch_permute(x, Lc["row_token"])
+    # the dedup layout's assign_row is the conventional position of each slot
+    assert np.array_equal(Ld["assign_row"], Lc["row_of_slot"])
+    out = oracle.dedup_expand(wire, Ld["row_of_slot"], Ld["assign_row"])
+    assert np.array_equal(out, conv)
+
+
+def test_expand_hand_example():
+    # two tokens, k=2; token 0 -> rows (wire 0, wire 0) to conv rows 2, 0;
+    # token 1 -> (wire 1, wire 2) to conv rows 1, 3
+    wire = np.array([[1, 2], [3, 4], [5, 6]], np.uint16)
+    rs = np.array([[0, 0], [1, 2]], np.int32)
+    ar = np.array([[2, 0], [1, 3]], np.int32)
+    out = oracle.dedup_expand(wire, rs, ar)
+    assert out.tolist() == [[1, 2], [3, 4], [1, 2], [5, 6]]
+
+
+def test_expand_rejects_bad_rows():
+    wire = np.zeros((2, 4), np.uint16)
+    with pytest.raises(ValueError):
+        oracle.dedup_expand(wire, np.array([[0, 2]], np.int32), np.array([[0, 1]], np.int32))
+    with pytest.raises(ValueError):
+        oracle.dedup_expand(wire, np.array([[0, 1]], np.int32), np.array([[0, 2]], np.int32))
