@@ -264,6 +264,8 @@ def run_native(args):
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+        "dispatch_combine_excl_router": round(
+            T * ws / ((per["dispatch_layout"] + per["dispatch_permute"] + per["combine"]) * 1e-3) / 1e6, 3),
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "T": T, "H": H, "E": E, "top_k": k, "ep_ranks": R,
                    "dispatch": args.dispatch, "combine": "fused", "gates": "topk_softmax",
@@ -347,6 +349,14 @@ def run_rows(args, md, device, stream, peak):
             r["combine_wire_us"] = round(t_wire * 1e3, 2)
             r["combine_wire"] = gbps(wb, t_wire)
             del z
+            # receiver side: dedup rows -> one row per (token, expert), expert-grouped
+            xc = torch.empty(T * k, H, dtype=torch.bfloat16, device=device)
+            t_exp = _time(lambda: md.md_dedup_expand(buf, L.row_of_slot, L.assign_row, out=xc,
+                                                     stream=stream), stream, reps)
+            eb = n * 2 * H + T * k * (2 * H + 8)
+            r["dedup_expand_us"] = round(t_exp * 1e3, 2)
+            r["dedup_expand"] = gbps(eb, t_exp)
+            del xc
         rows[f"zipf_pairs_e128_k8_{name}"] = r
         del L, wsp, buf, out
     t_topk = _time(lambda: md.md_route_topk(w.logits, k, topk_idx=idx, topk_w=gates, stream=stream),

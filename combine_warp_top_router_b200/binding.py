@@ -41,6 +41,7 @@ _SIGNATURES = {
     "md_dispatch_layout_noalloc": ([_P, _L, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                                     _P, _P, _P], _I),
     "md_dispatch_permute": ([_P, _L, _I, _I, _P, _L, _P, _P, _P], _I),
+    "md_dedup_expand": ([_P, _L, _I, _P, _P, _L, _I, _L, _P, _P, _P], _I),
     "md_combine": ([_P, _L, _P, _P, _P, _L, _I, _I, _I, _P, _L, _P, _P, _P, _P], _I),
     "md_coselect_stats": ([_P, _P, _L, _I, _I, _P, _P, _I, _P, _P], _I),
     "md_place_correlated_workspace_size": ([_I, _I], _S),
@@ -237,6 +238,25 @@ def md_dispatch_permute(x, row_of_slot, out_rows=None, out=None, dev_status=None
     rc = lib().md_dispatch_permute(_ptr(x), T, H, k, _ptr(row_of_slot), out.shape[0], _ptr(out),
                                    _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_dispatch_permute")
+    return out
+
+
+def md_dedup_expand(wire, row_of_slot, assign_row, out_rows=None, out=None, dev_status=None,
+                    stream=None):
+    """out[assign_row[t, j]] = wire[row_of_slot[t, j]]: dedup rows to expert-grouped rows."""
+    _need(wire, "wire", torch.bfloat16)
+    dev = wire.device
+    _need(row_of_slot, "row_of_slot", torch.int32, dev)
+    _need(assign_row, "assign_row", torch.int32, dev)
+    T, k = row_of_slot.shape
+    H = wire.shape[1]
+    if out is None:
+        out = torch.empty(out_rows if out_rows is not None else T * k, H, dtype=torch.bfloat16,
+                          device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    rc = lib().md_dedup_expand(_ptr(wire), wire.shape[0], H, _ptr(row_of_slot), _ptr(assign_row), T,
+                               k, out.shape[0], _ptr(out), _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_dedup_expand")
     return out
 
 

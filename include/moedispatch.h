@@ -194,6 +194,27 @@ int md_dispatch_permute(const void *x, int64_t T, int H, int k,
                         int32_t *dev_status, void *stream);
 
 /*
+ * md_dedup_expand -- receiver-side expand of deduplicated rows.
+ * "Expert Coupling ...", Method 1 (Deduplicating Dispatcher): a rank receives
+ * one row per (token, rank) carrying all of the token's experts on that rank;
+ * every selected expert then gets its own copy of the row, in the
+ * conventional expert-grouped order (p[e], e, t) a grouped GEMM consumes.
+ *
+ *   wire         bf16  [n_wire, H]   dedup dispatch buffer (md_dispatch_permute
+ *                                    with a MD_DEDUP layout)
+ *   row_of_slot  int32 [T, k]        dedup row of each slot   } both from one
+ *   assign_row   int32 [T, k]        conventional row of each } MD_DEDUP layout
+ *   out          bf16  [out_rows, H] out[assign_row[t][j]] = wire[row_of_slot[t][j]]
+ *                                    bit for bit; out_rows >= T*k for a full layout
+ *   wire and out 16-byte aligned, H % 8 == 0.  A slot whose source or
+ *   destination row is out of range is skipped and reported (MD_ERR_DATA).
+ *   The result equals md_dispatch_permute with the conventional layout.
+ */
+int md_dedup_expand(const void *wire, int64_t n_wire, int H, const int32_t *row_of_slot,
+                    const int32_t *assign_row, int64_t T, int k, int64_t out_rows, void *out,
+                    int32_t *dev_status, void *stream);
+
+/*
  * md_combine -- gate-weighted combine of the expert outputs.
  * "DODOCO ...", send_matrices.csv: combine, the second AlltoAll of each MoE
  * layer, returns the volumes of dispatch in reverse.  "Expert Coupling ...",

@@ -19,7 +19,8 @@ def _declared():
 def test_header_declares_the_entry_points():
     names = _declared()
     for n in ("md_route_topk", "md_dispatch_layout", "md_dispatch_permute", "md_combine",
-              "md_coselect_stats", "md_token_shuffle", "md_place_correlated", "md_gather_rows"):
+              "md_coselect_stats", "md_token_shuffle", "md_place_correlated", "md_gather_rows",
+              "md_dedup_expand"):
         assert n in names
 
 
@@ -45,3 +46,5 @@ def test_host_only_calls():
                         None) == binding.MD_ERR_ARG                          # H % 8 != 0
     assert L.md_token_shuffle(None, 2, None, None, 10, 8, 4, None, None, None, None, 0, None,
                               None) == binding.MD_ERR_ARG                    # T % R != 0
+    assert L.md_dedup_expand(None, 0, 12, None, None, 4, 2, 8, None, None,
+                             None) == binding.MD_ERR_ARG                     # H % 8 != 0
