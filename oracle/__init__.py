@@ -65,10 +65,14 @@ def _load():
             lib.oracle_placement_objective.restype = ctypes.c_longlong
             lib.oracle_place_correlated.argtypes = [P, I32, I32, I32, I32, P]
             lib.oracle_token_shuffle.argtypes = [P, P, P, I64, I32, I32, I32, P, P, P]
+            lib.oracle_coselect_pair.argtypes = [P, P, P, I64, I32, I32, P]
+            lib.oracle_token_shuffle_pair.argtypes = [P, P, P, P, P, I64, I32, I32, I32,
+                                                      ctypes.c_uint64, P, P, P, P]
             for name in ("oracle_route_topk", "oracle_dispatch_layout", "oracle_dispatch_permute",
                          "oracle_dedup_expand",
                          "oracle_combine", "oracle_coselect", "oracle_place_correlated",
-                         "oracle_token_shuffle"):
+                         "oracle_token_shuffle", "oracle_coselect_pair",
+                         "oracle_token_shuffle_pair"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -228,3 +232,36 @@ def token_shuffle(idx_l, C, expert_to_rank_next, R):
     _check(lib.oracle_token_shuffle(_ptr(a), _ptr(Cc), _ptr(p), T, E, k, R,
                                     _ptr(pred), _ptr(perm), _ptr(inv)), "token_shuffle")
     return pred, perm, inv
+
+
+def coselect_pair(idx_prev, idx_l, idx_next, E, T_fit=None):
+    """Pair counts C2[a, b, e'] over the first T_fit tokens: uint32 [E, E, E]."""
+    lib = _load()
+    a = _c(idx_prev, np.int32)
+    b = _c(idx_l, np.int32)
+    c = _c(idx_next, np.int32)
+    T, k = b.shape
+    T_fit = T if T_fit is None else int(T_fit)
+    C2 = np.empty((E, E, E), np.uint32)
+    _check(lib.oracle_coselect_pair(_ptr(a), _ptr(b), _ptr(c), T_fit, E, k, _ptr(C2)), "coselect_pair")
+    return C2
+
+
+def token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_obs):
+    """Pair-based prediction with single-expert fallback -> (pred, perm, inv, use_pair)."""
+    lib = _load()
+    a = _c(idx_prev, np.int32)
+    b = _c(idx_l, np.int32)
+    T, k = b.shape
+    E = C.shape[0]
+    Cc = _c(C, np.uint32)
+    C2c = _c(C2, np.uint32)
+    pn = _c(expert_to_rank_next, np.int32)
+    pred = np.empty(T, np.int32)
+    perm = np.empty(T, np.int32)
+    inv = np.empty(T, np.int32)
+    use = np.empty(T, np.int32)
+    _check(lib.oracle_token_shuffle_pair(_ptr(a), _ptr(b), _ptr(Cc), _ptr(C2c), _ptr(pn), T, E, k, R,
+                                         int(min_obs), _ptr(pred), _ptr(perm), _ptr(inv), _ptr(use)),
+           "token_shuffle_pair")
+    return pred, perm, inv, use

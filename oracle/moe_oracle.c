@@ -686,3 +686,131 @@ done:
     free(pref); free(num); free(den); free(sigma); free(order); free(load);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Pair-based shuffle prediction.                                            */
+/* [EC] "Method 2: Token Shuffling", Mechanism, Prediction: the owner rank at */
+/* layer l+1 is predicted from the experts the token selected at the two     */
+/* preceding layers -- a pair-based lookup -- with a fall back to the        */
+/* single-expert prediction where the pair has too few observations.        */
+/* The pair counts extend C the way C extends W:                             */
+/*   C2[a][b][e'] = #{t < T_fit : a in S_{l-1}(t), b in S_l(t),              */
+/*                                e' in S_{l+1}(t)}   (all k^3 triples).     */
+/* ------------------------------------------------------------------------ */
+
+int oracle_coselect_pair(const int32_t *idx_prev, const int32_t *idx_l, const int32_t *idx_next,
+                         int64_t T_fit, int E, int k, uint32_t *C2)
+{
+    if (T_fit < 0 || E < 1 || k < 1) return 1;
+    memset(C2, 0, sizeof(uint32_t) * (size_t)E * E * E);
+    for (int64_t t = 0; t < T_fit; ++t)
+        for (int i = 0; i < k; ++i)
+            for (int j = 0; j < k; ++j)
+                for (int m = 0; m < k; ++m) {
+                    int a = idx_prev[t * k + i], b = idx_l[t * k + j], c = idx_next[t * k + m];
+                    if (a < 0 || a >= E || b < 0 || b >= E || c < 0 || c >= E) return 1;
+                    C2[((int64_t)a * E + b) * E + c] += 1;
+                }
+    return 0;
+}
+
+/* preference list, confidence numerator and denominator of one count row,
+ * by the same rules as the single-expert form above */
+static void row_prediction(const uint32_t *row, int E, const int32_t *p_next, int R,
+                           uint64_t *sigma, int32_t *pl, uint64_t *num, uint64_t *den)
+{
+    uint64_t total = 0;
+    int best = 0;
+    for (int e = 0; e < E; ++e) {
+        total += row[e];
+        if (row[e] > row[best]) best = e;
+    }
+    *num = row[best];
+    *den = total;
+    for (int d = 0; d < R; ++d) sigma[d] = 0;
+    for (int e = 0; e < E; ++e) sigma[p_next[e]] += row[e];
+    pl[0] = p_next[best];
+    int n = 1;
+    while (n < R) {
+        int pick = -1;
+        for (int d = 0; d < R; ++d) {
+            int used = 0;
+            for (int i = 0; i < n; ++i)
+                if (pl[i] == d) used = 1;
+            if (used) continue;
+            if (pick < 0 || sigma[d] > sigma[pick]) pick = d;
+        }
+        pl[n++] = pick;
+    }
+}
+
+/*
+ * As oracle_token_shuffle, with the prediction row of token t chosen as:
+ *   a = idx_prev[t*k] (top-1 at l-1), b = idx_l[t*k] (top-1 at l);
+ *   the pair row C2[a][b] if its total is at least min_obs,
+ *   else the single-expert row C[b].
+ * Preference order, confidence, visit order and capacity rule are those of
+ * the single-expert form, applied to the chosen row.  use_pair[t] = 1 when
+ * the pair row was used.
+ */
+int oracle_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx_l, const uint32_t *C,
+                              const uint32_t *C2, const int32_t *p_next, int64_t T, int E, int k,
+                              int R, uint64_t min_obs, int32_t *pred_rank, int32_t *perm,
+                              int32_t *inv, int32_t *use_pair)
+{
+    if (T < 0 || E < 1 || k < 1 || R < 1 || T % R != 0 || min_obs < 1) return 1;
+    const int64_t Tr = T / R;
+    int32_t *pref = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1) * R);
+    uint64_t *sigma = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)R);
+    conf_t *order = (conf_t *)malloc(sizeof(conf_t) * (size_t)(T > 0 ? T : 1));
+    int64_t *load = (int64_t *)calloc((size_t)R, sizeof(int64_t));
+    int rc = 0;
+    if (!pref || !sigma || !order || !load) { rc = 2; goto done; }
+
+    for (int64_t t = 0; t < T; ++t) {
+        int a = idx_prev[t * k], b = idx_l[t * k];
+        if (a < 0 || a >= E || b < 0 || b >= E) { rc = 1; goto done; }
+        const uint32_t *prow = C2 + ((int64_t)a * E + b) * E;
+        uint64_t psum = 0;
+        for (int e = 0; e < E; ++e) psum += prow[e];
+        use_pair[t] = psum >= min_obs;
+        const uint32_t *row = use_pair[t] ? prow : C + (int64_t)b * E;
+        row_prediction(row, E, p_next, R, sigma, pref + t * R, &order[t].num, &order[t].den);
+        order[t].t = t;
+    }
+    /* the per-token denominators, kept by token before the sort reorders */
+    uint64_t *den_t = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)(T > 0 ? T : 1));
+    if (!den_t) { rc = 2; goto done; }
+    for (int64_t t = 0; t < T; ++t) den_t[t] = order[t].den;
+    qsort(order, (size_t)T, sizeof(conf_t), cmp_conf);
+
+    for (int64_t i = 0; i < T; ++i) {
+        int64_t t = order[i].t;
+        int chosen = -1;
+        if (den_t[t] == 0) {
+            int s = (int)(t / Tr);
+            if (load[s] < Tr) chosen = s;
+            for (int d = 0; chosen < 0 && d < R; ++d)
+                if (load[d] < Tr) chosen = d;
+        } else {
+            const int32_t *pl = pref + t * R;
+            for (int n = 0; chosen < 0 && n < R; ++n)
+                if (load[pl[n]] < Tr) chosen = pl[n];
+        }
+        pred_rank[t] = chosen;
+        load[chosen] += 1;
+    }
+    free(den_t);
+
+    for (int d = 0; d < R; ++d) load[d] = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        int d = pred_rank[t];
+        int64_t pos = (int64_t)d * Tr + load[d];
+        load[d] += 1;
+        perm[t] = (int32_t)pos;
+        inv[pos] = (int32_t)t;
+    }
+done:
+    free(pref); free(sigma); free(order); free(load);
+    return rc;
+}
