@@ -390,6 +390,36 @@ def run_rows(args, md, device, stream, peak):
     del w, a, b, C, sws, xs
     torch.cuda.empty_cache()
 
+    # pair-based shuffle prediction on the three-layer workload (counts fitted
+    # on the first 4096 tokens; a pair row is used when its total reaches 8k)
+    w = synth.make_workload("three_layer_e128_k6", seed=args.seed, device=device, with_rows=False)
+    g = [md.md_route_topk(lg, w.k)[0] for lg in (w.logits_prev, w.logits, w.logits_next)]
+    C2 = torch.empty(w.E, w.E, w.E, dtype=torch.int32, device=device)
+    t_c2 = _time(lambda: md.md_coselect_pair_stats(g[0], g[1], g[2], w.E, T_fit=w.fit_tokens, C2=C2,
+                                                   stream=stream), stream, reps)
+    _, C = md.md_coselect_stats(g[1], g[2], w.E, T_fit=w.fit_tokens, want_W=False)
+    pws = md.alloc_workspace(int(md.lib().md_token_shuffle_pair_workspace_size(w.T, w.E, w.R)), device)
+    pred = torch.empty(w.T, dtype=torch.int32, device=device)
+    perm, inv, use = torch.empty_like(pred), torch.empty_like(pred), torch.empty_like(pred)
+    min_obs = 8 * w.k
+    t_sp = _time(lambda: md.md_token_shuffle_pair(g[0], g[1], C, C2, w.expert_to_rank, w.R, min_obs,
+                                                  pred, perm, inv, use, workspace=pws,
+                                                  stream=stream), stream, reps)
+    nxt_rank = w.expert_to_rank[g[2].long()]
+    loc_pair = float(pred[:, None].eq(nxt_rank).float().mean())
+    use_share = float(use.float().mean())
+    sp = md.md_token_shuffle(g[1], C, w.expert_to_rank, w.R)[0]
+    loc_single = float(sp[:, None].eq(nxt_rank).float().mean())
+    loc_none = float((torch.arange(w.T, device=device) // (w.T // w.R))[:, None].eq(nxt_rank)
+                     .float().mean())
+    rows["token_shuffle_pair_e128_k6"] = {
+        "T": w.T, "min_obs": min_obs, "pair_counts_us": round(t_c2 * 1e3, 2),
+        "shuffle_pair_us": round(t_sp * 1e3, 2), "tokens_on_pair_rows": round(use_share, 4),
+        "locality_no_shuffle": round(loc_none, 4), "locality_single": round(loc_single, 4),
+        "locality_pair": round(loc_pair, 4)}
+    del w, g, C2, C, pws
+    torch.cuda.empty_cache()
+
     # the full pipeline at full size: T=262144, E=256, k=8, R=64
     w = synth.make_workload("full_e256_k8", seed=args.seed, device=device)
     T, H, E, k, R = w.T, w.H, w.E, w.k, w.R

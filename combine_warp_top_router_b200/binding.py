@@ -48,6 +48,10 @@ _SIGNATURES = {
     "md_place_correlated": ([_P, _I, _I, _I, _I, _P, _P, _S, _P, _P], _I),
     "md_token_shuffle_workspace_size": ([_L, _I, _I], _S),
     "md_token_shuffle": ([_P, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _S, _P, _P], _I),
+    "md_coselect_pair_stats": ([_P, _P, _P, _L, _I, _I, _P, _I, _P, _P], _I),
+    "md_token_shuffle_pair_workspace_size": ([_L, _I, _I], _S),
+    "md_token_shuffle_pair": ([_P, _P, _I, _P, _P, _P, _L, _I, _I, ctypes.c_uint32, _P, _P, _P, _P,
+                               _P, _S, _P, _P], _I),
     "md_gather_rows": ([_P, _L, _L, _P, _L, _P, _P, _P], _I),
 }
 
@@ -362,3 +366,51 @@ def md_token_shuffle(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None
                                 workspace.numel(), _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_token_shuffle")
     return pred_rank, perm, inv
+
+
+def md_coselect_pair_stats(idx_prev, idx_l, idx_next, E, T_fit=None, C2=None, accumulate=False,
+                           dev_status=None, stream=None):
+    """Pair counts C2[a, b, e'] (int32 view of uint32 [E, E, E])."""
+    _need(idx_l, "idx_l", torch.int32)
+    dev = idx_l.device
+    _need(idx_prev, "idx_prev", torch.int32, dev)
+    _need(idx_next, "idx_next", torch.int32, dev)
+    T, k = idx_l.shape
+    T_fit = T if T_fit is None else T_fit
+    if C2 is None:
+        C2 = torch.empty(E, E, E, dtype=torch.int32, device=dev)
+    _need(C2, "C2", torch.int32, dev)
+    rc = lib().md_coselect_pair_stats(_ptr(idx_prev), _ptr(idx_l), _ptr(idx_next), T_fit, E, k,
+                                      _ptr(C2), 1 if accumulate else 0, _ptr(dev_status),
+                                      _stream(stream, dev))
+    _check(rc, "md_coselect_pair_stats")
+    return C2
+
+
+def md_token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_obs, pred_rank=None,
+                          perm=None, inv=None, use_pair=None, workspace=None, dev_status=None,
+                          stream=None):
+    """Pair-based shuffle prediction with single-expert fallback -> (pred, perm, inv, use_pair)."""
+    _need(idx_l, "idx_l", torch.int32)
+    dev = idx_l.device
+    _need(idx_prev, "idx_prev", torch.int32, dev)
+    _need(C, "C", torch.int32, dev)
+    _need(C2, "C2", torch.int32, dev)
+    _need(expert_to_rank_next, "expert_to_rank_next", torch.int32, dev)
+    T, k = idx_l.shape
+    E = C.shape[0]
+    i32 = dict(dtype=torch.int32, device=dev)
+    pred_rank = torch.empty(T, **i32) if pred_rank is None else pred_rank
+    perm = torch.empty(T, **i32) if perm is None else perm
+    inv = torch.empty(T, **i32) if inv is None else inv
+    use_pair = torch.empty(T, **i32) if use_pair is None else use_pair
+    need = int(lib().md_token_shuffle_pair_workspace_size(T, E, R))
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    rc = lib().md_token_shuffle_pair(_ptr(idx_prev), _ptr(idx_l), k, _ptr(C), _ptr(C2),
+                                     _ptr(expert_to_rank_next), T, E, R, int(min_obs),
+                                     _ptr(pred_rank), _ptr(perm), _ptr(inv), _ptr(use_pair),
+                                     _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                     _stream(stream, dev))
+    _check(rc, "md_token_shuffle_pair")
+    return pred_rank, perm, inv, use_pair

@@ -12,6 +12,12 @@
 // blockIdx.x a chunk of tokens.  Each CTA counts the increments that fall in
 // its segment with shared-memory atomics and adds its non-zero counters to
 // W / C in global memory (both W[a][b] and W[b][a] for a != b).
+//
+// Pair counts (md_coselect_pair_stats), "Expert Coupling ...", Method 2,
+// Prediction (pair-based lookup over the two preceding layers):
+// C2[a][b][e'] counts every (a in S_{l-1}(t), b in S_l(t), e' in S_{l+1}(t))
+// triple.  The E^3 table lives in global memory; one thread per (token, a, b)
+// adds its k increments with global atomics.
 #include "common.cuh"
 
 namespace {
@@ -91,6 +97,31 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+__global__ void __launch_bounds__(256)
+    k_coselect_pair(const int32_t *__restrict__ idx_p, const int32_t *__restrict__ idx_l,
+                    const int32_t *__restrict__ idx_n, int64_t T_fit, int E, int k,
+                    uint32_t *__restrict__ C2, int32_t *status)
+{
+    const int kk = k * k;
+    const int64_t n = T_fit * kk;
+    for (int64_t f = (int64_t)blockIdx.x * 256 + threadIdx.x; f < n; f += (int64_t)gridDim.x * 256) {
+        const int64_t t = f / kk;
+        const int r = (int)(f - t * kk);
+        const int i = r / k, j = r - i * k;
+        const int a = __ldg(idx_p + t * k + i), b = __ldg(idx_l + t * k + j);
+        if (a < 0 || a >= E || b < 0 || b >= E) {
+            md::report(status, MD_ERR_DATA);
+            continue;
+        }
+        uint32_t *row = C2 + ((int64_t)a * E + b) * E;
+        for (int m = 0; m < k; ++m) {
+            const int c = __ldg(idx_n + t * k + m);
+            if (c >= 0 && c < E) atomicAdd(row + c, 1u);
+            else md::report(status, MD_ERR_DATA);
+        }
+    }
+}
+
 }  // namespace
 
 extern "C" int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, int64_t T_fit,
@@ -138,6 +169,32 @@ extern "C" int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, 
     dim3 grid((unsigned)nx, (unsigned)n_seg);
     k_coselect<<<grid, kThreads, (size_t)seg_len * sizeof(uint32_t), s>>>(
         idx_l, idx_next, T_fit, E, k, tpb, W, C, n_tri, seg_len, dev_status);
+    md::count_launches(1);
+    return md::launch_status();
+}
+
+extern "C" int md_coselect_pair_stats(const int32_t *idx_prev, const int32_t *idx_l,
+                                      const int32_t *idx_next, int64_t T_fit, int E, int k,
+                                      uint32_t *C2, int accumulate, int32_t *dev_status,
+                                      void *stream)
+{
+    if (T_fit < 0 || E < 1 || k < 1 || k > MD_MAX_TOPK || !C2) return MD_ERR_ARG;
+    if (E > MD_MAX_PAIR_EXPERTS) return MD_ERR_UNSUPPORTED;
+    if (T_fit > 0 && (!idx_prev || !idx_l || !idx_next)) return MD_ERR_ARG;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK) return rc;
+    if (!accumulate) {
+        md::count_launches(1);
+        if (cudaMemsetAsync(C2, 0, (size_t)E * E * E * sizeof(uint32_t), s) != cudaSuccess)
+            return MD_ERR_CUDA;
+    }
+    if (T_fit == 0) return MD_OK;
+    int64_t blocks = (T_fit * k * k + 255) / 256;
+    const int64_t cap = (int64_t)md::sm_count() * 16;
+    if (blocks > cap) blocks = cap;
+    k_coselect_pair<<<(unsigned)blocks, 256, 0, s>>>(idx_prev, idx_l, idx_next, T_fit, E, k, C2,
+                                                     dev_status);
     md::count_launches(1);
     return md::launch_status();
 }

@@ -290,10 +290,15 @@ __global__ void __launch_bounds__(32)
 constexpr int kGreedyThreads = 1024;
 constexpr int kGreedyWarps = kGreedyThreads / 32;
 
+// PAIR: the prediction row differs per token, so instead of first[e] each
+// token walks its own preference list (tpref[t*R ..], R bytes), and an empty
+// row is marked by a zero confidence key.
+template <bool PAIR>
 __global__ void __launch_bounds__(kGreedyThreads, 1)
     k_shuf_greedy(const int32_t *__restrict__ order, const int32_t *__restrict__ idx_l, int k,
-                  ShufWs ws, int64_t T, int E, int R, int64_t Tr, int32_t *__restrict__ pred,
-                  int32_t *status)
+                  ShufWs ws, const unsigned char *__restrict__ tpref,
+                  const unsigned long long *__restrict__ tconf, int64_t T, int E, int R, int64_t Tr,
+                  int32_t *__restrict__ pred, int32_t *status)
 {
     extern __shared__ __align__(16) unsigned char g_raw[];
     int *s_first = reinterpret_cast<int *>(g_raw);                    // [E]
@@ -306,7 +311,8 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
     __shared__ int s_first_any, s_over, s_pmin;
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
 
-    for (int i = tid; i < E * R; i += kGreedyThreads) s_pref[i] = (unsigned char)ws.pref[i];
+    if (!PAIR)
+        for (int i = tid; i < E * R; i += kGreedyThreads) s_pref[i] = (unsigned char)ws.pref[i];
     for (int d = tid; d < R; d += kGreedyThreads) {
         s_load[d] = 0;
         s_tot[d] = 0;
@@ -316,8 +322,9 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
         s_first_any = 0;
     }
     __syncthreads();
-    for (int e = tid; e < E; e += kGreedyThreads)
-        s_first[e] = ws.den[e] == 0ull ? -1 : (int)s_pref[(size_t)e * R];
+    if (!PAIR)
+        for (int e = tid; e < E; e += kGreedyThreads)
+            s_first[e] = ws.den[e] == 0ull ? -1 : (int)s_pref[(size_t)e * R];
     __syncthreads();
 
     // token ids are fetched two chunks ahead and their top-1 experts one chunk
@@ -326,18 +333,24 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
         const int64_t pos = base + tid;
         return pos < T ? (int64_t)order[pos] : -1;
     };
+    // single: the top-1 expert; pair: 1 when the token's prediction row is empty
+    auto key_of = [&](int64_t t) -> int {
+        if (t < 0) return 0;
+        if (PAIR) return tconf[t] == 0ull ? 1 : 0;
+        return idx_l[t * k];
+    };
     int64_t t_n1 = token_at(0);
-    int e_n1 = t_n1 >= 0 ? idx_l[t_n1 * k] : 0;
+    int e_n1 = key_of(t_n1);
     int64_t t_n2 = token_at(kGreedyThreads);
 
     for (int64_t base = 0; base < T; base += kGreedyThreads) {
         const int64_t t = t_n1;
         int e1 = e_n1;
         t_n1 = t_n2;
-        e_n1 = t_n1 >= 0 ? idx_l[t_n1 * k] : 0;
+        e_n1 = key_of(t_n1);
         t_n2 = token_at(base + 2 * kGreedyThreads);
         const bool have = t >= 0;
-        if (have && (e1 < 0 || e1 >= E)) {
+        if (!PAIR && have && (e1 < 0 || e1 >= E)) {
             md::report(status, MD_ERR_DATA);
             e1 = 0;
         }
@@ -347,7 +360,19 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
             // choice under the current set of full ranks
             int ch = -1;
             if (have && tid >= start) {
-                const int f = s_first[e1];
+                int f;
+                if (PAIR) {
+                    f = -1;
+                    if (!e1) {
+                        const unsigned char *pl = tpref + t * R;
+                        const unsigned long long full = s_full;
+                        int n = 0;
+                        while (n < R && ((full >> pl[n]) & 1ull)) ++n;
+                        f = n < R ? (int)pl[n] : 0;
+                    }
+                } else {
+                    f = s_first[e1];
+                }
                 ch = f >= 0 ? f : (((s_full >> src_rank) & 1ull) ? s_first_any : src_rank);
             }
             const unsigned g =
@@ -376,7 +401,7 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
                         s_full = f;
                     }
                     __syncthreads();
-                    for (int e = tid; e < E; e += kGreedyThreads) {
+                    for (int e = tid; !PAIR && e < E; e += kGreedyThreads) {
                         if (s_first[e] < 0) continue;
                         const unsigned char *pl = s_pref + (size_t)e * R;
                         int n = 0;
@@ -441,7 +466,7 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
                 s_full = f;
             }
             __syncthreads();
-            for (int e = tid; e < E; e += kGreedyThreads) {
+            for (int e = tid; !PAIR && e < E; e += kGreedyThreads) {
                 if (s_first[e] < 0) continue;
                 const unsigned char *pl = s_pref + (size_t)e * R;
                 int n = 0;
@@ -457,6 +482,189 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
             if (pmin >= kGreedyThreads - 1) break;
             start = pmin + 1;
         }
+    }
+}
+
+// ------------------------------------------------------------ pair shuffle
+// Each token's prediction row is the pair row C2[a][b] (a, b its top-1
+// experts at layers l-1 and l) when that row's total reaches min_obs, else
+// the single row C[b].  One warp per token computes from that row the
+// preference list (R bytes) and an exact confidence key:
+//     key = floor(num * 2^63 / den)   (0 for an empty row).
+// For den < 2^31, two different fractions num/den <= 1 differ by at least
+// 2^-62, i.e. by at least 2 after scaling, so the keys order the
+// confidences exactly and equal confidences get equal keys.  Tokens are then
+// sorted by (key desc, t asc) with a stable LSD radix sort (11-bit digits),
+// and the greedy walks each token's own preference list.
+constexpr int kRadixBits = 11;
+constexpr int kRadixBuckets = 1 << kRadixBits;
+constexpr int kRadixPasses = (64 + kRadixBits - 1) / kRadixBits;
+constexpr int kPairWarps = 8;
+
+struct PairWs {
+    unsigned char *tpref;      // [T*R] preference list of each token
+    unsigned long long *conf;  // [T]   confidence key of each token
+    int32_t *seq_a, *seq_b;    // [T]   radix sort ping-pong
+    int32_t *keys;             // [T]   bucket of each token in the final partition
+    int32_t *tile_hist;        // [n_tiles * max(2^11, R)]
+};
+
+size_t pair_layout(int64_t T, int R, PairWs *w, void *base)
+{
+    char *b = static_cast<char *>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        char *p = b ? b + o : nullptr;
+        o += md::align_up(bytes, 256);
+        return p;
+    };
+    const int64_t Tn = T > 0 ? T : 1;
+    const int64_t n_tiles = (Tn + kTile - 1) / kTile;
+    PairWs x;
+    x.tpref = reinterpret_cast<unsigned char *>(take((size_t)Tn * R));
+    x.conf = reinterpret_cast<unsigned long long *>(take((size_t)Tn * 8));
+    x.seq_a = reinterpret_cast<int32_t *>(take((size_t)Tn * 4));
+    x.seq_b = reinterpret_cast<int32_t *>(take((size_t)Tn * 4));
+    x.keys = reinterpret_cast<int32_t *>(take((size_t)Tn * 4));
+    const int nbk = kRadixBuckets > R ? kRadixBuckets : R;
+    x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)n_tiles * nbk * 4));
+    if (w) *w = x;
+    return o;
+}
+
+__global__ void __launch_bounds__(kPairWarps * 32)
+    k_pair_rows(const int32_t *__restrict__ idx_p, const int32_t *__restrict__ idx_l, int k,
+                const uint32_t *__restrict__ C, const uint32_t *__restrict__ C2,
+                const int32_t *__restrict__ p_next, int64_t T, int E, int R, uint32_t min_obs,
+                PairWs ws, int32_t *__restrict__ use_pair, int32_t *status)
+{
+    __shared__ unsigned long long s_sig[kPairWarps][MD_MAX_RANKS];
+    const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+    unsigned long long *sig = s_sig[wl];
+    const int64_t w0 = (int64_t)blockIdx.x * kPairWarps + wl;
+    const int64_t nw = (int64_t)gridDim.x * kPairWarps;
+    for (int64_t t = w0; t < T; t += nw) {
+        int a = __ldg(idx_p + t * k), b = __ldg(idx_l + t * k);
+        if (a < 0 || a >= E || b < 0 || b >= E) {
+            md::report(status, MD_ERR_DATA);
+            a = a < 0 || a >= E ? 0 : a;
+            b = b < 0 || b >= E ? 0 : b;
+        }
+        const uint32_t *prow = C2 + ((int64_t)a * E + b) * E;
+        unsigned long long psum = 0;
+        for (int e = lane; e < E; e += 32) psum += __ldg(prow + e);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
+        const bool use = psum >= min_obs;
+        const uint32_t *row = use ? prow : C + (int64_t)b * E;
+        for (int d = lane; d < R; d += 32) sig[d] = 0ull;
+        __syncwarp();
+        // total, arg-max (lowest index on ties) and per-rank sums
+        unsigned long long tot = 0;
+        uint32_t bv = 0;
+        int be = INT_MAX;
+        for (int e = lane; e < E; e += 32) {
+            const uint32_t v = __ldg(row + e);
+            tot += v;
+            if (v > bv || (v == bv && e < be)) {
+                bv = v;
+                be = e;
+            }
+            const int d = __ldg(p_next + e);
+            if (d < 0 || d >= R) md::report(status, MD_ERR_DATA);
+            else if (v) atomicAdd(&sig[d], (unsigned long long)v);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            tot += __shfl_xor_sync(0xffffffffu, tot, o);
+            const uint32_t v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int e2 = __shfl_xor_sync(0xffffffffu, be, o);
+            if (v2 > bv || (v2 == bv && e2 < be)) {
+                bv = v2;
+                be = e2;
+            }
+        }
+        __syncwarp();
+        int first = __ldg(p_next + be);
+        if (first < 0 || first >= R) first = 0;
+        unsigned char *pl = ws.tpref + t * R;
+        for (int d = lane; d < R; d += 32) {
+            int pos = 0;
+            if (d != first) {
+                pos = 1;
+                for (int d2 = 0; d2 < R; ++d2)
+                    if (d2 != first && d2 != d && (sig[d2] > sig[d] || (sig[d2] == sig[d] && d2 < d)))
+                        ++pos;
+            }
+            pl[pos] = (unsigned char)d;
+        }
+        if (lane == 0) {
+            unsigned long long key = 0ull;
+            if (tot > 0) {
+                if (tot >= (1ull << 31)) md::report(status, MD_ERR_UNSUPPORTED);
+                key = (unsigned long long)(((unsigned __int128)bv << 63) / tot);
+            }
+            ws.conf[t] = key;
+            if (use_pair) use_pair[t] = use ? 1 : 0;
+        }
+        __syncwarp();
+    }
+}
+
+// digit of the sort key for one LSD pass: confidence descending
+__device__ __forceinline__ int radix_digit(const unsigned long long *conf, int32_t tok, int shift)
+{
+    return (int)((~conf[tok] >> shift) & (kRadixBuckets - 1));
+}
+
+__global__ void __launch_bounds__(256)
+    k_radix_hist(const int32_t *__restrict__ seq, const unsigned long long *__restrict__ conf,
+                 int64_t T, int shift, int32_t *__restrict__ tile_hist)
+{
+    __shared__ int h[kRadixBuckets];
+    for (int b = threadIdx.x; b < kRadixBuckets; b += 256) h[b] = 0;
+    __syncthreads();
+    const int64_t t0 = (int64_t)blockIdx.x * kTile;
+    for (int i = threadIdx.x; i < kTile; i += 256) {
+        const int64_t pos = t0 + i;
+        if (pos < T) atomicAdd(&h[radix_digit(conf, seq ? seq[pos] : (int32_t)pos, shift)], 1);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < kRadixBuckets; b += 256)
+        tile_hist[(int64_t)blockIdx.x * kRadixBuckets + b] = h[b];
+}
+
+// One warp per tile, items in sequence order, stable within each digit.
+__global__ void __launch_bounds__(32)
+    k_radix_scatter(const int32_t *__restrict__ seq, const unsigned long long *__restrict__ conf,
+                    int64_t T, int shift, const int32_t *__restrict__ tile_hist,
+                    int32_t *__restrict__ seq_out)
+{
+    __shared__ int cnt[kRadixBuckets];
+    const int lane = threadIdx.x;
+    for (int b = lane; b < kRadixBuckets; b += 32)
+        cnt[b] = tile_hist[(int64_t)blockIdx.x * kRadixBuckets + b];
+    const int64_t t0 = (int64_t)blockIdx.x * kTile;
+    int tok[kTile / 32], dg[kTile / 32];
+#pragma unroll
+    for (int c = 0; c < kTile / 32; ++c) {
+        const int64_t pos = t0 + c * 32 + lane;
+        tok[c] = pos < T ? (seq ? seq[pos] : (int32_t)pos) : -1;
+    }
+#pragma unroll
+    for (int c = 0; c < kTile / 32; ++c) dg[c] = tok[c] >= 0 ? radix_digit(conf, tok[c], shift) : -1;
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < kTile / 32; ++c) {
+        const int key = dg[c];
+        const bool in = key >= 0;
+        const unsigned g = __match_any_sync(0xffffffffu, in ? (unsigned)key : (0x80000000u | lane));
+        int pos = 0;
+        if (in) pos = cnt[key] + __popc(g & md::lanemask_lt());
+        __syncwarp();
+        if (in && (g >> lane) == 1u) cnt[key] += __popc(g);
+        __syncwarp();
+        if (in) seq_out[pos] = tok[c];
     }
 }
 
@@ -499,11 +707,11 @@ extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
     k_bucket_scatter<<<n_tiles, 32, nbk0 * sizeof(int), s>>>(0, T, nbk0, ws.keys, ws.tile_hist,
                                                             ws.order, nullptr, nullptr);
     const size_t gsm = (size_t)E * sizeof(int) + (size_t)E * R;
-    if (cudaFuncSetAttribute(k_shuf_greedy, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm) !=
+    if (cudaFuncSetAttribute(k_shuf_greedy<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm) !=
         cudaSuccess)
         return MD_ERR_CUDA;
-    k_shuf_greedy<<<1, kGreedyThreads, gsm, s>>>(ws.order, idx_l, k, ws, T, E, R, Tr, pred_rank,
-                                                 dev_status);
+    k_shuf_greedy<false><<<1, kGreedyThreads, gsm, s>>>(ws.order, idx_l, k, ws, nullptr, nullptr, T,
+                                                        E, R, Tr, pred_rank, dev_status);
     // new positions: stable partition by assigned rank
     k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
                                                        ws.keys, ws.tile_hist);
@@ -511,5 +719,66 @@ extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
     k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, R, ws.keys, ws.tile_hist, nullptr,
                                                          perm, inv);
     md::count_launches(9);
+    return md::launch_status();
+}
+
+extern "C" size_t md_token_shuffle_pair_workspace_size(int64_t T, int E, int R)
+{
+    if (T < 0 || E < 1 || R < 1) return 0;
+    return pair_layout(T, R, nullptr, nullptr);
+}
+
+extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx_l, int k,
+                                     const uint32_t *C, const uint32_t *C2,
+                                     const int32_t *expert_to_rank_next, int64_t T, int E, int R,
+                                     uint32_t min_obs, int32_t *pred_rank, int32_t *perm,
+                                     int32_t *inv, int32_t *use_pair, void *workspace,
+                                     size_t workspace_bytes, int32_t *dev_status, void *stream)
+{
+    if (T < 0 || E < 1 || R < 1 || k < 1 || k > MD_MAX_TOPK || min_obs < 1) return MD_ERR_ARG;
+    if (E > MD_MAX_PAIR_EXPERTS || R > MD_MAX_RANKS || T >= ((int64_t)1 << 31))
+        return MD_ERR_UNSUPPORTED;
+    if (T % R != 0) return MD_ERR_ARG;
+    if (!C || !C2 || !expert_to_rank_next) return MD_ERR_ARG;
+    if (T > 0 && (!idx_prev || !idx_l || !pred_rank || !perm || !inv)) return MD_ERR_ARG;
+    const size_t need = pair_layout(T, R, nullptr, nullptr);
+    if (!workspace || workspace_bytes < need) return MD_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MD_ERR_ARG;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK || T == 0) return rc;
+    PairWs pw;
+    pair_layout(T, R, &pw, workspace);
+    const int n_tiles = (int)((T + kTile - 1) / kTile);
+    const int64_t Tr = T / R;
+
+    int64_t blocks = (T + kPairWarps - 1) / kPairWarps;
+    const int64_t cap = (int64_t)md::sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    k_pair_rows<<<(unsigned)blocks, kPairWarps * 32, 0, s>>>(idx_prev, idx_l, k, C, C2,
+                                                             expert_to_rank_next, T, E, R, min_obs,
+                                                             pw, use_pair, dev_status);
+    // visit order: stable LSD radix sort by (confidence key desc), from t ascending
+    const int32_t *in = nullptr;
+    int32_t *out = pw.seq_a;
+    for (int pass = 0; pass < kRadixPasses; ++pass) {
+        const int shift = pass * kRadixBits;
+        k_radix_hist<<<n_tiles, 256, 0, s>>>(in, pw.conf, T, shift, pw.tile_hist);
+        k_bucket_scan<<<1, 1024, kRadixBuckets * sizeof(int), s>>>(pw.tile_hist, n_tiles,
+                                                                  kRadixBuckets);
+        k_radix_scatter<<<n_tiles, 32, 0, s>>>(in, pw.conf, T, shift, pw.tile_hist, out);
+        in = out;
+        out = out == pw.seq_a ? pw.seq_b : pw.seq_a;
+    }
+    ShufWs none{};
+    k_shuf_greedy<true><<<1, kGreedyThreads, 0, s>>>(in, nullptr, k, none, pw.tpref, pw.conf, T, E,
+                                                     R, Tr, pred_rank, dev_status);
+    // new positions: stable partition by assigned rank
+    k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
+                                                       pw.keys, pw.tile_hist);
+    k_bucket_scan<<<1, 1024, R * sizeof(int), s>>>(pw.tile_hist, n_tiles, R);
+    k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, R, pw.keys, pw.tile_hist, nullptr,
+                                                         perm, inv);
+    md::count_launches(1 + 3 * kRadixPasses + 1 + 3);
     return md::launch_status();
 }

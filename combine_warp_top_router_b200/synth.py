@@ -31,6 +31,7 @@ import torch
 _T_LOGITS, _T_LOGITS_NEXT, _T_X, _T_Y = 1, 2, 3, 4
 _T_GROUPS, _T_ZIPF, _T_PAIRS, _T_PAIR_PICK, _T_PAIR_ON = 5, 6, 7, 8, 9
 _T_SUCC, _T_SKEW, _T_GROUPS_NEXT, _T_ZIPF_NEXT = 10, 11, 12, 13
+_T_LOGITS_PREV, _T_GROUPS_PREV, _T_ZIPF_PREV, _T_SUCC_PAIR = 14, 15, 16, 17
 
 
 def generator(seed: int, tag: int, device="cpu") -> torch.Generator:
@@ -124,6 +125,23 @@ def boost_successor(next_logits: torch.Tensor, prev_logits: torch.Tensor, succ: 
     return out
 
 
+def pair_successor_map(E: int, seed: int, device="cpu") -> torch.Tensor:
+    """A fixed random map (expert at l-1, expert at l) -> layer-l+1 expert, [E, E]."""
+    return torch.randint(0, E, (E, E), generator=generator(seed, _T_SUCC_PAIR, device),
+                         device=device)
+
+
+def boost_pair_successor(next_logits: torch.Tensor, prev2_logits: torch.Tensor,
+                         prev_logits: torch.Tensor, succ2: torch.Tensor,
+                         boost: float) -> torch.Tensor:
+    """Add `boost` at succ2[first argmax at l-1, first argmax at l] per token."""
+    a = torch.argmax(prev2_logits, dim=1)
+    b = torch.argmax(prev_logits, dim=1)
+    out = next_logits.clone()
+    out[torch.arange(out.shape[0], device=out.device), succ2[a, b]] += boost
+    return out
+
+
 @dataclass
 class Workload:
     """One synthetic problem.  Tensors live on `device`."""
@@ -140,6 +158,7 @@ class Workload:
     expert_to_rank: torch.Tensor   # int32 [E]
     logits_next: torch.Tensor | None = None
     fit_tokens: int = 0
+    logits_prev: torch.Tensor | None = None  # layer l-1, three-layer workloads only
     extra: dict = field(default_factory=dict)
 
 
@@ -156,6 +175,10 @@ SPECS = {
     "two_layer_e128_k6": dict(T=65536, H=2048, E=128, k=6, R=16, mode=1,
                               desc="T=65536 H=2048 E=128 top-6 R=16, two layers, layer l+1 boosted on a "
                                    "fixed successor of the layer-l top-1, token shuffle, dedup"),
+    "three_layer_e128_k6": dict(T=65536, H=2048, E=128, k=6, R=16, mode=1,
+                                desc="T=65536 H=2048 E=128 top-6 R=16, three layers: layer l boosted "
+                                     "on a fixed successor of the layer-(l-1) top-1, layer l+1 on a "
+                                     "fixed successor of the (l-1, l) top-1 pair; pair-based shuffle"),
     "full_e256_k8": dict(T=262144, H=2048, E=256, k=8, R=64, mode=1,
                          desc="T=262144 H=2048 E=256 top-8 R=64, +3.0 on one of 64 groups of 4 drawn "
                               "Zipf(1.1), x4 load skew, full pipeline, dedup"),
@@ -187,6 +210,15 @@ def make_workload(name: str, seed: int = 0, device="cpu", T: int | None = None,
                                    device=device)
         nxt = boost_successor(fresh, logits, successor_map(E, seed, device), 3.0)
         fit = min(T, 4096)
+    elif name == "three_layer_e128_k6":
+        prev = group_boost_logits(T, E, 2, 3.0, seed, _T_LOGITS_PREV, _T_GROUPS_PREV, _T_ZIPF_PREV,
+                                  device=device)
+        fresh = group_boost_logits(T, E, 2, 3.0, seed, _T_LOGITS, _T_GROUPS, _T_ZIPF, device=device)
+        logits = boost_successor(fresh, prev, successor_map(E, seed, device), 3.0)
+        fresh = group_boost_logits(T, E, 2, 3.0, seed, _T_LOGITS_NEXT, _T_GROUPS_NEXT, _T_ZIPF_NEXT,
+                                   device=device)
+        nxt = boost_pair_successor(fresh, prev, logits, pair_successor_map(E, seed, device), 3.0)
+        fit = min(T, 4096)
     elif name == "full_e256_k8":
         bias = load_skew_bias(E, 4.0, seed, device)
         logits = group_boost_logits(T, E, 4, 3.0, seed, _T_LOGITS, _T_GROUPS, _T_ZIPF,
@@ -201,4 +233,5 @@ def make_workload(name: str, seed: int = 0, device="cpu", T: int | None = None,
     y = normal_bf16(T * k, H, seed, _T_Y, device) if with_rows else None
     return Workload(name=name, T=T, H=H, E=E, k=k, R=R, mode=mode, logits=logits.contiguous(),
                     x=x, y=y, expert_to_rank=contiguous_placement(E, R, device),
-                    logits_next=None if nxt is None else nxt.contiguous(), fit_tokens=fit)
+                    logits_next=None if nxt is None else nxt.contiguous(), fit_tokens=fit,
+                    logits_prev=prev.contiguous() if name == "three_layer_e128_k6" else None)

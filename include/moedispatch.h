@@ -63,6 +63,7 @@ typedef enum md_status {
 #define MD_COMBINE_WIRE 1      /* per-rank partial sums (bf16), then sum   */
 #define MD_SEED_CONTIGUOUS 0   /* placement search starts contiguous       */
 #define MD_SEED_GREEDY_PAIRS 1 /* placement search starts from greedy pairs*/
+#define MD_MAX_PAIR_EXPERTS 256 /* pair counts are E^3 entries               */
 
 #define MD_MAX_TOPK 32
 #define MD_MAX_EXPERTS 1024
@@ -257,6 +258,22 @@ int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, int64_t T_f
                       void *stream);
 
 /*
+ * md_coselect_pair_stats -- pair counts for the pair-based shuffle predictor.
+ * "Expert Coupling ...", Method 2 (Token Shuffling), Prediction: the next
+ * layer is predicted from the experts of the two preceding layers.  Every
+ * (a, b, e') triple of a token is counted, as C counts every (b, e') pair:
+ *
+ *   idx_prev, idx_l, idx_next  int32 [>= T_fit, k]  layers l-1, l, l+1
+ *   C2  uint32 [E, E, E]: C2[a][b][e'] += #{(t,i,j,m) : S_l-1(t)_i = a,
+ *                                 S_l(t)_j = b, S_l+1(t)_m = e'}, t < T_fit
+ *   accumulate  0: C2 is cleared first; 1: counts are added.
+ *   Limits: E <= MD_MAX_PAIR_EXPERTS (the table has E^3 entries), k <= 32.
+ */
+int md_coselect_pair_stats(const int32_t *idx_prev, const int32_t *idx_l, const int32_t *idx_next,
+                           int64_t T_fit, int E, int k, uint32_t *C2, int accumulate,
+                           int32_t *dev_status, void *stream);
+
+/*
  * md_place_correlated -- correlated expert placement on the GPU.
  * "Expert Coupling ...", Correlated Placement: a Kernighan-Lin-style local
  * search from contiguous placement swaps experts between GPUs to maximise
@@ -306,6 +323,34 @@ int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
                      int32_t *pred_rank, int32_t *perm, int32_t *inv,
                      void *workspace, size_t workspace_bytes, int32_t *dev_status,
                      void *stream);
+
+/*
+ * md_token_shuffle_pair -- md_token_shuffle with the pair-based prediction
+ * and its single-expert fallback ("Expert Coupling ...", Method 2,
+ * Prediction: a pair-based lookup over the two preceding layers, falling
+ * back to single-expert prediction for sparse observations).  For token t
+ * with top-1 experts a (layer l-1) and b (layer l), the prediction row is
+ * C2[a][b] when its total is at least min_obs, else C[b]; preference order,
+ * confidence, visit order (confidence desc, t asc) and the capacity rule are
+ * those of md_token_shuffle applied to that row.
+ *
+ *   idx_prev   int32 [T, k]   layer-l-1 top-k (column 0 is the top-1)
+ *   idx_l      int32 [T, k]   layer-l top-k
+ *   C          uint32 [E, E]  layer l -> l+1 counts (md_coselect_stats)
+ *   C2         uint32 [E, E, E] pair counts (md_coselect_pair_stats)
+ *   min_obs    >= 1
+ *   use_pair   int32 [T] out (may be NULL): 1 where the pair row was used
+ *   other arguments as md_token_shuffle.
+ *   Limits: T % R == 0, E <= MD_MAX_PAIR_EXPERTS, R <= 64, T < 2^31; every
+ *   row total used must be below 2^31 (else MD_ERR_UNSUPPORTED in dev_status).
+ */
+size_t md_token_shuffle_pair_workspace_size(int64_t T, int E, int R);
+
+int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx_l, int k, const uint32_t *C,
+                          const uint32_t *C2, const int32_t *expert_to_rank_next, int64_t T, int E,
+                          int R, uint32_t min_obs, int32_t *pred_rank, int32_t *perm, int32_t *inv,
+                          int32_t *use_pair, void *workspace, size_t workspace_bytes,
+                          int32_t *dev_status, void *stream);
 
 /*
  * md_gather_rows -- dst[i] = src[index[i]] for i < n_out, rows of row_bytes.
