@@ -66,13 +66,17 @@ def _load():
             lib.oracle_place_correlated.argtypes = [P, I32, I32, I32, I32, P]
             lib.oracle_token_shuffle.argtypes = [P, P, P, I64, I32, I32, I32, P, P, P]
             lib.oracle_coselect_pair.argtypes = [P, P, P, I64, I32, I32, P]
+            lib.oracle_rank_stats.argtypes = [P, I64, I32, I32, I32, P, P]
+            lib.oracle_successor_share.argtypes = [P, P, I32, P, P]
+            lib.oracle_count_sums.argtypes = [P, P, I64, P]
             lib.oracle_token_shuffle_pair.argtypes = [P, P, P, P, P, I64, I32, I32, I32,
                                                       ctypes.c_uint64, P, P, P, P]
             for name in ("oracle_route_topk", "oracle_dispatch_layout", "oracle_dispatch_permute",
                          "oracle_dedup_expand",
                          "oracle_combine", "oracle_coselect", "oracle_place_correlated",
                          "oracle_token_shuffle", "oracle_coselect_pair",
-                         "oracle_token_shuffle_pair"):
+                         "oracle_token_shuffle_pair", "oracle_rank_stats",
+                         "oracle_successor_share", "oracle_count_sums"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -265,3 +269,46 @@ def token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_obs):
                                          int(min_obs), _ptr(pred), _ptr(perm), _ptr(inv), _ptr(use)),
            "token_shuffle_pair")
     return pred, perm, inv, use
+
+
+def rank_stats(idx, E, R, expert_to_rank):
+    """hist int64 [k+1]: tokens with exactly D distinct destination ranks."""
+    lib = _load()
+    ix = _c(idx, np.int32)
+    T, k = ix.shape
+    p = _c(expert_to_rank, np.int32)
+    hist = np.zeros(k + 1, np.int64)
+    _check(lib.oracle_rank_stats(_ptr(ix), T, E, k, R, _ptr(p), _ptr(hist)), "rank_stats")
+    return hist
+
+
+def successor_share(C, W):
+    """(num uint32 [E], den uint32 [E]): largest C[e, :] and W[e, e]."""
+    lib = _load()
+    Cc = _c(C, np.uint32)
+    Wc = _c(W, np.uint32)
+    E = Cc.shape[0]
+    num = np.empty(E, np.uint32)
+    den = np.empty(E, np.uint32)
+    _check(lib.oracle_successor_share(_ptr(Cc), _ptr(Wc), E, _ptr(num), _ptr(den)), "successor_share")
+    return num, den
+
+
+def count_sums(x, y):
+    """Exact (sx, sy, sxx, syy, sxy) of two uint32 count tables, as Python ints."""
+    lib = _load()
+    xc = _c(np.ravel(x), np.uint32)
+    yc = _c(np.ravel(y), np.uint32)
+    out = np.zeros(10, np.uint64)
+    _check(lib.oracle_count_sums(_ptr(xc), _ptr(yc), xc.shape[0], _ptr(out)), "count_sums")
+    return tuple(int(out[2 * i]) | (int(out[2 * i + 1]) << 64) for i in range(5))
+
+
+def pearson(x, y):
+    """Pearson correlation of two count tables from their exact sums."""
+    n = int(np.size(x))
+    sx, sy, sxx, syy, sxy = count_sums(x, y)
+    cov = n * sxy - sx * sy
+    vx = n * sxx - sx * sx
+    vy = n * syy - sy * sy
+    return cov / (vx * vy) ** 0.5 if vx > 0 and vy > 0 else float("nan")

@@ -814,3 +814,73 @@ done:
     free(pref); free(sigma); free(order); free(load);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Routing statistics.                                                       */
+/* [EC] Offline Placement and Prediction Statistics, Table I: "Same GPU" =   */
+/* share of tokens whose k experts all sit on one rank, "GPUs" = distinct    */
+/* ranks per token, "Dedup" = rows removed by deduplication = 1 - GPUs / k.  */
+/* hist[D] = number of tokens with exactly D distinct destination ranks.     */
+/* ------------------------------------------------------------------------ */
+
+int oracle_rank_stats(const int32_t *idx, int64_t T, int E, int k, int R, const int32_t *p,
+                      int64_t *hist)
+{
+    if (T < 0 || E < 1 || k < 1 || R < 1) return 1;
+    for (int d = 0; d <= k; ++d) hist[d] = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        int distinct = 0;
+        for (int j = 0; j < k; ++j) {
+            int e = idx[t * k + j];
+            if (e < 0 || e >= E || p[e] < 0 || p[e] >= R) return 1;
+            int seen = 0;
+            for (int i = 0; i < j; ++i)
+                if (p[idx[t * k + i]] == p[e]) seen = 1;
+            if (!seen) ++distinct;
+        }
+        hist[distinct] += 1;
+    }
+    return 0;
+}
+
+/* [EC] Cross-layer correlation: a layer-l expert "sends" a share of its      */
+/* tokens to one layer-l+1 expert.  With C (all k x k cross-layer pairs) and */
+/* W (diagonal = tokens selecting e) fitted on the same tokens, the share of */
+/* e's tokens that select e' next is C[e][e'] / W[e][e]; num[e] is the       */
+/* largest C[e][e'] and den[e] = W[e][e].                                    */
+int oracle_successor_share(const uint32_t *C, const uint32_t *W, int E, uint32_t *num,
+                           uint32_t *den)
+{
+    if (E < 1) return 1;
+    for (int e = 0; e < E; ++e) {
+        uint32_t m = 0;
+        for (int e2 = 0; e2 < E; ++e2)
+            if (C[(int64_t)e * E + e2] > m) m = C[(int64_t)e * E + e2];
+        num[e] = m;
+        den[e] = W[(int64_t)e * E + e];
+    }
+    return 0;
+}
+
+/* [EC] Correlation Formation and Stability: Pearson correlation between a    */
+/* fitted and a held-out count table.  The five sums are exact integers      */
+/* (128-bit); sums[0..4] = (sx, sy, sxx, syy, sxy), each as (low, high)      */
+/* 64-bit words.                                                             */
+int oracle_count_sums(const uint32_t *x, const uint32_t *y, int64_t n, uint64_t *sums)
+{
+    if (n < 0) return 1;
+    unsigned __int128 s[5] = {0, 0, 0, 0, 0};
+    for (int64_t i = 0; i < n; ++i) {
+        unsigned __int128 a = x[i], b = y[i];
+        s[0] += a;
+        s[1] += b;
+        s[2] += a * a;
+        s[3] += b * b;
+        s[4] += a * b;
+    }
+    for (int i = 0; i < 5; ++i) {
+        sums[2 * i] = (uint64_t)s[i];
+        sums[2 * i + 1] = (uint64_t)(s[i] >> 64);
+    }
+    return 0;
+}
