@@ -69,6 +69,7 @@ def _load():
             lib.oracle_rank_stats.argtypes = [P, I64, I32, I32, I32, P, P]
             lib.oracle_successor_share.argtypes = [P, P, I32, P, P]
             lib.oracle_count_sums.argtypes = [P, P, I64, P]
+            lib.oracle_place_two_level.argtypes = [P, I32, I32, I32, I32, I32, P]
             lib.oracle_token_shuffle_pair.argtypes = [P, P, P, P, P, I64, I32, I32, I32,
                                                       ctypes.c_uint64, P, P, P, P]
             for name in ("oracle_route_topk", "oracle_dispatch_layout", "oracle_dispatch_permute",
@@ -76,7 +77,8 @@ def _load():
                          "oracle_combine", "oracle_coselect", "oracle_place_correlated",
                          "oracle_token_shuffle", "oracle_coselect_pair",
                          "oracle_token_shuffle_pair", "oracle_rank_stats",
-                         "oracle_successor_share", "oracle_count_sums"):
+                         "oracle_successor_share", "oracle_count_sums",
+                         "oracle_place_two_level"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -312,3 +314,18 @@ def pearson(x, y):
     vx = n * sxx - sx * sx
     vy = n * syy - sy * sy
     return cov / (vx * vy) ** 0.5 if vx > 0 and vy > 0 else float("nan")
+
+
+REFINE_NONE, REFINE_SWAPS, REFINE_KL = 0, 1, 2
+
+
+def place_two_level(W, R, nodes=1, seed_mode=0, refine_mode=REFINE_SWAPS):
+    """Placement over `nodes` nodes of R/nodes ranks (nodes=1: one level), with
+    no refinement, best single swaps, or Kernighan-Lin passes."""
+    lib = _load()
+    Wc = _c(W, np.uint32)
+    E = Wc.shape[0]
+    p = np.empty(E, np.int32)
+    _check(lib.oracle_place_two_level(_ptr(Wc), E, R, nodes, seed_mode, refine_mode, _ptr(p)),
+           "place_two_level")
+    return p

@@ -884,3 +884,120 @@ int oracle_count_sums(const uint32_t *x, const uint32_t *y, int64_t n, uint64_t 
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Kernighan-Lin passes and two-level placement.                             */
+/* [EC] Correlated Placement: a Kernighan-Lin-style local search (Algorithm  */
+/* 1, not printed) swaps experts between GPUs; for multi-node groups the     */
+/* partition is made across nodes first, then across the GPUs of each node.  */
+/* A KL pass, as in Kernighan and Lin's graph bisection: repeatedly take the */
+/* best swap among experts not yet moved in this pass (gain may be           */
+/* negative; ties to the lowest (a, b)), move and lock both, until no        */
+/* unlocked pair on different ranks is left or E/2 swaps were made; then     */
+/* keep the shortest prefix of moves with the largest total gain and undo    */
+/* the rest.  Passes repeat while that total is positive (at most E passes). */
+/* ------------------------------------------------------------------------ */
+
+static void compute_A(const uint32_t *W, int E, int R, const int32_t *p, long long *A)
+{
+    for (int64_t i = 0; i < (int64_t)E * R; ++i) A[i] = 0;
+    for (int e = 0; e < E; ++e)
+        for (int e2 = 0; e2 < E; ++e2)
+            if (e2 != e) A[(int64_t)e * R + p[e2]] += W[(int64_t)e * E + e2];
+}
+
+static long long kl_pass(const uint32_t *W, int E, int R, int32_t *p, long long *A, char *locked,
+                         int *sa, int *sb, long long *sg)
+{
+    memset(locked, 0, (size_t)E);
+    int n = 0;
+    for (int step = 0; step < E / 2; ++step) {
+        compute_A(W, E, R, p, A);
+        int ba = -1, bb = -1;
+        long long best = 0;
+        for (int a = 0; a < E; ++a) {
+            if (locked[a]) continue;
+            for (int b = a + 1; b < E; ++b) {
+                if (locked[b] || p[a] == p[b]) continue;
+                int P = p[a], Q = p[b];
+                long long g = A[(int64_t)a * R + Q] - A[(int64_t)a * R + P] +
+                              A[(int64_t)b * R + P] - A[(int64_t)b * R + Q] -
+                              2LL * (long long)W[(int64_t)a * E + b];
+                if (ba < 0 || g > best) { best = g; ba = a; bb = b; }
+            }
+        }
+        if (ba < 0) break;
+        int P = p[ba];
+        p[ba] = p[bb];
+        p[bb] = P;
+        locked[ba] = locked[bb] = 1;
+        sa[n] = ba;
+        sb[n] = bb;
+        sg[n] = best;
+        ++n;
+    }
+    long long run = 0, keep = 0;
+    int m = 0;
+    for (int i = 0; i < n; ++i) {
+        run += sg[i];
+        if (run > keep) { keep = run; m = i + 1; }
+    }
+    for (int i = n - 1; i >= m; --i) {
+        int P = p[sa[i]];
+        p[sa[i]] = p[sb[i]];
+        p[sb[i]] = P;
+    }
+    return keep;
+}
+
+/* refine_mode: 0 none, 1 best single swaps (as oracle_place_correlated),
+ * 2 KL passes.  Single level. */
+static int place_one_level(const uint32_t *W, int E, int R, int seed_mode, int refine_mode,
+                           int32_t *p)
+{
+    int rc = oracle_place_correlated(W, E, R, seed_mode, refine_mode == 1, p);
+    if (rc || refine_mode != 2) return rc;
+    long long *A = (long long *)malloc(sizeof(long long) * (size_t)E * R);
+    char *locked = (char *)malloc((size_t)E);
+    int *sa = (int *)malloc(sizeof(int) * (size_t)(E / 2 + 1));
+    int *sb = (int *)malloc(sizeof(int) * (size_t)(E / 2 + 1));
+    long long *sg = (long long *)malloc(sizeof(long long) * (size_t)(E / 2 + 1));
+    if (!A || !locked || !sa || !sb || !sg) rc = 2;
+    for (int pass = 0; !rc && pass < E; ++pass)
+        if (kl_pass(W, E, R, p, A, locked, sa, sb, sg) <= 0) break;
+    free(A); free(locked); free(sa); free(sb); free(sg);
+    return rc;
+}
+
+/*
+ * Two-level placement over `nodes` nodes of R/nodes ranks each (nodes = 1:
+ * one level).  Level 1 places the experts on nodes (E/nodes each) with the
+ * seed and refinement given; level 2 places each node's experts, taken in
+ * ascending id, on its R/nodes ranks with W restricted to them.  p[e] =
+ * node * (R/nodes) + rank within the node.
+ */
+int oracle_place_two_level(const uint32_t *W, int E, int R, int nodes, int seed_mode,
+                           int refine_mode, int32_t *p)
+{
+    if (E < 1 || R < 1 || nodes < 1 || R % nodes != 0 || E % R != 0) return 1;
+    if (refine_mode < 0 || refine_mode > 2) return 1;
+    if (nodes == 1) return place_one_level(W, E, R, seed_mode, refine_mode, p);
+    const int G = R / nodes, En = E / nodes;
+    int32_t *pn = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    int *mem = (int *)malloc(sizeof(int) * (size_t)En);
+    uint32_t *sub = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)En * En);
+    int32_t *pg = (int32_t *)malloc(sizeof(int32_t) * (size_t)En);
+    int rc = (!pn || !mem || !sub || !pg) ? 2 : 0;
+    if (!rc) rc = place_one_level(W, E, nodes, seed_mode, refine_mode, pn);
+    for (int n = 0; !rc && n < nodes; ++n) {
+        int c = 0;
+        for (int e = 0; e < E; ++e)
+            if (pn[e] == n) mem[c++] = e;
+        for (int i = 0; i < En; ++i)
+            for (int j = 0; j < En; ++j) sub[(int64_t)i * En + j] = W[(int64_t)mem[i] * E + mem[j]];
+        rc = place_one_level(sub, En, G, seed_mode, refine_mode, pg);
+        for (int i = 0; !rc && i < En; ++i) p[mem[i]] = n * G + pg[i];
+    }
+    free(pn); free(mem); free(sub); free(pg);
+    return rc;
+}
