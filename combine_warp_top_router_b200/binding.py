@@ -24,6 +24,7 @@ MD_CONV, MD_DEDUP = 0, 1
 MD_GATE_TOPK_SOFTMAX, MD_GATE_FULL_SOFTMAX = 0, 1
 MD_COMBINE_FUSED, MD_COMBINE_WIRE = 0, 1
 MD_SEED_CONTIGUOUS, MD_SEED_GREEDY_PAIRS = 0, 1
+MD_REFINE_NONE, MD_REFINE_SWAPS, MD_REFINE_KL = 0, 1, 2
 
 _lock = threading.Lock()
 _lib = None
@@ -49,6 +50,11 @@ _SIGNATURES = {
     "md_token_shuffle_workspace_size": ([_L, _I, _I], _S),
     "md_token_shuffle": ([_P, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _S, _P, _P], _I),
     "md_coselect_pair_stats": ([_P, _P, _P, _L, _I, _I, _P, _I, _P, _P], _I),
+    "md_rank_stats": ([_P, _L, _I, _I, _I, _P, _P, _P, _P], _I),
+    "md_place_two_level_workspace_size": ([_I, _I, _I], _S),
+    "md_place_two_level": ([_P, _I, _I, _I, _I, _I, _P, _P, _S, _P, _P], _I),
+    "md_successor_share": ([_P, _P, _I, _P, _P, _P], _I),
+    "md_count_sums": ([_P, _P, _L, _P, _P], _I),
     "md_token_shuffle_pair_workspace_size": ([_L, _I, _I], _S),
     "md_token_shuffle_pair": ([_P, _P, _I, _P, _P, _P, _L, _I, _I, ctypes.c_uint32, _P, _P, _P, _P,
                                _P, _S, _P, _P], _I),
@@ -346,6 +352,25 @@ def md_place_correlated(W, R, seed_mode=MD_SEED_CONTIGUOUS, refine=True, out=Non
     return out
 
 
+def md_place_two_level(W, R, nodes=1, seed_mode=MD_SEED_CONTIGUOUS, refine_mode=MD_REFINE_SWAPS,
+                       out=None, workspace=None, dev_status=None, stream=None):
+    """Placement over `nodes` nodes of R/nodes ranks (nodes=1: one level), with no
+    refinement, best single swaps, or Kernighan-Lin passes."""
+    _need(W, "W", torch.int32)
+    dev = W.device
+    E = W.shape[0]
+    if out is None:
+        out = torch.empty(E, dtype=torch.int32, device=dev)
+    need = int(lib().md_place_two_level_workspace_size(E, R, nodes))
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    rc = lib().md_place_two_level(_ptr(W), E, R, nodes, seed_mode, refine_mode, _ptr(out),
+                                  _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                  _stream(stream, dev))
+    _check(rc, "md_place_two_level")
+    return out
+
+
 def md_token_shuffle(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None, inv=None,
                      workspace=None, dev_status=None, stream=None):
     _need(idx_l, "idx_l", torch.int32)
@@ -414,3 +439,61 @@ def md_token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_ob
                                      _stream(stream, dev))
     _check(rc, "md_token_shuffle_pair")
     return pred_rank, perm, inv, use_pair
+
+
+# ------------------------------------------------------------ statistics
+
+def md_rank_stats(topk_idx, E, R, expert_to_rank, hist=None, dev_status=None, stream=None):
+    """hist int64 [k+1]: tokens whose experts sit on exactly D distinct ranks."""
+    _need(topk_idx, "topk_idx", torch.int32)
+    dev = topk_idx.device
+    _need(expert_to_rank, "expert_to_rank", torch.int32, dev)
+    T, k = topk_idx.shape
+    hist = torch.empty(k + 1, dtype=torch.int64, device=dev) if hist is None else hist
+    _need(hist, "hist", torch.int64, dev)
+    rc = lib().md_rank_stats(_ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), _ptr(hist),
+                             _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_rank_stats")
+    return hist
+
+
+def table1_row(hist):
+    """Table I columns from a rank histogram: (same-rank %, ranks per token, dedup %)."""
+    h = [int(v) for v in hist.tolist()]
+    T, k = sum(h), len(h) - 1
+    gpus = sum(d * n for d, n in enumerate(h)) / T
+    return 100.0 * h[1] / T, gpus, 100.0 * (1.0 - gpus / k)
+
+
+def md_successor_share(C, W, stream=None):
+    """(num, den) int32 views of uint32 [E]: max_e' C[e, e'] and W[e, e]."""
+    _need(C, "C", torch.int32)
+    dev = C.device
+    _need(W, "W", torch.int32, dev)
+    E = C.shape[0]
+    num = torch.empty(E, dtype=torch.int32, device=dev)
+    den = torch.empty(E, dtype=torch.int32, device=dev)
+    rc = lib().md_successor_share(_ptr(C), _ptr(W), E, _ptr(num), _ptr(den), _stream(stream, dev))
+    _check(rc, "md_successor_share")
+    return num, den
+
+
+def md_count_sums(x, y, stream=None):
+    """Exact (sx, sy, sxx, syy, sxy) of two count tables (int32 views of uint32)."""
+    _need(x, "x", torch.int32)
+    dev = x.device
+    _need(y, "y", torch.int32, dev)
+    if x.numel() != y.numel():
+        raise MoeDispatchError("md_count_sums: tables differ in size")
+    out = torch.empty(10, dtype=torch.int64, device=dev)
+    rc = lib().md_count_sums(_ptr(x), _ptr(y), x.numel(), _ptr(out), _stream(stream, dev))
+    _check(rc, "md_count_sums")
+    w = [v & (2 ** 64 - 1) for v in out.cpu().tolist()]
+    return tuple(w[2 * i] | (w[2 * i + 1] << 64) for i in range(5))
+
+
+def pearson_from_sums(n, sums):
+    """Pearson correlation from the exact sums of md_count_sums."""
+    sx, sy, sxx, syy, sxy = sums
+    vx, vy = n * sxx - sx * sx, n * syy - sy * sy
+    return (n * sxy - sx * sy) / (vx * vy) ** 0.5 if vx > 0 and vy > 0 else float("nan")

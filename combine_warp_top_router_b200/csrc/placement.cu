@@ -86,6 +86,9 @@ struct Smem {
     int *cb;    // [E] refinement: best partner of row a (-1: no positive gain)
     int *list;  // [E] refinement: rows to rescan in this step
     long long *cg;  // [E] refinement: gain of (a, cb[a])
+    unsigned char *lock;  // [E] KL: moved in this pass
+    int *ka, *kb, *kP, *kQ;  // [E/2] KL: the moves of this pass
+    long long *kg;        // [E/2] KL: their gains
     long long *A;   // [E][ar]: A[e][d] at A[e * ar + d]
     int ar;         // row stride of A: R + 1, so that consecutive rows fall in different banks
 };
@@ -143,7 +146,10 @@ __device__ __forceinline__ long long gain_w(const Smem &s, int R, int a, int b, 
     return Aa[Q] - Aa[P] + Ab[P] - Ab[Q] - 2ll * (long long)wab;
 }
 
-// Best positive-gain partner b > a (p[b] != p[a]) of row a, lowest b on ties.
+// Best partner b > a (p[b] != p[a]) of row a, lowest b on ties: with a
+// positive gain for the swap search; any gain, among unlocked experts, in a
+// Kernighan-Lin pass (KL).  b = -1 when there is none.
+template <bool KL>
 __device__ __forceinline__ void refine_row(const uint32_t *__restrict__ W, const Smem &s, int E,
                                            int R, int a, long long &g_out, int &b_out)
 {
@@ -162,9 +168,9 @@ __device__ __forceinline__ void refine_row(const uint32_t *__restrict__ W, const
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int b = b0 + u * 32 + lane;
-            if (b >= E || s.p[b] == P) continue;
+            if (b >= E || s.p[b] == P || (KL && s.lock[b])) continue;
             const long long g = gain_w(s, R, a, b, wv[u]);
-            if (g > bg) {
+            if (KL ? (bb < 0 || g > bg) : g > bg) {
                 bg = g;
                 bb = b;
             }
@@ -183,15 +189,179 @@ __device__ __forceinline__ void refine_row(const uint32_t *__restrict__ W, const
     b_out = bb;
 }
 
+// Move a (rank P) to Q and b (rank Q) to P: columns P and Q of A, and (thread
+// 0) the rank lists.  The caller synchronises.
+__device__ __forceinline__ void apply_swap(const uint32_t *__restrict__ W, const Smem &s, int E,
+                                           int cap, int a, int b, int P, int Q)
+{
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+        const long long wa = e != a ? (long long)__ldg(W + (int64_t)e * E + a) : 0;
+        const long long wb = e != b ? (long long)__ldg(W + (int64_t)e * E + b) : 0;
+        s.A[(int64_t)e * s.ar + P] += wb - wa;
+        s.A[(int64_t)e * s.ar + Q] += wa - wb;
+    }
+    if (threadIdx.x == 0) {
+        const int sa = s.slot[a], sb = s.slot[b];
+        s.mem[P * cap + sa] = b;
+        s.mem[Q * cap + sb] = a;
+        s.slot[a] = sb;
+        s.slot[b] = sa;
+        s.p[a] = Q;
+        s.p[b] = P;
+    }
+}
+
+// The refinement.  !KL: repeat the best positive swap while there is one
+// (at most E*E).  KL: passes of tentative moves; each move is the best swap
+// among experts not yet moved in the pass, whatever its sign; the pass keeps
+// the shortest prefix of moves with the largest positive total and undoes
+// the rest; passes repeat while that total is positive (at most E passes).
+template <bool KL>
+__device__ void search(const uint32_t *__restrict__ W, const Smem &s, int E, int R, int cap,
+                       Cand *s_red, int *s_nlist, long long *s_keep, int *s_keep_m)
+{
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    const long long max_passes = KL ? E : 1;
+    const long long max_steps = KL ? E / 2 : (long long)E * E;
+    for (long long pass = 0; pass < max_passes; ++pass) {
+        for (int a = tid; a < E; a += kThreads) {
+            s.cb[a] = -1;
+            s.cg[a] = 0;
+            if (KL) s.lock[a] = 0;
+        }
+        if (tid == 0) *s_nlist = 0;
+        __syncthreads();
+        int lastP = -1, lastQ = -1;  // ranks of the last move (-1: scan every row)
+        int moves = 0;
+        for (long long it = 0; it < max_steps; ++it) {
+            // one thread per row: rows on lastP / lastQ, and rows whose partner
+            // sits there, are queued for a full rescan; every other row only
+            // compares its candidate with the pairs it forms with those ranks
+            for (int a = tid; a < E; a += kThreads) {
+                if (KL && s.lock[a]) {
+                    s.cb[a] = -1;
+                    continue;
+                }
+                const int pa = s.p[a];
+                long long cg = s.cg[a];
+                int cb = s.cb[a];
+                if (lastP < 0 || pa == lastP || pa == lastQ ||
+                    (cb >= 0 && (s.p[cb] == lastP || s.p[cb] == lastQ))) {
+                    s.list[atomicAdd(s_nlist, 1)] = a;
+                    continue;
+                }
+                const uint32_t *row = W + (int64_t)a * E;
+                for (int i0 = 0; i0 < 2 * cap; i0 += kBatch) {
+                    int bv[kBatch];
+                    uint32_t wv[kBatch];
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int i = i0 + u;
+                        bv[u] = i < 2 * cap ? s.mem[(i < cap ? lastP * cap + i : lastQ * cap + i - cap)]
+                                            : -1;
+                        wv[u] = bv[u] > a ? __ldg(row + bv[u]) : 0u;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int b = bv[u];
+                        if (b <= a || (KL && s.lock[b])) continue;
+                        const long long g = gain_w(s, R, a, b, wv[u]);
+                        if ((KL || g > 0) && (cb < 0 || g > cg || (g == cg && b < cb))) {
+                            cg = g;
+                            cb = b;
+                        }
+                    }
+                }
+                s.cg[a] = cg;
+                s.cb[a] = cb;
+            }
+            __syncthreads();
+            // the queued rows, one warp per row over all warps
+            const int nl = *s_nlist;
+            for (int i = wp; i < nl; i += kWarps) {
+                const int a = s.list[i];
+                long long g2;
+                int b2;
+                refine_row<KL>(W, s, E, R, a, g2, b2);
+                if (lane == 0) {
+                    s.cg[a] = g2;
+                    s.cb[a] = b2;
+                }
+            }
+            __syncthreads();
+            Cand v = {0, -1, -1, 0, 0};
+            for (int a = tid; a < E; a += kThreads) {
+                const int cb = s.cb[a];
+                if (cb < 0) continue;
+                const Cand c = {s.cg[a], a, cb, s.p[a], s.p[cb]};
+                if (better(c, v)) v = c;
+            }
+            v = warp_best(v);
+            if (lane == 0) s_red[wp] = v;
+            __syncthreads();
+            const Cand win = warp_best(s_red[lane]);
+            if (win.a < 0) break;  // uniform: every thread holds the same winner
+            apply_swap(W, s, E, cap, win.a, win.b, win.P, win.Q);
+            if (tid == 0) {
+                *s_nlist = 0;
+                if (KL) {
+                    s.lock[win.a] = 1;
+                    s.lock[win.b] = 1;
+                    s.ka[moves] = win.a;
+                    s.kb[moves] = win.b;
+                    s.kP[moves] = win.P;
+                    s.kQ[moves] = win.Q;
+                    s.kg[moves] = win.g;
+                }
+            }
+            ++moves;
+            lastP = win.P;
+            lastQ = win.Q;
+            __syncthreads();
+        }
+        if (!KL) break;
+        // keep the shortest prefix with the largest total gain, undo the rest
+        if (tid == 0) {
+            long long run = 0, keep = 0;
+            int m = 0;
+            for (int i = 0; i < moves; ++i) {
+                run += s.kg[i];
+                if (run > keep) {
+                    keep = run;
+                    m = i + 1;
+                }
+            }
+            *s_keep = keep;
+            *s_keep_m = m;
+        }
+        __syncthreads();
+        const int m = *s_keep_m;
+        const long long keep = *s_keep;
+        for (int i = moves - 1; i >= m; --i) {
+            // move i took a from P to Q and b from Q to P; take them back
+            apply_swap(W, s, E, cap, s.ka[i], s.kb[i], s.kQ[i], s.kP[i]);
+            __syncthreads();
+        }
+        if (keep <= 0) break;
+    }
+}
+
+// One CTA per independent problem (blockIdx.x): W, p_out and A_global point
+// at problem 0 and advance by E*E, E and E*(R+1).  refine: 0 none, 1 best
+// single swaps, 2 Kernighan-Lin passes.
 __global__ void __launch_bounds__(kThreads, 1)
     k_place(const uint32_t *__restrict__ W, int E, int R, int seed_mode, int refine,
             int32_t *__restrict__ p_out, long long *__restrict__ A_global, int a_in_smem)
 {
     extern __shared__ __align__(16) unsigned char sm_raw[];
     __shared__ Cand s_red[kWarps];
-    __shared__ int s_maxfree, s_roomiest, s_nlist;
+    __shared__ int s_maxfree, s_roomiest, s_nlist, s_keep_m;
+    __shared__ long long s_keep;
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     const int cap = E / R;
+    W += (int64_t)blockIdx.x * E * E;
+    p_out += (int64_t)blockIdx.x * E;
+    if (A_global) A_global += (int64_t)blockIdx.x * E * (R + 1);
 
     Smem s;
     s.A = a_in_smem ? reinterpret_cast<long long *>(sm_raw) : A_global;
@@ -204,6 +374,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     s.slot = ip + 2 * E + R;
     s.cb = ip + 3 * E + R;
     s.list = ip + 4 * E + R;
+    {
+        // KL records after the int arrays: ka, kb, kP, kQ [E/2 + 1] ints, kg
+        // [E/2 + 1] int64 (8-byte aligned), lock [E] bytes
+        int *kp = ip + 5 * E + R;
+        const int h = E / 2 + 1;
+        s.ka = kp;
+        s.kb = kp + h;
+        s.kP = kp + 2 * h;
+        s.kQ = kp + 3 * h;
+        unsigned char *after = reinterpret_cast<unsigned char *>(kp + 4 * h);
+        after = reinterpret_cast<unsigned char *>(((uintptr_t)after + 7) & ~(uintptr_t)7);
+        s.kg = reinterpret_cast<long long *>(after);
+        s.lock = reinterpret_cast<unsigned char *>(s.kg + h);
+    }
 
     // greedy seed: lane j of warp w keeps the candidate of row w + 32 j
     const int a_own = wp + 32 * lane;
@@ -308,104 +492,93 @@ __global__ void __launch_bounds__(kThreads, 1)
                               (unsigned long long)row[e2]);
         }
         __syncthreads();
-
-        for (int a = tid; a < E; a += kThreads) {
-            s.cb[a] = -1;
-            s.cg[a] = 0;
-        }
-        if (tid == 0) s_nlist = 0;
-        __syncthreads();
-        int lastP = -1, lastQ = -1;  // ranks of the last swap (-1: scan every row)
-        for (long long it = 0; it < (long long)E * E; ++it) {
-            // one thread per row: rows on lastP / lastQ, and rows whose partner
-            // sits there, are queued for a full rescan; every other row only
-            // compares its candidate with the pairs it forms with those ranks
-            for (int a = tid; a < E; a += kThreads) {
-                const int pa = s.p[a];
-                long long cg = s.cg[a];
-                int cb = s.cb[a];
-                if (lastP < 0 || pa == lastP || pa == lastQ ||
-                    (cb >= 0 && (s.p[cb] == lastP || s.p[cb] == lastQ))) {
-                    s.list[atomicAdd(&s_nlist, 1)] = a;
-                    continue;
-                }
-                const uint32_t *row = W + (int64_t)a * E;
-                for (int i0 = 0; i0 < 2 * cap; i0 += kBatch) {
-                    int bv[kBatch];
-                    uint32_t wv[kBatch];
-#pragma unroll
-                    for (int u = 0; u < kBatch; ++u) {
-                        const int i = i0 + u;
-                        bv[u] = i < 2 * cap ? s.mem[(i < cap ? lastP * cap + i : lastQ * cap + i - cap)]
-                                            : -1;
-                        wv[u] = bv[u] > a ? __ldg(row + bv[u]) : 0u;
-                    }
-#pragma unroll
-                    for (int u = 0; u < kBatch; ++u) {
-                        const int b = bv[u];
-                        if (b <= a) continue;
-                        const long long g = gain_w(s, R, a, b, wv[u]);
-                        if (g > 0 && (cb < 0 || g > cg || (g == cg && b < cb))) {
-                            cg = g;
-                            cb = b;
-                        }
-                    }
-                }
-                s.cg[a] = cg;
-                s.cb[a] = cb;
-            }
-            __syncthreads();
-            // the queued rows, one warp per row over all warps
-            const int nl = s_nlist;
-            for (int i = wp; i < nl; i += kWarps) {
-                const int a = s.list[i];
-                long long g2;
-                int b2;
-                refine_row(W, s, E, R, a, g2, b2);
-                if (lane == 0) {
-                    s.cg[a] = g2;
-                    s.cb[a] = b2;
-                }
-            }
-            __syncthreads();
-            Cand v = {0, -1, -1, 0, 0};
-            for (int a = tid; a < E; a += kThreads) {
-                const int cb = s.cb[a];
-                if (cb < 0) continue;
-                const Cand c = {s.cg[a], a, cb, s.p[a], s.p[cb]};
-                if (better(c, v)) v = c;
-            }
-            v = warp_best(v);
-            if (lane == 0) s_red[wp] = v;
-            __syncthreads();
-            const Cand win = warp_best(s_red[lane]);
-            if (win.a < 0) break;
-            const int a = win.a, b = win.b, P = win.P, Q = win.Q;
-            for (int e = tid; e < E; e += kThreads) {
-                const long long wa = e != a ? (long long)__ldg(W + (int64_t)e * E + a) : 0;
-                const long long wb = e != b ? (long long)__ldg(W + (int64_t)e * E + b) : 0;
-                s.A[(int64_t)e * s.ar + P] += wb - wa;
-                s.A[(int64_t)e * s.ar + Q] += wa - wb;
-            }
-            if (tid == 0) {
-                const int sa = s.slot[a], sb = s.slot[b];
-                s.mem[P * cap + sa] = b;
-                s.mem[Q * cap + sb] = a;
-                s.slot[a] = sb;
-                s.slot[b] = sa;
-                s.p[a] = Q;
-                s.p[b] = P;
-                s_nlist = 0;
-            }
-            lastP = P;
-            lastQ = Q;
-            __syncthreads();
-        }
+        if (refine == 1) search<false>(W, s, E, R, cap, s_red, &s_nlist, &s_keep, &s_keep_m);
+        else search<true>(W, s, E, R, cap, s_red, &s_nlist, &s_keep, &s_keep_m);
     }
     for (int e = tid; e < E; e += kThreads) p_out[e] = s.p[e];
 }
 
-size_t int_smem(int E, int R) { return (size_t)E * sizeof(long long) + (size_t)(5 * E + R) * sizeof(int); }
+size_t int_smem(int E, int R)
+{
+    const size_t h = (size_t)E / 2 + 1;
+    return (size_t)E * sizeof(long long) + (size_t)(5 * E + R) * sizeof(int) + 4 * h * sizeof(int) +
+           8 + h * sizeof(long long) + (size_t)E;
+}
+
+// Two-level placement, between the levels: the experts of each node in
+// ascending id (mem[n*En + i]) and the node's restriction of W
+// (sub[n][i][j] = W[mem_i][mem_j]).  One CTA; E <= 1024.
+__global__ void __launch_bounds__(kThreads)
+    k_node_split(const uint32_t *__restrict__ W, int E, int nodes, const int32_t *__restrict__ pn,
+                 int32_t *__restrict__ mem, uint32_t *__restrict__ sub)
+{
+    const int En = E / nodes;
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+        const int n = pn[e];
+        int pos = 0;
+        for (int e2 = 0; e2 < e; ++e2) pos += pn[e2] == n;
+        mem[n * En + pos] = e;
+    }
+    __syncthreads();
+    const int64_t cells = (int64_t)E * En;  // nodes * En * En
+    for (int64_t c = threadIdx.x; c < cells; c += kThreads) {
+        const int n = (int)(c / ((int64_t)En * En));
+        const int64_t r = c - (int64_t)n * En * En;
+        const int i = (int)(r / En), j = (int)(r - (int64_t)i * En);
+        sub[c] = W[(int64_t)mem[n * En + i] * E + mem[n * En + j]];
+    }
+}
+
+// p[mem[n*En + i]] = n * G + pg[n*En + i]
+__global__ void k_node_merge(int E, int nodes, int G, const int32_t *__restrict__ mem,
+                             const int32_t *__restrict__ pg, int32_t *__restrict__ p)
+{
+    const int En = E / nodes;
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < E; c += gridDim.x * blockDim.x)
+        p[mem[c]] = (c / En) * G + pg[c];
+}
+
+int launch_place(const uint32_t *W, int problems, int E, int R, int seed_mode, int refine,
+                 int32_t *p, long long *A, cudaStream_t s)
+{
+    const size_t a_bytes = (size_t)E * (R + 1) * sizeof(long long);
+    const int a_in_smem = refine && a_bytes <= kSmemA ? 1 : 0;
+    const size_t smem = int_smem(E, R) + (a_in_smem ? a_bytes : 0);
+    if (cudaFuncSetAttribute(k_place, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+        return MD_ERR_CUDA;
+    k_place<<<problems, kThreads, smem, s>>>(W, E, R, seed_mode, refine, p, A, a_in_smem);
+    md::count_launches(1);
+    return MD_OK;
+}
+
+struct PlaceWs {
+    long long *A1, *A2;
+    int32_t *pn, *mem, *pg;
+    uint32_t *sub;
+};
+
+size_t place_layout(int E, int R, int nodes, PlaceWs *w, void *base)
+{
+    char *b = static_cast<char *>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        char *q = b ? b + o : nullptr;
+        o += md::align_up(bytes, 256);
+        return q;
+    };
+    PlaceWs x{};
+    x.A1 = reinterpret_cast<long long *>(take((size_t)E * (nodes + 1) * sizeof(long long)));
+    if (nodes > 1) {
+        x.A2 = reinterpret_cast<long long *>(take((size_t)E * (R / nodes + 1) * sizeof(long long)));
+        x.pn = reinterpret_cast<int32_t *>(take((size_t)E * 4));
+        x.mem = reinterpret_cast<int32_t *>(take((size_t)E * 4));
+        x.pg = reinterpret_cast<int32_t *>(take((size_t)E * 4));
+        x.sub = reinterpret_cast<uint32_t *>(take((size_t)E * (E / nodes) * 4));
+    }
+    if (w) *w = x;
+    return o;
+}
 
 }  // namespace
 
@@ -428,14 +601,48 @@ extern "C" int md_place_correlated(const uint32_t *W, int E, int R, int seed_mod
     cudaStream_t s = md::as_stream(stream);
     int rc = md::clear_status(dev_status, s);
     if (rc != MD_OK) return rc;
-    const size_t a_bytes = (size_t)E * (R + 1) * sizeof(long long);
-    const int a_in_smem = refine && a_bytes <= kSmemA ? 1 : 0;
-    const size_t smem = int_smem(E, R) + (a_in_smem ? a_bytes : 0);
-    if (cudaFuncSetAttribute(k_place, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-        return MD_ERR_CUDA;
-    k_place<<<1, kThreads, smem, s>>>(W, E, R, seed_mode, refine ? 1 : 0, expert_to_rank,
-                                      static_cast<long long *>(workspace), a_in_smem);
+    rc = launch_place(W, 1, E, R, seed_mode, refine ? 1 : 0, expert_to_rank,
+                      static_cast<long long *>(workspace), s);
+    return rc != MD_OK ? rc : md::launch_status();
+}
+
+extern "C" size_t md_place_two_level_workspace_size(int E, int R, int nodes)
+{
+    if (E < 1 || R < 1 || nodes < 1 || R % nodes != 0) return 0;
+    return place_layout(E, R, nodes, nullptr, nullptr);
+}
+
+extern "C" int md_place_two_level(const uint32_t *W, int E, int R, int nodes, int seed_mode,
+                                  int refine_mode, int32_t *expert_to_rank, void *workspace,
+                                  size_t workspace_bytes, int32_t *dev_status, void *stream)
+{
+    if (E < 1 || R < 1 || nodes < 1 || R % nodes != 0 || E % R != 0) return MD_ERR_ARG;
+    if (E > MD_MAX_EXPERTS || R > MD_MAX_RANKS) return MD_ERR_UNSUPPORTED;
+    if (seed_mode != MD_SEED_CONTIGUOUS && seed_mode != MD_SEED_GREEDY_PAIRS) return MD_ERR_ARG;
+    if (refine_mode != MD_REFINE_NONE && refine_mode != MD_REFINE_SWAPS &&
+        refine_mode != MD_REFINE_KL)
+        return MD_ERR_ARG;
+    if (!W || !expert_to_rank) return MD_ERR_ARG;
+    if (!workspace || workspace_bytes < md_place_two_level_workspace_size(E, R, nodes))
+        return MD_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MD_ERR_ARG;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK) return rc;
+    PlaceWs w;
+    place_layout(E, R, nodes, &w, workspace);
+    if (nodes == 1) {
+        rc = launch_place(W, 1, E, R, seed_mode, refine_mode, expert_to_rank, w.A1, s);
+        return rc != MD_OK ? rc : md::launch_status();
+    }
+    const int G = R / nodes, En = E / nodes;
+    rc = launch_place(W, 1, E, nodes, seed_mode, refine_mode, w.pn, w.A1, s);
+    if (rc != MD_OK) return rc;
+    k_node_split<<<1, kThreads, 0, s>>>(W, E, nodes, w.pn, w.mem, w.sub);
+    md::count_launches(1);
+    rc = launch_place(w.sub, nodes, En, G, seed_mode, refine_mode, w.pg, w.A2, s);
+    if (rc != MD_OK) return rc;
+    k_node_merge<<<(E + 255) / 256, 256, 0, s>>>(E, nodes, G, w.mem, w.pg, expert_to_rank);
     md::count_launches(1);
     return md::launch_status();
 }

@@ -64,6 +64,9 @@ typedef enum md_status {
 #define MD_SEED_CONTIGUOUS 0   /* placement search starts contiguous       */
 #define MD_SEED_GREEDY_PAIRS 1 /* placement search starts from greedy pairs*/
 #define MD_MAX_PAIR_EXPERTS 256 /* pair counts are E^3 entries               */
+#define MD_REFINE_NONE 0       /* placement: seed only                      */
+#define MD_REFINE_SWAPS 1      /* best positive single swaps                */
+#define MD_REFINE_KL 2         /* Kernighan-Lin passes                      */
 
 #define MD_MAX_TOPK 32
 #define MD_MAX_EXPERTS 1024
@@ -296,6 +299,31 @@ int md_place_correlated(const uint32_t *W, int E, int R, int seed_mode, int refi
                         int32_t *dev_status, void *stream);
 
 /*
+ * md_place_two_level -- placement with a choice of refinement and, for
+ * multi-node groups, two levels ("Expert Coupling ...", Correlated
+ * Placement: first across nodes, then across the GPUs within each node).
+ *
+ *   nodes        >= 1, R % nodes == 0; nodes == 1 is one level
+ *   seed_mode    as md_place_correlated, at both levels
+ *   refine_mode  MD_REFINE_NONE, MD_REFINE_SWAPS (as md_place_correlated) or
+ *                MD_REFINE_KL: Kernighan-Lin passes -- in a pass, repeatedly
+ *                the best swap among experts not yet moved in the pass
+ *                (gain of any sign, lowest (a, b) on ties) until none is left
+ *                or E/2 moves; keep the shortest prefix with the largest
+ *                positive total, undo the rest; repeat while positive (at
+ *                most E passes)
+ *   Level 1 places experts on nodes (E/nodes each); level 2 places each
+ *   node's experts, in ascending id, on its R/nodes ranks with W restricted
+ *   to them: expert_to_rank[e] = node * (R/nodes) + rank within the node.
+ *   Limits: E % R == 0, E <= 1024, R <= 64.
+ */
+size_t md_place_two_level_workspace_size(int E, int R, int nodes);
+
+int md_place_two_level(const uint32_t *W, int E, int R, int nodes, int seed_mode, int refine_mode,
+                       int32_t *expert_to_rank, void *workspace, size_t workspace_bytes,
+                       int32_t *dev_status, void *stream);
+
+/*
  * md_token_shuffle -- capacity-constrained token shuffle to predicted owners.
  * "Expert Coupling ...", Method 2 (Token Shuffling), Mechanism: predict each
  * token's owner rank at layer l+1; every rank owns exactly T/EP tokens, so
@@ -362,6 +390,34 @@ int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx_l, int k, 
  */
 int md_gather_rows(const void *src, int64_t src_rows, int64_t row_bytes, const int32_t *index,
                    int64_t n_out, void *dst, int32_t *dev_status, void *stream);
+
+/*
+ * Routing statistics ("Expert Coupling ...").
+ *
+ * md_rank_stats -- Table I (Offline Placement and Prediction Statistics):
+ *   hist  int64 [k+1] device, out: hist[D] = tokens whose k experts sit on
+ *         exactly D distinct ranks under expert_to_rank.  "Same GPU" =
+ *         hist[1] / T, "GPUs" = sum D hist[D] / T, "Dedup" = 1 - GPUs / k.
+ *   An expert or rank out of range is reported (MD_ERR_DATA).
+ *
+ * md_successor_share -- Cross-layer correlation: with C (md_coselect_stats,
+ *   layers l, l+1) and W (layer l) fitted on the same tokens, the share of
+ *   expert e's tokens that select e' next is C[e][e'] / W[e][e].
+ *   num uint32 [E] out: max_e' C[e][e'];  den uint32 [E] out: W[e][e].
+ *
+ * md_count_sums -- Correlation Formation and Stability: the Pearson
+ *   correlation of two count tables x, y (uint32 [n]) follows from
+ *   sums uint64 [10] device, out: (sx, sy, sxx, syy, sxy), each exact as a
+ *   128-bit value in two words (low, high).  n < 2^31.
+ */
+int md_rank_stats(const int32_t *topk_idx, int64_t T, int E, int k, int R,
+                  const int32_t *expert_to_rank, int64_t *hist, int32_t *dev_status,
+                  void *stream);
+
+int md_successor_share(const uint32_t *C, const uint32_t *W, int E, uint32_t *num, uint32_t *den,
+                       void *stream);
+
+int md_count_sums(const uint32_t *x, const uint32_t *y, int64_t n, uint64_t *sums, void *stream);
 
 #ifdef __cplusplus
 }

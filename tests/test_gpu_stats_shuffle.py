@@ -182,3 +182,44 @@ def test_shuffle_full_size_and_gather_round_trip():
     assert np.array_equal(perm.cpu().numpy(), want[1])
     assert np.array_equal(inv.cpu().numpy(), want[2])
     assert torch.equal(back, w.x)  # shuffle then restore is the identity
+
+
+# ------------------------------------------------- KL passes and two levels
+@pytest.mark.parametrize("E,R,nodes,hi", [(8, 2, 1, 4), (64, 8, 1, 1000), (128, 16, 1, 5),
+                                          (256, 64, 1, 4), (128, 16, 4, 9), (256, 64, 8, 50),
+                                          (64, 8, 8, 7), (1024, 64, 8, 9)])
+@pytest.mark.parametrize("refine_mode", [0, 1, 2])
+@pytest.mark.parametrize("seed_mode", [0, 1])
+def test_place_two_level_matches_oracle(E, R, nodes, hi, refine_mode, seed_mode):
+    if E == 1024 and refine_mode == 2 and seed_mode == 1:
+        pytest.skip("covered by the contiguous seed at this size (oracle minutes)")
+    W = _random_w(E, E * 3 + R + nodes, hi)
+    p = md.md_place_two_level(torch.from_numpy(W.view(np.int32)).to(DEV), R, nodes, seed_mode,
+                              refine_mode)
+    torch.cuda.synchronize()
+    want = oracle.place_two_level(W, R, nodes, seed_mode, refine_mode)
+    assert np.array_equal(p.cpu().numpy(), want)
+
+
+def test_kl_escapes_where_swaps_stop():
+    # the 8-expert instance from the oracle pins: KL reaches the optimum 24
+    from test_oracle_placement_kl import W_STUCK
+    Wd = torch.from_numpy(W_STUCK.view(np.int32)).to(DEV)
+    sw = md.md_place_two_level(Wd, 2, 1, 0, md.MD_REFINE_SWAPS)
+    kl = md.md_place_two_level(Wd, 2, 1, 0, md.MD_REFINE_KL)
+    torch.cuda.synchronize()
+    assert oracle.placement_objective(W_STUCK, sw.cpu().numpy()) == 22
+    assert oracle.placement_objective(W_STUCK, kl.cpu().numpy()) == 24
+
+
+@pytest.mark.parametrize("nodes", [1, 8])
+@pytest.mark.parametrize("refine_mode", [1, 2])
+def test_place_two_level_full_workload(nodes, refine_mode):
+    # full-pipeline workload: W over all T=262144 tokens, E=256, R=64
+    w = synth.make_workload("full_e256_k8", device=DEV, with_rows=False)
+    a, _ = md.md_route_topk(w.logits, 8)
+    W, _ = md.md_coselect_stats(a, None, 256)
+    p = md.md_place_two_level(W, 64, nodes, 0, refine_mode)
+    torch.cuda.synchronize()
+    want = oracle.place_two_level(u32(W), 64, nodes, 0, refine_mode)
+    assert np.array_equal(p.cpu().numpy(), want)
