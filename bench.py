@@ -478,6 +478,36 @@ def run_rows(args, md, device, stream, peak):
     contiguous = synth.contiguous_placement(E, R, device)
     torch.cuda.synchronize()
     Lc = md.md_dispatch_layout(a, E, R, contiguous, md.MD_DEDUP)
+    # placement refinements on this workload: best single swaps vs
+    # Kernighan-Lin passes, one level vs 8 nodes of 8 GPUs
+    modes = {}
+    for label, nodes, refine in (("swaps", 1, md.MD_REFINE_SWAPS), ("kl", 1, md.MD_REFINE_KL),
+                                 ("kl_8_nodes", 8, md.MD_REFINE_KL)):
+        q = torch.empty(E, dtype=torch.int32, device=device)
+        qws = md.alloc_workspace(int(md.lib().md_place_two_level_workspace_size(E, R, nodes)), device)
+        t_q = _time(lambda: md.md_place_two_level(W, R, nodes, md.MD_SEED_CONTIGUOUS, refine, out=q,
+                                                  workspace=qws, stream=stream), stream, 3)
+        torch.cuda.synchronize()
+        Lq = md.md_dispatch_layout(a, E, R, q, md.MD_DEDUP)
+        modes[label] = {"us": round(t_q * 1e3, 1),
+                        "rows_per_token": round(int(Lq.n_rows.item()) / T, 4)}
+    rows["placement_modes_e256_k8"] = modes
+
+    # the pages' routing statistics on this workload: Table I columns for both
+    # placements, the cross-layer successor share, fitted vs held-out W
+    s_corr = md.table1_row(md.md_rank_stats(a, E, R, p))
+    s_cont = md.table1_row(md.md_rank_stats(a, E, R, contiguous))
+    Wf, Cf = md.md_coselect_stats(a[:4096], b[:4096], E)
+    Wh, _ = md.md_coselect_stats(a[4096:8192], None, E)
+    num, den = md.md_successor_share(Cf, Wf)
+    share = (num.double() / den.double().clamp(min=1)).cpu()
+    rows["routing_stats_e256_k8"] = {
+        "same_rank_pct": {"contiguous": round(s_cont[0], 2), "correlated": round(s_corr[0], 2)},
+        "ranks_per_token": {"contiguous": round(s_cont[1], 3), "correlated": round(s_corr[1], 3)},
+        "dedup_pct": {"contiguous": round(s_cont[2], 2), "correlated": round(s_corr[2], 2)},
+        "experts_with_successor_share_ge_30pct": int((share >= 0.30).sum()),
+        "median_successor_share": round(float(share.median()), 4),
+        "pearson_W_fit4096_vs_next4096": round(md.pearson_from_sums(E * E, md.md_count_sums(Wf, Wh)), 4)}
     rows["full_e256_k8_pipeline"] = {
         "T": T, "ms": round(total, 3), "Mtokens_per_s": round(T / (total * 1e-3) / 1e6, 2),
         "parts_us": {kk: round(v * 1e3, 1) for kk, v in parts.items()},

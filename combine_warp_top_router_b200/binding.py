@@ -51,6 +51,7 @@ _SIGNATURES = {
     "md_token_shuffle": ([_P, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _S, _P, _P], _I),
     "md_coselect_pair_stats": ([_P, _P, _P, _L, _I, _I, _P, _I, _P, _P], _I),
     "md_rank_stats": ([_P, _L, _I, _I, _I, _P, _P, _P, _P], _I),
+    "md_set_test_hooks": ([ctypes.c_longlong, _I, ctypes.c_longlong], None),
     "md_place_two_level_workspace_size": ([_I, _I, _I], _S),
     "md_place_two_level": ([_P, _I, _I, _I, _I, _I, _P, _P, _S, _P, _P], _I),
     "md_successor_share": ([_P, _P, _I, _P, _P, _P], _I),
@@ -497,3 +498,8 @@ def pearson_from_sums(n, sums):
     sx, sy, sxx, syy, sxy = sums
     vx, vy = n * sxx - sx * sx, n * syy - sy * sy
     return (n * sxy - sx * sy) / (vx * vy) ** 0.5 if vx > 0 and vy > 0 else float("nan")
+
+
+def md_set_test_hooks(poll_limit=0, layout_skip_tile=-1, expand_skip_unit=-1):
+    """Fault injection for tests: make a bounded device-side wait run out."""
+    lib().md_set_test_hooks(int(poll_limit), int(layout_skip_tile), int(expand_skip_unit))

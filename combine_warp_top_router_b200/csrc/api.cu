@@ -6,7 +6,28 @@
 namespace md {
 static std::atomic<uint64_t> g_launches{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// Fault injection for tests (md_set_test_hooks): a short poll limit and one
+// publish / one copy left out, so that a bounded wait runs out.
+static std::atomic<long long> g_poll_limit{0};
+static std::atomic<int> g_layout_skip_tile{-1};
+static std::atomic<long long> g_expand_skip_unit{-1};
+long long hook_poll_limit(long long dflt)
+{
+    const long long v = g_poll_limit.load(std::memory_order_relaxed);
+    return v > 0 ? v : dflt;
+}
+int hook_layout_skip_tile() { return g_layout_skip_tile.load(std::memory_order_relaxed); }
+long long hook_expand_skip_unit() { return g_expand_skip_unit.load(std::memory_order_relaxed); }
 }  // namespace md
+
+extern "C" void md_set_test_hooks(long long poll_limit, int layout_skip_tile,
+                                  long long expand_skip_unit)
+{
+    md::g_poll_limit.store(poll_limit, std::memory_order_relaxed);
+    md::g_layout_skip_tile.store(layout_skip_tile, std::memory_order_relaxed);
+    md::g_expand_skip_unit.store(expand_skip_unit, std::memory_order_relaxed);
+}
 
 extern "C" const char *md_status_string(int status)
 {

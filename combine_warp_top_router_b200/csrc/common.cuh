@@ -5,6 +5,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "moedispatch.h"
 
 namespace md {
@@ -13,6 +15,11 @@ namespace md {
 
 // Host-side count of enqueued kernels / memsets (md_launch_count).
 void count_launches(int n);
+
+// Test hooks (md_set_test_hooks); the defaults leave every kernel unchanged.
+long long hook_poll_limit(long long dflt);
+int hook_layout_skip_tile();        // -1: none
+long long hook_expand_skip_unit();  // -1: none
 
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -45,6 +52,18 @@ inline int sm_count()
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Run f() once per device of the process (function attributes are per device).
+template <class F>
+inline void once_per_device(std::atomic<uint64_t> &done, F f)
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load(std::memory_order_acquire) & bit) return;
+    f();
+    done.fetch_or(bit, std::memory_order_acq_rel);
+}
 
 // -------------------------------------------------------------- device side
 

@@ -149,12 +149,11 @@ extern "C" int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, 
     }
     if (T_fit == 0) return MD_OK;
 
-    static bool attr_set = false;
-    if (!attr_set) {
+    static std::atomic<uint64_t> attr_done{0};
+    md::once_per_device(attr_done, [] {
         cudaFuncSetAttribute(k_coselect, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kSegEntries * (int)sizeof(uint32_t));
-        attr_set = true;
-    }
+    });
     const int64_t n_tri = (int64_t)E * (E + 1) / 2;
     const int64_t n_total = (W ? n_tri : 0) + (C ? (int64_t)E * E : 0);
     const int64_t n_seg = (n_total + kSegEntries - 1) / kSegEntries;

@@ -31,7 +31,8 @@ constexpr long long kPolls = 1ll << 22;
 __global__ void __launch_bounds__(kWarps * 32)
     k_expand_tma(const char *__restrict__ wire, int64_t n_wire, int rowbytes, int pieces,
                  const int32_t *__restrict__ row_of_slot, const int32_t *__restrict__ assign_row,
-                 int64_t n_slots, int64_t out_rows, char *__restrict__ out, int32_t *status)
+                 int64_t n_slots, int64_t out_rows, char *__restrict__ out, int32_t *status,
+                 long long polls, int64_t skip_unit)
 {
     extern __shared__ __align__(128) unsigned char ring_all[];
     __shared__ uint64_t bars[kWarps][kStages];
@@ -77,6 +78,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         return j < 32 ? a : b;
     };
     auto issue = [&](int64_t u, int src, int st) {
+        if (u == skip_unit) return;  // test hook: this unit's slot never completes
         if (src >= 0 && src < n_wire) {
             const uint32_t nb = bytes_of(u);
             md::mbar_expect_tx(&bar[st], nb);
@@ -113,7 +115,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         const int src = __shfl_sync(0xffffffffu, cs, j);
         const int dst = __shfl_sync(0xffffffffu, cd, j);
         int ok = 1;
-        if (lane == 0) ok = md::mbar_wait_bounded(&bar[st], (uint32_t)((i / kStages) & 1), kPolls);
+        if (lane == 0) ok = md::mbar_wait_bounded(&bar[st], (uint32_t)((i / kStages) & 1), polls);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
             md::report(status, MD_ERR_TIMEOUT);
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(kWarps * 32)
                 for (int a = 1; a <= kAhead; ++a)
                     if (u + a * nw < U)
                         md::mbar_wait_bounded(&bar[(i + a) % kStages],
-                                              (uint32_t)(((i + a) / kStages) & 1), kPolls);
+                                              (uint32_t)(((i + a) / kStages) & 1), polls);
             break;
         }
         const bool valid = src >= 0 && src < n_wire && dst >= 0 && dst < out_rows;
@@ -183,7 +185,8 @@ extern "C" int md_dedup_expand(const void *wire, int64_t n_wire, int H, const in
         if (blocks > md::sm_count()) blocks = md::sm_count();
         k_expand_tma<<<(unsigned)(blocks < 1 ? 1 : blocks), kWarps * 32, smem, s>>>(
             static_cast<const char *>(wire), n_wire, rowbytes, pieces, row_of_slot, assign_row,
-            n_slots, out_rows, static_cast<char *>(out), dev_status);
+            n_slots, out_rows, static_cast<char *>(out), dev_status, md::hook_poll_limit(kPolls),
+            md::hook_expand_skip_unit());
     } else {
         int64_t blocks = (n_slots + 7) / 8;
         const int64_t cap = (int64_t)md::sm_count() * 8;

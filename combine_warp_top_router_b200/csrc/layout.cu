@@ -37,6 +37,8 @@ constexpr unsigned long long kValMask = (1ull << 62) - 1;
 constexpr long long kPollLimit = 1ll << 22;
 
 struct Ws {
+    long long poll_limit;         // bound of every lookback wait
+    int skip_tile;                // test hook: this tile publishes nothing (-1: none)
     unsigned int *ctrl;           // [0] rank tile ticket
     int *hist_e;                  // [E]   assignments per expert
     int *send;                    // [R*R] rows per (source, destination)
@@ -80,6 +82,8 @@ Ws carve(void *ws, const Plan &p)
 {
     char *b = static_cast<char *>(ws);
     Ws w;
+    w.poll_limit = md::hook_poll_limit(kPollLimit);
+    w.skip_tile = md::hook_layout_skip_tile();
     w.ctrl = reinterpret_cast<unsigned int *>(b);
     w.hist_e = reinterpret_cast<int *>(b + p.off_hist);
     w.send = reinterpret_cast<int *>(b + p.off_send);
@@ -409,8 +413,9 @@ __global__ void __launch_bounds__(kRankThreads, 1)
             run += c;
         }
         s_pref[b] = run;
-        md::st_relaxed_u64(ws.tiles + (size_t)b * n_tiles + tile,
-                           (tile == 0 ? kFlagP : kFlagA) | (unsigned long long)run);
+        if (tile != ws.skip_tile)
+            md::st_relaxed_u64(ws.tiles + (size_t)b * n_tiles + tile,
+                               (tile == 0 ? kFlagP : kFlagA) | (unsigned long long)run);
     }
     __syncthreads();
     // tile-local start of each output bucket (the mode's buckets, in order)
@@ -505,7 +510,7 @@ __global__ void __launch_bounds__(kRankThreads, 1)
                 for (int u = 0; u < 2; ++u) {
                     // a word not yet published: bounded wait
                     while ((v[q][u] >> 62) == 0ull) {
-                        if (++polls > kPollLimit) {
+                        if (++polls > ws.poll_limit) {
                             md::report(status, MD_ERR_TIMEOUT);
                             s_timeout = 1;
                             v[q][u] = kFlagP;
@@ -535,7 +540,7 @@ __global__ void __launch_bounds__(kRankThreads, 1)
         for (int q = 0; q < kLookBatch; ++q) {
             const int b = b0 + q * kRankWarps;
             if (b < NB && lane == 0) {
-                if (tile > 0)
+                if (tile > 0 && tile != ws.skip_tile)
                     md::st_relaxed_u64(ws.tiles + (size_t)b * n_tiles + tile,
                                        kFlagP | (unsigned long long)(excl[q] + s_pref[b]));
                 s_pref[b] = s_base[b] + excl[q];
@@ -658,16 +663,15 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
     cudaStream_t s = md::as_stream(stream);
     const Ws ws = carve(workspace, pl);
 
-    static bool attr_set = false;
-    if (!attr_set) {
+    static std::atomic<uint64_t> attr_done{0};
+    md::once_per_device(attr_done, [] {
         set_attrs<0>();
         set_attrs<1>();
         set_attrs<2>();
         set_attrs<4>();
         set_attrs<6>();
         set_attrs<8>();
-        attr_set = true;
-    }
+    });
     {
         const size_t n16 = pl.total / 16;
         int zb = (int)((n16 + 255) / 256);

@@ -35,13 +35,17 @@ namespace {
 
 constexpr int kTile = 1024;  // items per bucket-sort tile
 
+// bytes per token preference list in the pair form: a multiple of 16, so that
+// a list moves by 16-byte async copies
+inline __host__ __device__ int pref_stride(int R) { return (R + 15) / 16 * 16; }
+
 struct ShufWs {
     int32_t *pref;                 // [E*R]
     unsigned long long *num, *den; // [E]
     int32_t *cls;                  // [E]
     int32_t *order;                // [T]
     int32_t *keys;                 // [T] bucket of each token in the current sort
-    int32_t *tile_hist;            // [n_tiles * max(E+1, R)]
+    int32_t *tile_hist;            // [(n_tiles + 1) * max(E+1, R)]
 };
 
 size_t shuf_layout(int64_t T, int E, int R, ShufWs *w, void *base)
@@ -62,7 +66,7 @@ size_t shuf_layout(int64_t T, int E, int R, ShufWs *w, void *base)
     x.order = reinterpret_cast<int32_t *>(take((size_t)(T > 0 ? T : 1) * 4));
     x.keys = reinterpret_cast<int32_t *>(take((size_t)(T > 0 ? T : 1) * 4));
     const int nbk = E + 1 > R ? E + 1 : R;
-    x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)(n_tiles > 0 ? n_tiles : 1) * nbk * 4));
+    x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)((n_tiles > 0 ? n_tiles : 1) + 1) * nbk * 4));
     if (w) *w = x;
     return o;
 }
@@ -185,54 +189,64 @@ __global__ void __launch_bounds__(256)
     for (int b = threadIdx.x; b < nbk; b += 256) tile_hist[(int64_t)blockIdx.x * nbk + b] = h[b];
 }
 
-// tile_hist[tile][b] <- first output position of bucket b's items in tile.
-// A warp scans one bucket's column over the tiles; then the bucket totals are
-// scanned and added.
-__global__ void __launch_bounds__(1024)
+// tile_hist[tile][b] <- items of bucket b in the tiles before `tile` (column
+// scan), and row n_tiles <- the first output position of bucket b (scan of
+// the bucket totals); a scatter starts bucket b of a tile at the sum of the
+// two.  One thread per bucket walks its column with 8 loads in flight
+// (adjacent threads read adjacent buckets, so each tile row is coalesced).
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads)
     k_bucket_scan(int32_t *__restrict__ tile_hist, int n_tiles, int nbk)
 {
     extern __shared__ int tot[];
-    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
-    for (int b = wp; b < nbk; b += 32) {
+    __shared__ int s_warp[kScanThreads / 32];
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    for (int b = tid; b < nbk; b += kScanThreads) {
         int run = 0;
-        for (int i0 = 0; i0 < n_tiles; i0 += 32) {
-            const int i = i0 + lane;
-            const int v = i < n_tiles ? tile_hist[(int64_t)i * nbk + b] : 0;
-            int incl = v;
+        for (int i0 = 0; i0 < n_tiles; i0 += 8) {
+            int v[8];
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            if (i < n_tiles) tile_hist[(int64_t)i * nbk + b] = run + incl - v;
-            run += __shfl_sync(0xffffffffu, incl, 31);
+            for (int u = 0; u < 8; ++u)
+                v[u] = i0 + u < n_tiles ? tile_hist[(int64_t)(i0 + u) * nbk + b] : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (i0 + u < n_tiles) {
+                    tile_hist[(int64_t)(i0 + u) * nbk + b] = run;
+                    run += v[u];
+                }
         }
-        if (lane == 0) tot[b] = run;
+        tot[b] = run;
     }
+    __syncthreads();
+    // exclusive scan of the bucket totals: thread i takes a contiguous run
+    const int per = (nbk + kScanThreads - 1) / kScanThreads;
+    const int lo = tid * per, hi = min(nbk, lo + per);
+    int sum = 0;
+    for (int b = lo; b < hi; ++b) sum += tot[b];
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_warp[wp] = incl;
     __syncthreads();
     if (wp == 0) {
-        // exclusive scan of the bucket totals: lane L takes a contiguous run
-        const int per = (nbk + 31) / 32;
-        const int lo = lane * per, hi = min(nbk, lo + per);
-        int sum = 0;
-        for (int b = lo; b < hi; ++b) sum += tot[b];
-        int incl = sum;
+        int w = s_warp[lane], wi = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
+            const int y = __shfl_up_sync(0xffffffffu, wi, o);
+            if (lane >= o) wi += y;
         }
-        int run = incl - sum;
-        for (int b = lo; b < hi; ++b) {
-            const int v = tot[b];
-            tot[b] = run;
-            run += v;
-        }
+        s_warp[lane] = wi - w;
     }
     __syncthreads();
-    for (int b = wp; b < nbk; b += 32) {
-        const int base = tot[b];
-        for (int i = lane; i < n_tiles; i += 32) tile_hist[(int64_t)i * nbk + b] += base;
+    int run = s_warp[wp] + incl - sum;
+    int32_t *base = tile_hist + (int64_t)n_tiles * nbk;
+    for (int b = lo; b < hi; ++b) {
+        base[b] = run;
+        run += tot[b];
     }
 }
 
@@ -245,7 +259,8 @@ __global__ void __launch_bounds__(32)
 {
     extern __shared__ int cnt[];
     const int lane = threadIdx.x;
-    for (int b = lane; b < nbk; b += 32) cnt[b] = tile_hist[(int64_t)blockIdx.x * nbk + b];
+    const int32_t *base = tile_hist + (int64_t)gridDim.x * nbk;
+    for (int b = lane; b < nbk; b += 32) cnt[b] = tile_hist[(int64_t)blockIdx.x * nbk + b] + base[b];
     const int64_t t0 = (int64_t)blockIdx.x * kTile;
     int kv[kTile / 32];
 #pragma unroll
@@ -291,8 +306,10 @@ constexpr int kGreedyThreads = 1024;
 constexpr int kGreedyWarps = kGreedyThreads / 32;
 
 // PAIR: the prediction row differs per token, so instead of first[e] each
-// token walks its own preference list (tpref[t*R ..], R bytes), and an empty
-// row is marked by a zero confidence key.
+// token walks its own preference list, and an empty row is marked by a zero
+// confidence key.  A thread's list is staged in shared memory by 16-byte
+// async copies one chunk ahead (two buffers), so walks after a fill event
+// read shared memory only.
 template <bool PAIR>
 __global__ void __launch_bounds__(kGreedyThreads, 1)
     k_shuf_greedy(const int32_t *__restrict__ order, const int32_t *__restrict__ idx_l, int k,
@@ -333,6 +350,20 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
         const int64_t pos = base + tid;
         return pos < T ? (int64_t)order[pos] : -1;
     };
+    // pair: per-thread list slots, two chunk buffers
+    const int Rs = pref_stride(R);
+    unsigned char *s_lists = g_raw;
+    auto stage_list = [&](int64_t t, int buf) {
+        if (PAIR && t >= 0) {
+            unsigned char *dst = s_lists + ((size_t)buf * kGreedyThreads + tid) * Rs;
+            const unsigned char *src = tpref + t * Rs;
+            for (int o = 0; o < Rs; o += 16)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(md::smem_addr(dst + o)),
+                             "l"(src + o)
+                             : "memory");
+        }
+        if (PAIR) asm volatile("cp.async.commit_group;" ::: "memory");
+    };
     // single: the top-1 expert; pair: 1 when the token's prediction row is empty
     auto key_of = [&](int64_t t) -> int {
         if (t < 0) return 0;
@@ -341,14 +372,20 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
     };
     int64_t t_n1 = token_at(0);
     int e_n1 = key_of(t_n1);
+    stage_list(t_n1, 0);
     int64_t t_n2 = token_at(kGreedyThreads);
 
-    for (int64_t base = 0; base < T; base += kGreedyThreads) {
+    int chunk = 0;
+    for (int64_t base = 0; base < T; base += kGreedyThreads, ++chunk) {
         const int64_t t = t_n1;
         int e1 = e_n1;
         t_n1 = t_n2;
         e_n1 = key_of(t_n1);
+        stage_list(t_n1, (chunk + 1) & 1);
         t_n2 = token_at(base + 2 * kGreedyThreads);
+        // this chunk's list copies are done (the next chunk's may be pending)
+        if (PAIR) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        const unsigned char *my_list = s_lists + ((size_t)(chunk & 1) * kGreedyThreads + tid) * Rs;
         const bool have = t >= 0;
         if (!PAIR && have && (e1 < 0 || e1 >= E)) {
             md::report(status, MD_ERR_DATA);
@@ -364,7 +401,7 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
                 if (PAIR) {
                     f = -1;
                     if (!e1) {
-                        const unsigned char *pl = tpref + t * R;
+                        const unsigned char *pl = my_list;
                         const unsigned long long full = s_full;
                         int n = 0;
                         while (n < R && ((full >> pl[n]) & 1ull)) ++n;
@@ -502,11 +539,11 @@ constexpr int kRadixPasses = (64 + kRadixBits - 1) / kRadixBits;
 constexpr int kPairWarps = 8;
 
 struct PairWs {
-    unsigned char *tpref;      // [T*R] preference list of each token
+    unsigned char *tpref;      // [T*Rs] preference list of each token, Rs = R rounded up to 16
     unsigned long long *conf;  // [T]   confidence key of each token
     int32_t *seq_a, *seq_b;    // [T]   radix sort ping-pong
     int32_t *keys;             // [T]   bucket of each token in the final partition
-    int32_t *tile_hist;        // [n_tiles * max(2^11, R)]
+    int32_t *tile_hist;        // [(n_tiles + 1) * max(2^11, R)]
 };
 
 size_t pair_layout(int64_t T, int R, PairWs *w, void *base)
@@ -521,13 +558,13 @@ size_t pair_layout(int64_t T, int R, PairWs *w, void *base)
     const int64_t Tn = T > 0 ? T : 1;
     const int64_t n_tiles = (Tn + kTile - 1) / kTile;
     PairWs x;
-    x.tpref = reinterpret_cast<unsigned char *>(take((size_t)Tn * R));
+    x.tpref = reinterpret_cast<unsigned char *>(take((size_t)Tn * pref_stride(R)));
     x.conf = reinterpret_cast<unsigned long long *>(take((size_t)Tn * 8));
     x.seq_a = reinterpret_cast<int32_t *>(take((size_t)Tn * 4));
     x.seq_b = reinterpret_cast<int32_t *>(take((size_t)Tn * 4));
     x.keys = reinterpret_cast<int32_t *>(take((size_t)Tn * 4));
     const int nbk = kRadixBuckets > R ? kRadixBuckets : R;
-    x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)n_tiles * nbk * 4));
+    x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)(n_tiles + 1) * nbk * 4));
     if (w) *w = x;
     return o;
 }
@@ -539,8 +576,28 @@ __global__ void __launch_bounds__(kPairWarps * 32)
                 PairWs ws, int32_t *__restrict__ use_pair, int32_t *status)
 {
     __shared__ unsigned long long s_sig[kPairWarps][MD_MAX_RANKS];
+    __shared__ int s_rmem[MD_MAX_PAIR_EXPERTS];   // experts grouped by next-layer rank
+    __shared__ int s_rstart[MD_MAX_RANKS + 1];
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     unsigned long long *sig = s_sig[wl];
+    if (threadIdx.x == 0) {
+        // counting sort of the experts by rank; an out-of-range rank is
+        // reported and the expert left out of every rank's sum
+        for (int d = 0; d <= R; ++d) s_rstart[d] = 0;
+        for (int e = 0; e < E; ++e) {
+            const int d = p_next[e];
+            if (d >= 0 && d < R) ++s_rstart[d + 1];
+            else md::report(status, MD_ERR_DATA);
+        }
+        for (int d = 0; d < R; ++d) s_rstart[d + 1] += s_rstart[d];
+        int fill[MD_MAX_RANKS];
+        for (int d = 0; d < R; ++d) fill[d] = s_rstart[d];
+        for (int e = 0; e < E; ++e) {
+            const int d = p_next[e];
+            if (d >= 0 && d < R) s_rmem[fill[d]++] = e;
+        }
+    }
+    __syncthreads();
     const int64_t w0 = (int64_t)blockIdx.x * kPairWarps + wl;
     const int64_t nw = (int64_t)gridDim.x * kPairWarps;
     for (int64_t t = w0; t < T; t += nw) {
@@ -557,9 +614,13 @@ __global__ void __launch_bounds__(kPairWarps * 32)
         for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
         const bool use = psum >= min_obs;
         const uint32_t *row = use ? prow : C + (int64_t)b * E;
-        for (int d = lane; d < R; d += 32) sig[d] = 0ull;
-        __syncwarp();
-        // total, arg-max (lowest index on ties) and per-rank sums
+        // per-rank sums: lane d adds its rank's experts
+        for (int d = lane; d < R; d += 32) {
+            unsigned long long sd = 0;
+            for (int i = s_rstart[d]; i < s_rstart[d + 1]; ++i) sd += __ldg(row + s_rmem[i]);
+            sig[d] = sd;
+        }
+        // total and arg-max (lowest index on ties)
         unsigned long long tot = 0;
         uint32_t bv = 0;
         int be = INT_MAX;
@@ -570,9 +631,6 @@ __global__ void __launch_bounds__(kPairWarps * 32)
                 bv = v;
                 be = e;
             }
-            const int d = __ldg(p_next + e);
-            if (d < 0 || d >= R) md::report(status, MD_ERR_DATA);
-            else if (v) atomicAdd(&sig[d], (unsigned long long)v);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -587,7 +645,7 @@ __global__ void __launch_bounds__(kPairWarps * 32)
         __syncwarp();
         int first = __ldg(p_next + be);
         if (first < 0 || first >= R) first = 0;
-        unsigned char *pl = ws.tpref + t * R;
+        unsigned char *pl = ws.tpref + t * pref_stride(R);
         for (int d = lane; d < R; d += 32) {
             int pos = 0;
             if (d != first) {
@@ -642,8 +700,9 @@ __global__ void __launch_bounds__(32)
 {
     __shared__ int cnt[kRadixBuckets];
     const int lane = threadIdx.x;
+    const int32_t *base = tile_hist + (int64_t)gridDim.x * kRadixBuckets;
     for (int b = lane; b < kRadixBuckets; b += 32)
-        cnt[b] = tile_hist[(int64_t)blockIdx.x * kRadixBuckets + b];
+        cnt[b] = tile_hist[(int64_t)blockIdx.x * kRadixBuckets + b] + base[b];
     const int64_t t0 = (int64_t)blockIdx.x * kTile;
     int tok[kTile / 32], dg[kTile / 32];
 #pragma unroll
@@ -703,7 +762,7 @@ extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
     const int nbk0 = E + 1;
     k_bucket_hist<<<n_tiles, 256, nbk0 * sizeof(int), s>>>(0, T, idx_l, k, ws.cls, E, nullptr, nbk0,
                                                           ws.keys, ws.tile_hist);
-    k_bucket_scan<<<1, 1024, nbk0 * sizeof(int), s>>>(ws.tile_hist, n_tiles, nbk0);
+    k_bucket_scan<<<1, kScanThreads, nbk0 * sizeof(int), s>>>(ws.tile_hist, n_tiles, nbk0);
     k_bucket_scatter<<<n_tiles, 32, nbk0 * sizeof(int), s>>>(0, T, nbk0, ws.keys, ws.tile_hist,
                                                             ws.order, nullptr, nullptr);
     const size_t gsm = (size_t)E * sizeof(int) + (size_t)E * R;
@@ -715,7 +774,7 @@ extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
     // new positions: stable partition by assigned rank
     k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
                                                        ws.keys, ws.tile_hist);
-    k_bucket_scan<<<1, 1024, R * sizeof(int), s>>>(ws.tile_hist, n_tiles, R);
+    k_bucket_scan<<<1, kScanThreads, R * sizeof(int), s>>>(ws.tile_hist, n_tiles, R);
     k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, R, ws.keys, ws.tile_hist, nullptr,
                                                          perm, inv);
     md::count_launches(9);
@@ -764,19 +823,23 @@ extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx
     for (int pass = 0; pass < kRadixPasses; ++pass) {
         const int shift = pass * kRadixBits;
         k_radix_hist<<<n_tiles, 256, 0, s>>>(in, pw.conf, T, shift, pw.tile_hist);
-        k_bucket_scan<<<1, 1024, kRadixBuckets * sizeof(int), s>>>(pw.tile_hist, n_tiles,
+        k_bucket_scan<<<1, kScanThreads, kRadixBuckets * sizeof(int), s>>>(pw.tile_hist, n_tiles,
                                                                   kRadixBuckets);
         k_radix_scatter<<<n_tiles, 32, 0, s>>>(in, pw.conf, T, shift, pw.tile_hist, out);
         in = out;
         out = out == pw.seq_a ? pw.seq_b : pw.seq_a;
     }
     ShufWs none{};
-    k_shuf_greedy<true><<<1, kGreedyThreads, 0, s>>>(in, nullptr, k, none, pw.tpref, pw.conf, T, E,
-                                                     R, Tr, pred_rank, dev_status);
+    const size_t lsm = (size_t)2 * kGreedyThreads * pref_stride(R);
+    if (cudaFuncSetAttribute(k_shuf_greedy<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)lsm) != cudaSuccess)
+        return MD_ERR_CUDA;
+    k_shuf_greedy<true><<<1, kGreedyThreads, lsm, s>>>(in, nullptr, k, none, pw.tpref, pw.conf, T, E,
+                                                       R, Tr, pred_rank, dev_status);
     // new positions: stable partition by assigned rank
     k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
                                                        pw.keys, pw.tile_hist);
-    k_bucket_scan<<<1, 1024, R * sizeof(int), s>>>(pw.tile_hist, n_tiles, R);
+    k_bucket_scan<<<1, kScanThreads, R * sizeof(int), s>>>(pw.tile_hist, n_tiles, R);
     k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, R, pw.keys, pw.tile_hist, nullptr,
                                                          perm, inv);
     md::count_launches(1 + 3 * kRadixPasses + 1 + 3);

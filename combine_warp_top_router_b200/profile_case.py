@@ -4,7 +4,8 @@ profiling a single kernel under ncu on a small case.
     python -m combine_warp_top_router_b200.profile_case --steps layout,permute \
         --workload zipf_pairs_e128_k8 --T 16384 --reps 3
 
-Steps: topk, layout, permute, combine, wire, coselect, place, shuffle, gather.
+Steps: topk, layout, permute, combine, wire, expand, coselect, place, shuffle,
+shuffle_pair (three_layer_e128_k6 only), gather.
 Every listed step runs once as warm-up and then `reps` times.
 """
 from __future__ import annotations
@@ -29,7 +30,7 @@ def main():
     a = ap.parse_args()
     steps = a.steps.split(",")
     dev = torch.device("cuda", 0)
-    rows = any(s in steps for s in ("permute", "combine", "wire", "gather"))
+    rows = any(s in steps for s in ("permute", "combine", "wire", "expand", "gather"))
     w = synth.make_workload(a.workload, device=dev, T=a.T, H=a.H, R=a.R, with_rows=rows)
     mode = md.MD_DEDUP if a.mode == "dedup" else md.MD_CONV
     T, E, k, R = w.T, w.E, w.k, w.R
@@ -42,6 +43,12 @@ def main():
     buf = torch.empty(L.row_capacity, w.H, dtype=torch.bfloat16, device=dev) if rows else None
     out = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev) if rows else None
     z = torch.empty(L.row_capacity, w.H, dtype=torch.bfloat16, device=dev) if "wire" in steps else None
+    xc = torch.empty(T * k, w.H, dtype=torch.bfloat16, device=dev) if "expand" in steps else None
+    if "shuffle_pair" in steps:
+        if w.logits_prev is None:
+            raise SystemExit("shuffle_pair needs a three-layer workload")
+        idx0, _ = md.md_route_topk(w.logits_prev, k)
+        C2 = md.md_coselect_pair_stats(idx0, idx, idx2, E, T_fit=w.fit_tokens or T)
     torch.cuda.synchronize()
 
     def once():
@@ -57,6 +64,10 @@ def main():
             elif s == "wire":
                 md.md_combine(w.y, L.assign_row, idx, gates, md.MD_COMBINE_WIRE,
                               row_of_slot=L.row_of_slot, z=z, out=out)
+            elif s == "expand":
+                md.md_dedup_expand(buf, L.row_of_slot, L.assign_row, out=xc)
+            elif s == "shuffle_pair":
+                md.md_token_shuffle_pair(idx0, idx, C, C2, w.expert_to_rank, R, 8 * k)
             elif s == "coselect":
                 md.md_coselect_stats(idx, idx2, E, T_fit=w.fit_tokens or T, W=W, C=C)
             elif s == "place":

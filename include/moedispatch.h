@@ -419,6 +419,18 @@ int md_successor_share(const uint32_t *C, const uint32_t *W, int E, uint32_t *nu
 
 int md_count_sums(const uint32_t *x, const uint32_t *y, int64_t n, uint64_t *sums, void *stream);
 
+/*
+ * md_set_test_hooks -- fault injection for tests; not for production use.
+ * Every bounded device-side wait gives up after a poll limit and reports
+ * MD_ERR_TIMEOUT.  These hooks make such a wait run out on purpose, with no
+ * fault: poll_limit > 0 replaces the default limits; layout_skip_tile >= 0
+ * makes that md_dispatch_layout tile publish no lookback word, so the tiles
+ * after it wait in vain; expand_skip_unit >= 0 makes md_dedup_expand (bulk-copy
+ * path) never fill that unit's shared-memory slot.  (0, -1, -1) restores the
+ * defaults.  Process-wide; set them only while no other call is in flight.
+ */
+void md_set_test_hooks(long long poll_limit, int layout_skip_tile, long long expand_skip_unit);
+
 #ifdef __cplusplus
 }
 #endif
