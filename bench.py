@@ -596,10 +596,50 @@ def cpu_baseline(args):
         if time.perf_counter() - t0 >= args.cpu_seconds:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(T_s * reps / dt / 1e6, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{reps} x {T_s}-token sample of the same workload recipe "
-                      f"(E=128, top-8, 16 ranks, H=2048), single-threaded C oracle, "
-                      f"{dt:.1f} s", "host_cores": os.cpu_count()}
+    out = {"value": round(T_s * reps / dt / 1e6, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{reps} x {T_s}-token sample of the same workload recipe "
+                     f"(E=128, top-8, 16 ranks, H=2048), single-threaded C oracle, "
+                     f"{dt:.1f} s", "host_cores": os.cpu_count()}
+    if args.rows:
+        out["rows"] = cpu_rows(oracle, args.seed)
+    return out
+
+
+def cpu_rows(oracle, seed):
+    """The oracle timed on the planner rows' workloads (single core, one run
+    each), beside the GPU times of the `rows` object."""
+    from combine_warp_top_router_b200 import synth
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        r = fn()
+        return r, round((time.perf_counter() - t0) * 1e3, 1)
+
+    res = {}
+    w = synth.make_workload("two_layer_e128_k6", seed=seed, with_rows=False)
+    a = oracle.route_topk(w.logits.numpy(), w.k)[0]
+    b = oracle.route_topk(w.logits_next.numpy(), w.k)[0]
+    _, C = oracle.coselect(a, b, w.E, T_fit=w.fit_tokens)
+    _, res["token_shuffle_e128_k6_ms"] = timed(
+        lambda: oracle.token_shuffle(a, C, w.expert_to_rank.numpy(), w.R))
+    w = synth.make_workload("three_layer_e128_k6", seed=seed, with_rows=False)
+    g = [oracle.route_topk(lg.numpy(), w.k)[0] for lg in (w.logits_prev, w.logits, w.logits_next)]
+    C2, res["pair_counts_ms"] = timed(lambda: oracle.coselect_pair(g[0], g[1], g[2], w.E,
+                                                                   T_fit=w.fit_tokens))
+    _, C = oracle.coselect(g[1], g[2], w.E, T_fit=w.fit_tokens)
+    _, res["token_shuffle_pair_e128_k6_ms"] = timed(
+        lambda: oracle.token_shuffle_pair(g[0], g[1], C, C2, w.expert_to_rank.numpy(), w.R, 8 * w.k))
+    w = synth.make_workload("full_e256_k8", seed=seed, with_rows=False)
+    a, res["route_topk_e256_k8_T262144_ms"] = timed(lambda: oracle.route_topk(w.logits.numpy(), 8)[0])
+    (W, _), res["coselect_W_e256_ms"] = timed(lambda: oracle.coselect(a, None, 256))
+    for label, refine in (("swaps", oracle.REFINE_SWAPS), ("kl", oracle.REFINE_KL)):
+        _, res[f"place_{label}_e256_r64_ms"] = timed(
+            lambda: oracle.place_two_level(W, 64, 1, 0, refine))
+    _, res["place_kl_8_nodes_e256_r64_ms"] = timed(
+        lambda: oracle.place_two_level(W, 64, 8, 0, oracle.REFINE_KL))
+    _, res["layout_dedup_e256_T262144_ms"] = timed(
+        lambda: oracle.dispatch_layout(a, 256, 64, w.expert_to_rank.numpy(), 1))
+    return res
 
 
 def run_reference(args):

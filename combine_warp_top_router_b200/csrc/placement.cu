@@ -32,6 +32,11 @@
 //   compares its candidate with the pairs it forms with the 2 E/R experts of
 //   P and Q.  A lives in shared memory when it fits, rows padded to R + 1
 //   entries so that lanes reading consecutive rows hit different banks.
+// For E <= 256, when W is symmetric with entries below 2^16 (co-selection
+// counts fitted on fewer than 65536 tokens, or sparse enough), W is copied
+// into shared memory as uint16 and A kept as int32 beside it, so that no
+// step waits on L2; otherwise W is read from global memory.  The choice is
+// made on the device from the data, per problem.
 #include <climits>
 
 #include "common.cuh"
@@ -41,6 +46,7 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr size_t kSmemA = 160 * 1024;  // largest A kept in shared memory
+constexpr int kCompactMaxE = 256;      // largest E whose W (uint16) fits beside A
 
 struct Cand {
     long long g;
@@ -89,8 +95,56 @@ struct Smem {
     unsigned char *lock;  // [E] KL: moved in this pass
     int *ka, *kb, *kP, *kQ;  // [E/2] KL: the moves of this pass
     long long *kg;        // [E/2] KL: their gains
-    long long *A;   // [E][ar]: A[e][d] at A[e * ar + d]
-    int ar;         // row stride of A: R + 1, so that consecutive rows fall in different banks
+};
+
+// Where W and A live.
+//   Store<false>: W (uint32) in global memory, read through L1/L2; A (int64)
+//     in shared memory when it fits, else in the workspace.
+//   Store<true>, when W is symmetric with entries below 2^16 and row sums
+//     below 2^31 (E <= 256): W as uint16 and A as int32, both in shared
+//     memory.  Symmetry lets column reads use rows, so threads on
+//     consecutive experts read consecutive halfwords.
+// A[e][d] sits at A[e * ar + d] with ar = R + 1, so that consecutive rows
+// fall in different banks.
+template <bool COMPACT>
+struct Store;
+
+template <>
+struct Store<false> {
+    const uint32_t *W;
+    long long *A;
+    int E, ar;
+    __device__ __forceinline__ uint32_t w_row(int a, int b) const  // threads vary b
+    {
+        return __ldg(W + (int64_t)a * E + b);
+    }
+    __device__ __forceinline__ uint32_t w_col(int a, int b) const  // threads vary a
+    {
+        return __ldg(W + (int64_t)a * E + b);
+    }
+    __device__ __forceinline__ long long a_get(int e, int d) const { return A[(int64_t)e * ar + d]; }
+    __device__ __forceinline__ void a_add(int e, int d, long long v) const { A[(int64_t)e * ar + d] += v; }
+    __device__ __forceinline__ void a_atomic_add(int e, int d, uint32_t v) const
+    {
+        atomicAdd(reinterpret_cast<unsigned long long *>(A + (int64_t)e * ar + d), (unsigned long long)v);
+    }
+    __device__ __forceinline__ void a_zero(int64_t i) const { A[i] = 0; }
+};
+
+template <>
+struct Store<true> {
+    const uint16_t *W;
+    int *A;
+    int E, ar;
+    __device__ __forceinline__ uint32_t w_row(int a, int b) const { return W[a * E + b]; }
+    __device__ __forceinline__ uint32_t w_col(int a, int b) const { return W[b * E + a]; }
+    __device__ __forceinline__ long long a_get(int e, int d) const { return A[e * ar + d]; }
+    __device__ __forceinline__ void a_add(int e, int d, long long v) const { A[e * ar + d] += (int)v; }
+    __device__ __forceinline__ void a_atomic_add(int e, int d, uint32_t v) const
+    {
+        atomicAdd(A + e * ar + d, (int)v);
+    }
+    __device__ __forceinline__ void a_zero(int64_t i) const { A[i] = 0; }
 };
 
 // ------------------------------------------------------------ greedy seed
@@ -108,19 +162,19 @@ __device__ __forceinline__ bool eligible(const Smem &s, int a, int b, int cap, i
 // b = -1 when none.
 constexpr int kBatch = 4;
 
-__device__ __forceinline__ void greedy_row(const uint32_t *__restrict__ W, const Smem &s, int E,
-                                           int a, int cap, int maxfree, uint32_t &w_out, int &b_out)
+template <class St>
+__device__ __forceinline__ void greedy_row(const St &st, const Smem &s, int E, int a, int cap,
+                                           int maxfree, uint32_t &w_out, int &b_out)
 {
     const int lane = threadIdx.x & 31;
     uint32_t bw = 0;
     int bb = INT_MAX;
-    const uint32_t *row = W + (int64_t)a * E;
     for (int b0 = a + 1; b0 < E; b0 += 32 * kBatch) {
         uint32_t wv[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int b = b0 + u * 32 + lane;
-            wv[u] = b < E ? __ldg(row + b) : 0u;
+            wv[u] = b < E ? st.w_row(a, b) : 0u;
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
@@ -139,23 +193,22 @@ __device__ __forceinline__ void greedy_row(const uint32_t *__restrict__ W, const
 }
 
 // ------------------------------------------------------------- refinement
-__device__ __forceinline__ long long gain_w(const Smem &s, int R, int a, int b, uint32_t wab)
+template <class St>
+__device__ __forceinline__ long long gain_w(const St &st, const Smem &s, int a, int b, uint32_t wab)
 {
     const int P = s.p[a], Q = s.p[b];
-    const long long *Aa = s.A + (int64_t)a * s.ar, *Ab = s.A + (int64_t)b * s.ar;
-    return Aa[Q] - Aa[P] + Ab[P] - Ab[Q] - 2ll * (long long)wab;
+    return st.a_get(a, Q) - st.a_get(a, P) + st.a_get(b, P) - st.a_get(b, Q) - 2ll * (long long)wab;
 }
 
 // Best partner b > a (p[b] != p[a]) of row a, lowest b on ties: with a
 // positive gain for the swap search; any gain, among unlocked experts, in a
 // Kernighan-Lin pass (KL).  b = -1 when there is none.
-template <bool KL>
-__device__ __forceinline__ void refine_row(const uint32_t *__restrict__ W, const Smem &s, int E,
-                                           int R, int a, long long &g_out, int &b_out)
+template <bool KL, class St>
+__device__ __forceinline__ void refine_row(const St &st, const Smem &s, int E, int a,
+                                           long long &g_out, int &b_out)
 {
     const int lane = threadIdx.x & 31;
     const int P = s.p[a];
-    const uint32_t *row = W + (int64_t)a * E;
     long long bg = 0;
     int bb = -1;
     for (int b0 = a + 1; b0 < E; b0 += 32 * kBatch) {
@@ -163,13 +216,13 @@ __device__ __forceinline__ void refine_row(const uint32_t *__restrict__ W, const
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int b = b0 + u * 32 + lane;
-            wv[u] = b < E ? __ldg(row + b) : 0u;
+            wv[u] = b < E ? st.w_row(a, b) : 0u;
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int b = b0 + u * 32 + lane;
             if (b >= E || s.p[b] == P || (KL && s.lock[b])) continue;
-            const long long g = gain_w(s, R, a, b, wv[u]);
+            const long long g = gain_w(st, s, a, b, wv[u]);
             if (KL ? (bb < 0 || g > bg) : g > bg) {
                 bg = g;
                 bb = b;
@@ -191,14 +244,15 @@ __device__ __forceinline__ void refine_row(const uint32_t *__restrict__ W, const
 
 // Move a (rank P) to Q and b (rank Q) to P: columns P and Q of A, and (thread
 // 0) the rank lists.  The caller synchronises.
-__device__ __forceinline__ void apply_swap(const uint32_t *__restrict__ W, const Smem &s, int E,
-                                           int cap, int a, int b, int P, int Q)
+template <class St>
+__device__ __forceinline__ void apply_swap(const St &st, const Smem &s, int E, int cap, int a,
+                                           int b, int P, int Q)
 {
     for (int e = threadIdx.x; e < E; e += kThreads) {
-        const long long wa = e != a ? (long long)__ldg(W + (int64_t)e * E + a) : 0;
-        const long long wb = e != b ? (long long)__ldg(W + (int64_t)e * E + b) : 0;
-        s.A[(int64_t)e * s.ar + P] += wb - wa;
-        s.A[(int64_t)e * s.ar + Q] += wa - wb;
+        const long long wa = e != a ? (long long)st.w_col(e, a) : 0;
+        const long long wb = e != b ? (long long)st.w_col(e, b) : 0;
+        st.a_add(e, P, wb - wa);
+        st.a_add(e, Q, wa - wb);
     }
     if (threadIdx.x == 0) {
         const int sa = s.slot[a], sb = s.slot[b];
@@ -216,9 +270,9 @@ __device__ __forceinline__ void apply_swap(const uint32_t *__restrict__ W, const
 // among experts not yet moved in the pass, whatever its sign; the pass keeps
 // the shortest prefix of moves with the largest positive total and undoes
 // the rest; passes repeat while that total is positive (at most E passes).
-template <bool KL>
-__device__ void search(const uint32_t *__restrict__ W, const Smem &s, int E, int R, int cap,
-                       Cand *s_red, int *s_nlist, long long *s_keep, int *s_keep_m)
+template <bool KL, class St>
+__device__ void search(const St &st, const Smem &s, int E, int R, int cap, Cand *s_red, int *s_nlist,
+                       long long *s_keep, int *s_keep_m)
 {
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     const long long max_passes = KL ? E : 1;
@@ -250,7 +304,6 @@ __device__ void search(const uint32_t *__restrict__ W, const Smem &s, int E, int
                     s.list[atomicAdd(s_nlist, 1)] = a;
                     continue;
                 }
-                const uint32_t *row = W + (int64_t)a * E;
                 for (int i0 = 0; i0 < 2 * cap; i0 += kBatch) {
                     int bv[kBatch];
                     uint32_t wv[kBatch];
@@ -259,13 +312,13 @@ __device__ void search(const uint32_t *__restrict__ W, const Smem &s, int E, int
                         const int i = i0 + u;
                         bv[u] = i < 2 * cap ? s.mem[(i < cap ? lastP * cap + i : lastQ * cap + i - cap)]
                                             : -1;
-                        wv[u] = bv[u] > a ? __ldg(row + bv[u]) : 0u;
+                        wv[u] = bv[u] > a ? st.w_col(a, bv[u]) : 0u;
                     }
 #pragma unroll
                     for (int u = 0; u < kBatch; ++u) {
                         const int b = bv[u];
                         if (b <= a || (KL && s.lock[b])) continue;
-                        const long long g = gain_w(s, R, a, b, wv[u]);
+                        const long long g = gain_w(st, s, a, b, wv[u]);
                         if ((KL || g > 0) && (cb < 0 || g > cg || (g == cg && b < cb))) {
                             cg = g;
                             cb = b;
@@ -282,7 +335,7 @@ __device__ void search(const uint32_t *__restrict__ W, const Smem &s, int E, int
                 const int a = s.list[i];
                 long long g2;
                 int b2;
-                refine_row<KL>(W, s, E, R, a, g2, b2);
+                refine_row<KL>(st, s, E, a, g2, b2);
                 if (lane == 0) {
                     s.cg[a] = g2;
                     s.cb[a] = b2;
@@ -301,7 +354,7 @@ __device__ void search(const uint32_t *__restrict__ W, const Smem &s, int E, int
             __syncthreads();
             const Cand win = warp_best(s_red[lane]);
             if (win.a < 0) break;  // uniform: every thread holds the same winner
-            apply_swap(W, s, E, cap, win.a, win.b, win.P, win.Q);
+            apply_swap(st, s, E, cap, win.a, win.b, win.P, win.Q);
             if (tid == 0) {
                 *s_nlist = 0;
                 if (KL) {
@@ -339,56 +392,21 @@ __device__ void search(const uint32_t *__restrict__ W, const Smem &s, int E, int
         const long long keep = *s_keep;
         for (int i = moves - 1; i >= m; --i) {
             // move i took a from P to Q and b from Q to P; take them back
-            apply_swap(W, s, E, cap, s.ka[i], s.kb[i], s.kQ[i], s.kP[i]);
+            apply_swap(st, s, E, cap, s.ka[i], s.kb[i], s.kQ[i], s.kP[i]);
             __syncthreads();
         }
         if (keep <= 0) break;
     }
 }
 
-// One CTA per independent problem (blockIdx.x): W, p_out and A_global point
-// at problem 0 and advance by E*E, E and E*(R+1).  refine: 0 none, 1 best
-// single swaps, 2 Kernighan-Lin passes.
-__global__ void __launch_bounds__(kThreads, 1)
-    k_place(const uint32_t *__restrict__ W, int E, int R, int seed_mode, int refine,
-            int32_t *__restrict__ p_out, long long *__restrict__ A_global, int a_in_smem)
+// Seed and refinement of one problem, with W and A where `st` says.
+template <class St>
+__device__ void place_body(const St &st, const Smem &s, int E, int R, int seed_mode, int refine,
+                           Cand *s_red, int *s_maxfree, int *s_roomiest, int *s_nlist,
+                           long long *s_keep, int *s_keep_m)
 {
-    extern __shared__ __align__(16) unsigned char sm_raw[];
-    __shared__ Cand s_red[kWarps];
-    __shared__ int s_maxfree, s_roomiest, s_nlist, s_keep_m;
-    __shared__ long long s_keep;
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     const int cap = E / R;
-    W += (int64_t)blockIdx.x * E * E;
-    p_out += (int64_t)blockIdx.x * E;
-    if (A_global) A_global += (int64_t)blockIdx.x * E * (R + 1);
-
-    Smem s;
-    s.A = a_in_smem ? reinterpret_cast<long long *>(sm_raw) : A_global;
-    s.ar = R + 1;
-    s.cg = reinterpret_cast<long long *>(sm_raw + (a_in_smem ? (size_t)E * (R + 1) * 8 : 0));
-    int *ip = reinterpret_cast<int *>(s.cg + E);
-    s.p = ip;
-    s.fill = ip + E;
-    s.mem = ip + E + R;
-    s.slot = ip + 2 * E + R;
-    s.cb = ip + 3 * E + R;
-    s.list = ip + 4 * E + R;
-    {
-        // KL records after the int arrays: ka, kb, kP, kQ [E/2 + 1] ints, kg
-        // [E/2 + 1] int64 (8-byte aligned), lock [E] bytes
-        int *kp = ip + 5 * E + R;
-        const int h = E / 2 + 1;
-        s.ka = kp;
-        s.kb = kp + h;
-        s.kP = kp + 2 * h;
-        s.kQ = kp + 3 * h;
-        unsigned char *after = reinterpret_cast<unsigned char *>(kp + 4 * h);
-        after = reinterpret_cast<unsigned char *>(((uintptr_t)after + 7) & ~(uintptr_t)7);
-        s.kg = reinterpret_cast<long long *>(after);
-        s.lock = reinterpret_cast<unsigned char *>(s.kg + h);
-    }
-
     // greedy seed: lane j of warp w keeps the candidate of row w + 32 j
     const int a_own = wp + 32 * lane;
     const bool own = a_own < E;
@@ -400,14 +418,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = tid; e < E; e += kThreads) s.p[e] = -1;
         for (int d = tid; d < R; d += kThreads) s.fill[d] = 0;
         if (tid == 0) {
-            s_maxfree = cap;
-            s_roomiest = 0;
+            *s_maxfree = cap;
+            *s_roomiest = 0;
         }
         __syncthreads();
         uint32_t cw = 0;
         int cb = -2;  // -2: not scanned yet, -1: no eligible partner left
         for (int it = 0; it < E; ++it) {
-            const int maxfree = s_maxfree;
+            const int maxfree = *s_maxfree;
             const bool need = own && (cb == -2 || (cb >= 0 && !eligible(s, a_own, cb, cap, maxfree)));
             unsigned m = __ballot_sync(0xffffffffu, need);
             while (m) {
@@ -415,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 m &= m - 1;
                 uint32_t w2;
                 int b2;
-                greedy_row(W, s, E, wp + 32 * j, cap, maxfree, w2, b2);
+                greedy_row(st, s, E, wp + 32 * j, cap, maxfree, w2, b2);
                 if (lane == j) {
                     cw = w2;
                     cb = b2;
@@ -432,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) {
                     const int pa = s.p[win.a], pb = s.p[win.b];
                     if (pa < 0 && pb < 0) {
-                        const int best = s_roomiest;
+                        const int best = *s_roomiest;
                         s.p[win.a] = best;
                         s.p[win.b] = best;
                         s.fill[best] += 2;
@@ -450,8 +468,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int d = lane; d < R; d += 32) key = min(key, (unsigned)s.fill[d] * 64u + (unsigned)d);
                 key = __reduce_min_sync(0xffffffffu, key);
                 if (lane == 0) {
-                    s_maxfree = cap - (int)(key >> 6);
-                    s_roomiest = (int)(key & 63u);
+                    *s_maxfree = cap - (int)(key >> 6);
+                    *s_roomiest = (int)(key & 63u);
                 }
             }
             __syncthreads();
@@ -474,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (refine) {
         // member lists (in any order: every use breaks ties by expert id) and A
         for (int d = tid; d < R; d += kThreads) s.fill[d] = 0;
-        for (int64_t i = tid; i < (int64_t)E * s.ar; i += kThreads) s.A[i] = 0;
+        for (int64_t i = tid; i < (int64_t)E * st.ar; i += kThreads) st.a_zero(i);
         __syncthreads();
         for (int e = tid; e < E; e += kThreads) {
             const int d = s.p[e];
@@ -483,17 +501,94 @@ __global__ void __launch_bounds__(kThreads, 1)
             s.mem[d * cap + sl] = e;
         }
         __syncthreads();
+        for (int e = wp; e < E; e += kWarps)
+            for (int e2 = lane; e2 < E; e2 += 32) {
+                const uint32_t v = st.w_row(e, e2);
+                if (e2 != e && v) st.a_atomic_add(e, s.p[e2], v);
+            }
+        __syncthreads();
+        if (refine == 1) search<false>(st, s, E, R, cap, s_red, s_nlist, s_keep, s_keep_m);
+        else search<true>(st, s, E, R, cap, s_red, s_nlist, s_keep, s_keep_m);
+    }
+}
+
+// One CTA per independent problem (blockIdx.x): W, p_out and A_global point
+// at problem 0 and advance by E*E, E and E*(R+1).  refine: 0 none, 1 best
+// single swaps, 2 Kernighan-Lin passes.  The first `region` bytes of dynamic
+// shared memory hold A (a_in_smem), or W and A compacted when compact_ok and
+// the problem's W allows it; the index arrays follow.
+__global__ void __launch_bounds__(kThreads, 1)
+    k_place(const uint32_t *__restrict__ W, int E, int R, int seed_mode, int refine,
+            int32_t *__restrict__ p_out, long long *__restrict__ A_global, int a_in_smem,
+            int compact_ok, int region)
+{
+    extern __shared__ __align__(16) unsigned char sm_raw[];
+    __shared__ Cand s_red[kWarps];
+    __shared__ int s_maxfree, s_roomiest, s_nlist, s_keep_m;
+    __shared__ long long s_keep;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    W += (int64_t)blockIdx.x * E * E;
+    p_out += (int64_t)blockIdx.x * E;
+    if (A_global) A_global += (int64_t)blockIdx.x * E * (R + 1);
+
+    Smem s;
+    s.cg = reinterpret_cast<long long *>(sm_raw + region);
+    int *ip = reinterpret_cast<int *>(s.cg + E);
+    s.p = ip;
+    s.fill = ip + E;
+    s.mem = ip + E + R;
+    s.slot = ip + 2 * E + R;
+    s.cb = ip + 3 * E + R;
+    s.list = ip + 4 * E + R;
+    {
+        // KL records after the int arrays: ka, kb, kP, kQ [E/2 + 1] ints, kg
+        // [E/2 + 1] int64 (8-byte aligned), lock [E] bytes
+        int *kp = ip + 5 * E + R;
+        const int h = E / 2 + 1;
+        s.ka = kp;
+        s.kb = kp + h;
+        s.kP = kp + 2 * h;
+        s.kQ = kp + 3 * h;
+        unsigned char *after = reinterpret_cast<unsigned char *>(kp + 4 * h);
+        after = reinterpret_cast<unsigned char *>(((uintptr_t)after + 7) & ~(uintptr_t)7);
+        s.kg = reinterpret_cast<long long *>(after);
+        s.lock = reinterpret_cast<unsigned char *>(s.kg + h);
+    }
+
+    int compact = 0;
+    if (compact_ok) {
+        // W symmetric, entries below 2^16, row sums (off the diagonal) below 2^31
+        int bad = 0;
+        for (int64_t i = tid; i < (int64_t)E * E; i += kThreads) {
+            const int a = (int)(i / E), b = (int)(i - (int64_t)a * E);
+            const uint32_t v = __ldg(W + i);
+            if (v > 0xffffu || (b > a && v != __ldg(W + (int64_t)b * E + a))) bad = 1;
+        }
         for (int e = wp; e < E; e += kWarps) {
-            const uint32_t *row = W + (int64_t)e * E;
-            long long *Ae = s.A + (int64_t)e * s.ar;
+            unsigned long long rs = 0;
             for (int e2 = lane; e2 < E; e2 += 32)
-                if (e2 != e && row[e2])
-                    atomicAdd(reinterpret_cast<unsigned long long *>(&Ae[s.p[e2]]),
-                              (unsigned long long)row[e2]);
+                if (e2 != e) rs += __ldg(W + (int64_t)e * E + e2);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+            if (rs >= (1ull << 31)) bad = 1;
+        }
+        compact = !__syncthreads_or(bad);
+        if (compact) {
+            uint16_t *w16 = reinterpret_cast<uint16_t *>(sm_raw);
+            for (int64_t i = tid; i < (int64_t)E * E; i += kThreads) w16[i] = (uint16_t)__ldg(W + i);
         }
         __syncthreads();
-        if (refine == 1) search<false>(W, s, E, R, cap, s_red, &s_nlist, &s_keep, &s_keep_m);
-        else search<true>(W, s, E, R, cap, s_red, &s_nlist, &s_keep, &s_keep_m);
+    }
+    if (compact) {
+        const size_t wb = ((size_t)E * E * 2 + 15) & ~(size_t)15;
+        const Store<true> st{reinterpret_cast<const uint16_t *>(sm_raw),
+                             reinterpret_cast<int *>(sm_raw + wb), E, R + 1};
+        place_body(st, s, E, R, seed_mode, refine, s_red, &s_maxfree, &s_roomiest, &s_nlist, &s_keep,
+                   &s_keep_m);
+    } else {
+        const Store<false> st{W, a_in_smem ? reinterpret_cast<long long *>(sm_raw) : A_global, E, R + 1};
+        place_body(st, s, E, R, seed_mode, refine, s_red, &s_maxfree, &s_roomiest, &s_nlist, &s_keep,
+                   &s_keep_m);
     }
     for (int e = tid; e < E; e += kThreads) p_out[e] = s.p[e];
 }
@@ -543,11 +638,18 @@ int launch_place(const uint32_t *W, int problems, int E, int R, int seed_mode, i
 {
     const size_t a_bytes = (size_t)E * (R + 1) * sizeof(long long);
     const int a_in_smem = refine && a_bytes <= kSmemA ? 1 : 0;
-    const size_t smem = int_smem(E, R) + (a_in_smem ? a_bytes : 0);
+    // W (uint16) and A (int32) in shared memory, if the data allows it
+    const size_t c_bytes = ((size_t)E * E * 2 + 15) / 16 * 16 + (size_t)E * (R + 1) * sizeof(int);
+    const int compact_ok = E <= kCompactMaxE ? 1 : 0;
+    size_t region = a_in_smem ? a_bytes : 0;
+    if (compact_ok && c_bytes > region) region = c_bytes;
+    region = md::align_up(region, 16);
+    const size_t smem = region + int_smem(E, R);
     if (cudaFuncSetAttribute(k_place, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
         return MD_ERR_CUDA;
-    k_place<<<problems, kThreads, smem, s>>>(W, E, R, seed_mode, refine, p, A, a_in_smem);
+    k_place<<<problems, kThreads, smem, s>>>(W, E, R, seed_mode, refine, p, A, a_in_smem, compact_ok,
+                                             (int)region);
     md::count_launches(1);
     return MD_OK;
 }

@@ -223,3 +223,25 @@ def test_place_two_level_full_workload(nodes, refine_mode):
     torch.cuda.synchronize()
     want = oracle.place_two_level(u32(W), 64, nodes, 0, refine_mode)
     assert np.array_equal(p.cpu().numpy(), want)
+
+
+# The search keeps W and A in shared memory (uint16 / int32) when W is
+# symmetric with entries below 2^16; otherwise it reads W from global memory.
+# Both paths must give the oracle's placements.
+@pytest.mark.parametrize("kind", ["large_values", "asymmetric", "large_diagonal"])
+@pytest.mark.parametrize("refine_mode", [1, 2])
+@pytest.mark.parametrize("seed_mode", [0, 1])
+def test_placement_outside_the_compact_path(kind, refine_mode, seed_mode):
+    E, R = 64, 8
+    rng = np.random.default_rng(17)
+    if kind == "large_values":
+        W = _random_w(E, 5, 200_000)
+    elif kind == "asymmetric":
+        W = rng.integers(0, 50, (E, E)).astype(np.uint32)
+    else:
+        W = _random_w(E, 6, 30)
+        W[np.arange(E), np.arange(E)] = 70_000   # only the diagonal is too large
+    p = md.md_place_two_level(torch.from_numpy(W.view(np.int32)).to(DEV), R, 1, seed_mode,
+                              refine_mode)
+    torch.cuda.synchronize()
+    assert np.array_equal(p.cpu().numpy(), oracle.place_two_level(W, R, 1, seed_mode, refine_mode))
