@@ -124,6 +124,13 @@ def _need(t, name, dtype, device=None):
     return t
 
 
+def _room(t, name, n):
+    """The kernels write by computed offsets: a buffer must hold n elements."""
+    if t is not None and t.numel() < n:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs {n}")
+    return t
+
+
 def new_status(device) -> torch.Tensor:
     """A device status word for the dev_status arguments."""
     return torch.zeros(1, dtype=torch.int32, device=device)
@@ -149,6 +156,8 @@ def md_route_topk(logits, k, gate_mode=MD_GATE_TOPK_SOFTMAX, topk_idx=None, topk
         topk_w = torch.empty(T, k, dtype=torch.float32, device=dev)
     _need(topk_idx, "topk_idx", torch.int32, dev)
     _need(topk_w, "topk_w", torch.float32, dev)
+    _room(topk_idx, "topk_idx", T * k)
+    _room(topk_w, "topk_w", T * k)
     rc = lib().md_route_topk(_ptr(logits), T, E, k, gate_mode, _ptr(topk_idx), _ptr(topk_w),
                              _stream(stream, dev))
     _check(rc, "md_route_topk")
@@ -171,6 +180,17 @@ class Layout:
     rank_offsets: torch.Tensor  # int32 [R+1]
     n_rows: torch.Tensor        # int32 [1]
     row_capacity: int
+
+
+def _check_layout(L, T, E, k, R, mode, dev):
+    """A caller's Layout must have the buffers md_dispatch_layout writes."""
+    cap = T * k if mode == MD_CONV else T * min(k, R)
+    for name, n in (("row_of_slot", T * k), ("assign_row", T * k), ("row_token", cap),
+                    ("row_mask", cap), ("send_counts", R * R), ("expert_counts", E),
+                    ("expert_offsets", E + 1), ("rank_offsets", R + 1), ("n_rows", 1)):
+        t = getattr(L, name)
+        _need(t, name, torch.int32, dev)
+        _room(t, name, n)
 
 
 def dispatch_layout_workspace_size(T, E, k, R, mode) -> int:
@@ -200,6 +220,7 @@ def md_dispatch_layout(topk_idx, E, R, expert_to_rank, mode, out: Layout | None 
     T, k = topk_idx.shape
     if out is None:
         out = alloc_layout(T, E, k, R, mode, dev)
+    _check_layout(out, T, E, k, R, mode, dev)
     need = dispatch_layout_workspace_size(T, E, k, R, mode)
     if workspace is None:
         workspace = alloc_workspace(need, dev)
@@ -225,6 +246,7 @@ def md_dispatch_layout_noalloc(topk_idx, E, R, expert_to_rank, mode, out: Layout
     T, k = topk_idx.shape
     if out is None:
         out = alloc_layout(T, E, k, R, mode, dev)
+    _check_layout(out, T, E, k, R, mode, dev)
     rc = lib().md_dispatch_layout_noalloc(
         _ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), mode, _ptr(out.row_of_slot),
         _ptr(out.assign_row), _ptr(out.row_token), _ptr(out.row_mask), _ptr(out.send_counts),
@@ -246,6 +268,8 @@ def md_dispatch_permute(x, row_of_slot, out_rows=None, out=None, dev_status=None
         out = torch.empty(out_rows if out_rows is not None else T * k, H, dtype=torch.bfloat16,
                           device=dev)
     _need(out, "out", torch.bfloat16, dev)
+    if out.dim() != 2 or out.shape[1] != H:
+        raise ValueError(f"out must be [rows, {H}]")
     rc = lib().md_dispatch_permute(_ptr(x), T, H, k, _ptr(row_of_slot), out.shape[0], _ptr(out),
                                    _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_dispatch_permute")
@@ -261,10 +285,14 @@ def md_dedup_expand(wire, row_of_slot, assign_row, out_rows=None, out=None, dev_
     _need(assign_row, "assign_row", torch.int32, dev)
     T, k = row_of_slot.shape
     H = wire.shape[1]
+    if assign_row.shape != row_of_slot.shape:
+        raise ValueError("assign_row and row_of_slot differ in shape")
     if out is None:
         out = torch.empty(out_rows if out_rows is not None else T * k, H, dtype=torch.bfloat16,
                           device=dev)
     _need(out, "out", torch.bfloat16, dev)
+    if out.dim() != 2 or out.shape[1] != H:
+        raise ValueError(f"out must be [rows, {H}]")
     rc = lib().md_dedup_expand(_ptr(wire), wire.shape[0], H, _ptr(row_of_slot), _ptr(assign_row), T,
                                k, out.shape[0], _ptr(out), _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_dedup_expand")
@@ -283,10 +311,14 @@ def md_combine(y, assign_row, topk_idx, topk_w, mode=MD_COMBINE_FUSED, row_of_sl
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
     _need(out, "out", torch.bfloat16, dev)
+    _room(out, "out", T * H)
+    _room(assign_row, "assign_row", T * k)
+    _room(topk_w, "topk_w", T * k)
     z_rows = 0
     if mode == MD_COMBINE_WIRE:
         _need(row_of_slot, "row_of_slot", torch.int32, dev)
         _need(z, "z", torch.bfloat16, dev)
+        _room(row_of_slot, "row_of_slot", T * k)
         z_rows = z.shape[0]
     rc = lib().md_combine(_ptr(y), y.shape[0], _ptr(assign_row), _ptr(topk_idx), _ptr(topk_w), T,
                           k, H, mode, _ptr(row_of_slot), z_rows, _ptr(z), _ptr(out),
@@ -303,8 +335,9 @@ def md_gather_rows(src, index, out=None, dev_status=None, stream=None):
     n = index.shape[0]
     if out is None:
         out = torch.empty((n,) + tuple(src.shape[1:]), dtype=src.dtype, device=dev)
-    if out.dtype != src.dtype or not out.is_contiguous():
-        raise ValueError("out must be contiguous and of src's dtype")
+    if out.dtype != src.dtype or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor of src's dtype")
+    _room(out, "out", n * (src[0].numel() if src.shape[0] else out[0].numel()))
     row_bytes = src[0].numel() * src.element_size() if src.shape[0] else \
         out[0].numel() * out.element_size()
     rc = lib().md_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out),
@@ -327,9 +360,16 @@ def md_coselect_stats(idx_l, idx_next, E, T_fit=None, W=None, C=None, accumulate
         W = torch.empty(E, E, dtype=torch.int32, device=dev)
     if C is None and want_C and idx_next is not None:
         C = torch.empty(E, E, dtype=torch.int32, device=dev)
+    if idx_next is not None and idx_next.shape[1] != k:
+        raise ValueError("idx_l and idx_next differ in k")
+    if idx_next is not None and idx_next.shape[0] < T_fit:
+        raise ValueError("idx_next has fewer than T_fit rows")
+    if T_fit > T:
+        raise ValueError("T_fit exceeds the rows of idx_l")
     for t, n in ((W, "W"), (C, "C")):
         if t is not None:
             _need(t, n, torch.int32, dev)
+            _room(t, n, E * E)
     rc = lib().md_coselect_stats(_ptr(idx_l), _ptr(idx_next), T_fit, E, k, _ptr(W), _ptr(C),
                                  1 if accumulate else 0, _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_coselect_stats")
@@ -341,8 +381,12 @@ def md_place_correlated(W, R, seed_mode=MD_SEED_CONTIGUOUS, refine=True, out=Non
     _need(W, "W", torch.int32)
     dev = W.device
     E = W.shape[0]
+    if W.dim() != 2 or W.shape[1] != E:
+        raise ValueError("W must be [E, E]")
     if out is None:
         out = torch.empty(E, dtype=torch.int32, device=dev)
+    _need(out, "out", torch.int32, dev)
+    _room(out, "out", E)
     need = int(lib().md_place_correlated_workspace_size(E, R))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
@@ -360,8 +404,12 @@ def md_place_two_level(W, R, nodes=1, seed_mode=MD_SEED_CONTIGUOUS, refine_mode=
     _need(W, "W", torch.int32)
     dev = W.device
     E = W.shape[0]
+    if W.dim() != 2 or W.shape[1] != E:
+        raise ValueError("W must be [E, E]")
     if out is None:
         out = torch.empty(E, dtype=torch.int32, device=dev)
+    _need(out, "out", torch.int32, dev)
+    _room(out, "out", E)
     need = int(lib().md_place_two_level_workspace_size(E, R, nodes))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
@@ -370,6 +418,15 @@ def md_place_two_level(W, R, nodes=1, seed_mode=MD_SEED_CONTIGUOUS, refine_mode=
                                   _stream(stream, dev))
     _check(rc, "md_place_two_level")
     return out
+
+
+def _shuffle_checks(C, E, p_next, T, dev, **outs):
+    if C.dim() != 2 or C.shape[1] != E:
+        raise ValueError("C must be [E, E]")
+    _room(p_next, "expert_to_rank_next", E)
+    for name, t in outs.items():
+        _need(t, name, torch.int32, dev)
+        _room(t, name, T)
 
 
 def md_token_shuffle(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None, inv=None,
@@ -384,6 +441,7 @@ def md_token_shuffle(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None
     pred_rank = torch.empty(T, **i32) if pred_rank is None else pred_rank
     perm = torch.empty(T, **i32) if perm is None else perm
     inv = torch.empty(T, **i32) if inv is None else inv
+    _shuffle_checks(C, E, expert_to_rank_next, T, dev, pred_rank=pred_rank, perm=perm, inv=inv)
     need = int(lib().md_token_shuffle_workspace_size(T, E, R))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
@@ -406,6 +464,11 @@ def md_coselect_pair_stats(idx_prev, idx_l, idx_next, E, T_fit=None, C2=None, ac
     if C2 is None:
         C2 = torch.empty(E, E, E, dtype=torch.int32, device=dev)
     _need(C2, "C2", torch.int32, dev)
+    _room(C2, "C2", E * E * E)
+    if idx_prev.shape[1] != k or idx_next.shape[1] != k:
+        raise ValueError("idx_prev, idx_l and idx_next differ in k")
+    if min(idx_prev.shape[0], idx_next.shape[0], T) < T_fit:
+        raise ValueError("fewer than T_fit rows")
     rc = lib().md_coselect_pair_stats(_ptr(idx_prev), _ptr(idx_l), _ptr(idx_next), T_fit, E, k,
                                       _ptr(C2), 1 if accumulate else 0, _ptr(dev_status),
                                       _stream(stream, dev))
@@ -430,7 +493,11 @@ def md_token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_ob
     perm = torch.empty(T, **i32) if perm is None else perm
     inv = torch.empty(T, **i32) if inv is None else inv
     use_pair = torch.empty(T, **i32) if use_pair is None else use_pair
-    need = int(lib().md_token_shuffle_pair_workspace_size(T, E, R))
+    _shuffle_checks(C, E, expert_to_rank_next, T, dev, pred_rank=pred_rank, perm=perm, inv=inv,
+                    use_pair=use_pair)
+    if idx_prev.shape != idx_l.shape:
+        raise ValueError("idx_prev and idx_l differ in shape")
+    _room(C2, "C2", E * E * E)
     if workspace is None:
         workspace = alloc_workspace(need, dev)
     rc = lib().md_token_shuffle_pair(_ptr(idx_prev), _ptr(idx_l), k, _ptr(C), _ptr(C2),
@@ -452,6 +519,8 @@ def md_rank_stats(topk_idx, E, R, expert_to_rank, hist=None, dev_status=None, st
     T, k = topk_idx.shape
     hist = torch.empty(k + 1, dtype=torch.int64, device=dev) if hist is None else hist
     _need(hist, "hist", torch.int64, dev)
+    _room(hist, "hist", k + 1)
+    _room(expert_to_rank, "expert_to_rank", E)
     rc = lib().md_rank_stats(_ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), _ptr(hist),
                              _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_rank_stats")
@@ -472,6 +541,8 @@ def md_successor_share(C, W, stream=None):
     dev = C.device
     _need(W, "W", torch.int32, dev)
     E = C.shape[0]
+    if C.shape != (E, E) or W.shape != (E, E):
+        raise ValueError("C and W must be [E, E]")
     num = torch.empty(E, dtype=torch.int32, device=dev)
     den = torch.empty(E, dtype=torch.int32, device=dev)
     rc = lib().md_successor_share(_ptr(C), _ptr(W), E, _ptr(num), _ptr(den), _stream(stream, dev))
