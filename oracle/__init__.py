@@ -70,6 +70,7 @@ def _load():
             lib.oracle_successor_share.argtypes = [P, P, I32, P, P]
             lib.oracle_count_sums.argtypes = [P, P, I64, P]
             lib.oracle_place_two_level.argtypes = [P, I32, I32, I32, I32, I32, P]
+            lib.oracle_token_shuffle_rounds.argtypes = [P, P, P, I64, I32, I32, I32, P, P, P, P]
             lib.oracle_token_shuffle_pair.argtypes = [P, P, P, P, P, I64, I32, I32, I32,
                                                       ctypes.c_uint64, P, P, P, P]
             for name in ("oracle_route_topk", "oracle_dispatch_layout", "oracle_dispatch_permute",
@@ -78,7 +79,7 @@ def _load():
                          "oracle_token_shuffle", "oracle_coselect_pair",
                          "oracle_token_shuffle_pair", "oracle_rank_stats",
                          "oracle_successor_share", "oracle_count_sums",
-                         "oracle_place_two_level"):
+                         "oracle_place_two_level", "oracle_token_shuffle_rounds"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -329,3 +330,20 @@ def place_two_level(W, R, nodes=1, seed_mode=0, refine_mode=REFINE_SWAPS):
     _check(lib.oracle_place_two_level(_ptr(Wc), E, R, nodes, seed_mode, refine_mode, _ptr(p)),
            "place_two_level")
     return p
+
+
+def token_shuffle_rounds(idx_l, C, expert_to_rank_next, R):
+    """Rounds-based capacity assignment -> (pred, perm, inv, rounds)."""
+    lib = _load()
+    ix = _c(idx_l, np.int32)
+    T, k = ix.shape
+    Cc = _c(C, np.uint32)
+    E = Cc.shape[0]
+    pn = _c(expert_to_rank_next, np.int32)
+    pred = np.empty(T, np.int32)
+    perm = np.empty(T, np.int32)
+    inv = np.empty(T, np.int32)
+    rounds = np.zeros(1, np.int32)
+    _check(lib.oracle_token_shuffle_rounds(_ptr(ix), _ptr(Cc), _ptr(pn), T, E, k, R, _ptr(pred),
+                                           _ptr(perm), _ptr(inv), _ptr(rounds)), "token_shuffle_rounds")
+    return pred, perm, inv, int(rounds[0])

@@ -1001,3 +1001,96 @@ int oracle_place_two_level(const uint32_t *W, int E, int R, int nodes, int seed_
     free(pn); free(mem); free(sub); free(pg);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Rounds-based capacity assignment (a parallel alternative to the          */
+/* sequential visit of [EC] Method 2, Capacity Constraint).  Priorities and */
+/* preference lists are those of oracle_token_shuffle.  In each round every  */
+/* unassigned token proposes to the first rank of its list that was not     */
+/* full when the round began; each rank accepts its highest-priority         */
+/* proposers up to its remaining capacity and the others stay unassigned.   */
+/* Rounds repeat until every token is assigned: a round either accepts all  */
+/* its proposers or fills at least one rank, so there are at most R + 1.    */
+/* rounds_out = the number of rounds that accepted at least one token.      */
+/* ------------------------------------------------------------------------ */
+
+int oracle_token_shuffle_rounds(const int32_t *idx_l, const uint32_t *C, const int32_t *p_next,
+                                int64_t T, int E, int k, int R, int32_t *pred_rank,
+                                int32_t *perm, int32_t *inv, int32_t *rounds_out)
+{
+    if (T < 0 || E < 1 || k < 1 || R < 1 || T % R != 0) return 1;
+    const int64_t Tr = T / R;
+    int32_t *pref = (int32_t *)malloc(sizeof(int32_t) * (size_t)E * R);
+    uint64_t *num = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)E);
+    uint64_t *den = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)E);
+    uint64_t *sigma = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)R);
+    conf_t *order = (conf_t *)malloc(sizeof(conf_t) * (size_t)(T > 0 ? T : 1));
+    int64_t *load = (int64_t *)calloc((size_t)R, sizeof(int64_t));
+    int64_t *taken = (int64_t *)calloc((size_t)R, sizeof(int64_t));
+    char *full = (char *)calloc((size_t)R, 1);
+    int rc = 0, rounds = 0;
+    if (!pref || !num || !den || !sigma || !order || !load || !taken || !full) { rc = 2; goto done; }
+
+    for (int e1 = 0; e1 < E; ++e1)
+        row_prediction(C + (int64_t)e1 * E, E, p_next, R, sigma, pref + (int64_t)e1 * R, &num[e1],
+                       &den[e1]);
+    for (int64_t t = 0; t < T; ++t) {
+        int e1 = idx_l[t * k];
+        if (e1 < 0 || e1 >= E) { rc = 1; goto done; }
+        order[t].num = num[e1];
+        order[t].den = den[e1];
+        order[t].t = t;
+        pred_rank[t] = -1;
+    }
+    qsort(order, (size_t)T, sizeof(conf_t), cmp_conf);
+
+    for (int round = 0; round <= R; ++round) {
+        int64_t accepted = 0, left = 0;
+        for (int d = 0; d < R; ++d) {
+            taken[d] = 0;
+            full[d] = load[d] >= Tr;
+        }
+        /* visiting proposers in priority order, rank d accepts while it has
+         * room left from the start of the round */
+        for (int64_t i = 0; i < T; ++i) {
+            int64_t t = order[i].t;
+            if (pred_rank[t] >= 0) continue;
+            int e1 = idx_l[t * k], d = -1;
+            if (den[e1] == 0) {
+                int s = (int)(t / Tr);
+                if (!full[s]) d = s;
+                for (int q = 0; d < 0 && q < R; ++q)
+                    if (!full[q]) d = q;
+            } else {
+                const int32_t *pl = pref + (int64_t)e1 * R;
+                for (int n = 0; d < 0 && n < R; ++n)
+                    if (!full[pl[n]]) d = pl[n];
+            }
+            if (d < 0) { rc = 1; goto done; }
+            if (load[d] + taken[d] < Tr) {
+                pred_rank[t] = d;
+                taken[d] += 1;
+                ++accepted;
+            } else {
+                ++left;
+            }
+        }
+        for (int d = 0; d < R; ++d) load[d] += taken[d];
+        if (accepted) ++rounds;
+        if (!left) break;
+    }
+    *rounds_out = rounds;
+
+    for (int d = 0; d < R; ++d) load[d] = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        int d = pred_rank[t];
+        if (d < 0) { rc = 1; goto done; }
+        int64_t pos = (int64_t)d * Tr + load[d];
+        load[d] += 1;
+        perm[t] = (int32_t)pos;
+        inv[pos] = (int32_t)t;
+    }
+done:
+    free(pref); free(num); free(den); free(sigma); free(order); free(load); free(taken); free(full);
+    return rc;
+}
