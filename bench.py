@@ -386,10 +386,22 @@ def run_rows(args, md, device, stream, peak):
     bs = b[inv.long()]
     loc_after = float((torch.arange(w.T, device=device) // (w.T // w.R)).eq(
         w.expert_to_rank[bs.long()].T).float().mean())
+    # the rounds-based parallel assignment on the same inputs
+    rws = md.alloc_workspace(int(md.lib().md_token_shuffle_rounds_workspace_size(w.T, w.E, w.R)),
+                             device)
+    rp, rperm, rinv = torch.empty_like(pred), torch.empty_like(pred), torch.empty_like(pred)
+    holder = {}
+    t_rd = _time(lambda: holder.__setitem__("r", md.md_token_shuffle_rounds(
+        a, C, w.expert_to_rank, w.R, rp, rperm, rinv, workspace=rws, stream=stream)[3]), stream, reps)
+    n_rounds = int(holder["r"].item())
+    loc_rounds = float((torch.arange(w.T, device=device) // (w.T // w.R)).eq(
+        w.expert_to_rank[b[rinv.long()].long()].T).float().mean())
     rows["token_shuffle_e128_k6"] = {
         "T": w.T, "shuffle_us": round(t_sh * 1e3, 2), "gather_x_us": round(t_g * 1e3, 2),
         "gather": gbps(2 * w.T * 2 * w.H + 4 * w.T, t_g),
-        "locality_before": round(loc_before, 4), "locality_after": round(loc_after, 4)}
+        "locality_before": round(loc_before, 4), "locality_after": round(loc_after, 4),
+        "rounds_variant": {"us": round(t_rd * 1e3, 2), "rounds": n_rounds,
+                           "locality_after": round(loc_rounds, 4)}}
     del w, a, b, C, sws, xs
     torch.cuda.empty_cache()
 

@@ -50,6 +50,8 @@ _SIGNATURES = {
     "md_token_shuffle_workspace_size": ([_L, _I, _I], _S),
     "md_token_shuffle": ([_P, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _S, _P, _P], _I),
     "md_coselect_pair_stats": ([_P, _P, _P, _L, _I, _I, _P, _I, _P, _P], _I),
+    "md_token_shuffle_rounds_workspace_size": ([_L, _I, _I], _S),
+    "md_token_shuffle_rounds": ([_P, _I, _P, _P, _L, _I, _I, _P, _P, _P, _P, _P, _S, _P, _P], _I),
     "md_rank_stats": ([_P, _L, _I, _I, _I, _P, _P, _P, _P], _I),
     "md_set_test_hooks": ([ctypes.c_longlong, _I, ctypes.c_longlong], None),
     "md_place_two_level_workspace_size": ([_I, _I, _I], _S),
@@ -450,6 +452,32 @@ def md_token_shuffle(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None
                                 workspace.numel(), _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_token_shuffle")
     return pred_rank, perm, inv
+
+
+def md_token_shuffle_rounds(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None,
+                            inv=None, workspace=None, dev_status=None, stream=None):
+    """Rounds-based capacity assignment -> (pred, perm, inv, rounds [1] device tensor)."""
+    _need(idx_l, "idx_l", torch.int32)
+    dev = idx_l.device
+    _need(C, "C", torch.int32, dev)
+    _need(expert_to_rank_next, "expert_to_rank_next", torch.int32, dev)
+    T, k = idx_l.shape
+    E = C.shape[0]
+    i32 = dict(dtype=torch.int32, device=dev)
+    pred_rank = torch.empty(T, **i32) if pred_rank is None else pred_rank
+    perm = torch.empty(T, **i32) if perm is None else perm
+    inv = torch.empty(T, **i32) if inv is None else inv
+    _shuffle_checks(C, E, expert_to_rank_next, T, dev, pred_rank=pred_rank, perm=perm, inv=inv)
+    rounds = torch.zeros(1, **i32)
+    need = int(lib().md_token_shuffle_rounds_workspace_size(T, E, R))
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    rc = lib().md_token_shuffle_rounds(_ptr(idx_l), k, _ptr(C), _ptr(expert_to_rank_next), T, E, R,
+                                       _ptr(pred_rank), _ptr(perm), _ptr(inv), _ptr(rounds),
+                                       _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                       _stream(stream, dev))
+    _check(rc, "md_token_shuffle_rounds")
+    return pred_rank, perm, inv, rounds
 
 
 def md_coselect_pair_stats(idx_prev, idx_l, idx_next, E, T_fit=None, C2=None, accumulate=False,

@@ -727,6 +727,214 @@ __global__ void __launch_bounds__(32)
     }
 }
 
+// ------------------------------------------------------ rounds assignment
+// A parallel alternative to the sequential visit.  In each round every
+// unassigned token proposes to the first rank of its preference list that
+// was not full when the round began, and each rank accepts its
+// highest-priority proposers up to its remaining capacity.  One cooperative
+// launch: CTA c owns positions [c*1024, (c+1)*1024) of the priority order.
+// Phase 1 counts the tile's proposals per rank; after a grid barrier, phase
+// 2 places each proposer among the proposers of its rank (earlier tiles
+// first, then tile order, one warp with __match_any_sync) and accepts it if
+// that place is inside the remaining capacity; after a second barrier the
+// next round starts.  At most R + 1 rounds.  The grid barrier waits are
+// bounded (MD_ERR_TIMEOUT, and every CTA then stops).
+constexpr int kRoundThreads = 256;
+constexpr long long kBarrierPolls = 1ll << 22;
+
+struct RoundWs {
+    int32_t *rem;        // [R] capacity left at the start of the round
+    int32_t *cnt;        // [n_tiles * R] proposals per tile and rank
+    unsigned *bar;       // [0] arrivals, [1] generation
+    int32_t *abort;      // [0] set when a barrier wait ran out
+    int32_t *rounds;     // [0] rounds that accepted a token
+};
+
+size_t round_layout(int64_t T, int R, RoundWs *w, void *base)
+{
+    char *b = static_cast<char *>(base);
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        char *q = b ? b + o : nullptr;
+        o += md::align_up(bytes, 256);
+        return q;
+    };
+    const int64_t n_tiles = T > 0 ? (T + kTile - 1) / kTile : 1;
+    RoundWs x;
+    x.bar = reinterpret_cast<unsigned *>(take(4 * sizeof(unsigned)));
+    x.abort = reinterpret_cast<int32_t *>(take(sizeof(int32_t)));
+    x.rounds = reinterpret_cast<int32_t *>(take(sizeof(int32_t)));
+    x.rem = reinterpret_cast<int32_t *>(take((size_t)R * 4));
+    x.cnt = reinterpret_cast<int32_t *>(take((size_t)n_tiles * R * 4));
+    if (w) *w = x;
+    return o;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// All CTAs of the (cooperative, hence co-resident) grid meet here; false if
+// a wait ran out somewhere.
+__device__ bool grid_barrier(RoundWs rw, unsigned n_ctas, int32_t *status)
+{
+    __shared__ int s_ok;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned gen = ld_acquire_u32(rw.bar + 1);
+        __threadfence();
+        if (atomicAdd(rw.bar, 1u) + 1u == n_ctas) {
+            atomicExch(rw.bar, 0u);
+            __threadfence();
+            atomicAdd(rw.bar + 1, 1u);
+        } else {
+            long long n = 0;
+            while (ld_acquire_u32(rw.bar + 1) == gen) {
+                if (++n > kBarrierPolls || *(volatile int32_t *)rw.abort) {
+                    md::report(status, MD_ERR_TIMEOUT);
+                    atomicExch(rw.abort, 1);
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        s_ok = *(volatile int32_t *)rw.abort == 0;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+__global__ void __launch_bounds__(kRoundThreads)
+    k_shuf_rounds(const int32_t *__restrict__ order, const int32_t *__restrict__ idx_l, int k,
+                  ShufWs ws, RoundWs rw, int64_t T, int E, int R, int64_t Tr,
+                  int32_t *__restrict__ pred, int32_t *status)
+{
+    extern __shared__ unsigned char s_pref[];  // [E*R] preference lists, staged once
+    __shared__ int s_tok[kTile];              // token at each position of the tile (-1: none)
+    __shared__ short s_key[kTile];            // its top-1 expert, or -1 for an empty row
+    __shared__ signed char s_prop[kTile];     // this round's proposal (-1: none)
+    __shared__ unsigned char s_done[kTile];   // placed in an earlier round
+    __shared__ int s_cnt[MD_MAX_RANKS], s_rem[MD_MAX_RANKS], s_base[MD_MAX_RANKS], s_tot[MD_MAX_RANKS];
+    __shared__ unsigned long long s_full;
+    __shared__ int s_any;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    const int tile = blockIdx.x;
+    const unsigned n_ctas = gridDim.x;
+    const int64_t p0 = (int64_t)tile * kTile;
+
+    for (int i = tid; i < E * R; i += kRoundThreads) s_pref[i] = (unsigned char)ws.pref[i];
+    for (int i = tid; i < kTile; i += kRoundThreads) {
+        const int64_t pos = p0 + i;
+        int t = -1, key = -1;
+        s_done[i] = 0;
+        if (pos < T) {
+            t = order[pos];
+            int e1 = idx_l[(int64_t)t * k];
+            if (e1 < 0 || e1 >= E) {
+                md::report(status, MD_ERR_DATA);
+                e1 = 0;
+            }
+            key = ws.den[e1] == 0ull ? -1 : e1;
+            pred[t] = -1;
+        }
+        s_tok[i] = t;
+        s_key[i] = (short)key;
+    }
+    if (tile == 0) {
+        for (int d = tid; d < R; d += kRoundThreads) rw.rem[d] = (int)Tr;
+        if (tid == 0) *rw.rounds = 0;
+    }
+    if (!grid_barrier(rw, n_ctas, status)) return;
+
+    for (int round = 0; round <= R; ++round) {
+        // ---- phase 1: proposals
+        for (int d = tid; d < R; d += kRoundThreads) {
+            s_rem[d] = rw.rem[d];
+            s_cnt[d] = 0;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            unsigned long long f = 0ull;
+            for (int d = 0; d < R; ++d)
+                if (s_rem[d] <= 0) f |= 1ull << d;
+            s_full = f;
+        }
+        __syncthreads();
+        const unsigned long long full = s_full;
+        for (int i = tid; i < kTile; i += kRoundThreads) {
+            const int t = s_tok[i];
+            int d = -1;
+            if (t >= 0 && !s_done[i]) {
+                const int key = s_key[i];
+                if (key < 0) {
+                    const int src = (int)(t / Tr);
+                    if (!((full >> src) & 1ull)) d = src;
+                    for (int q = 0; d < 0 && q < R; ++q)
+                        if (!((full >> q) & 1ull)) d = q;
+                } else {
+                    const unsigned char *pl = s_pref + (size_t)key * R;
+                    for (int n = 0; d < 0 && n < R; ++n)
+                        if (!((full >> pl[n]) & 1ull)) d = pl[n];
+                }
+                if (d >= 0) atomicAdd(&s_cnt[d], 1);
+            }
+            s_prop[i] = (signed char)d;
+        }
+        __syncthreads();
+        for (int d = tid; d < R; d += kRoundThreads) rw.cnt[(int64_t)tile * R + d] = s_cnt[d];
+        if (!grid_barrier(rw, n_ctas, status)) return;
+
+        // ---- phase 2: places among each rank's proposers, acceptance.  The
+        // (tile, rank) counts are summed by all threads at once: the earlier
+        // tiles' counts give this tile's base, all tiles' the rank's total.
+        for (int d = tid; d < R; d += kRoundThreads) {
+            s_base[d] = 0;
+            s_tot[d] = 0;
+            s_cnt[d] = 0;
+        }
+        if (tid == 0) s_any = 0;
+        __syncthreads();
+        for (int64_t c = tid; c < (int64_t)n_ctas * R; c += kRoundThreads) {
+            const int v = rw.cnt[c];
+            if (!v) continue;
+            const int j = (int)(c / R), d = (int)(c - (int64_t)j * R);
+            atomicAdd(&s_tot[d], v);
+            if (j < tile) atomicAdd(&s_base[d], v);
+            s_any = 1;
+        }
+        __syncthreads();
+        if (!s_any) break;  // every token placed (the same on every CTA)
+        if (wp == 0) {
+            for (int c0 = 0; c0 < kTile; c0 += 32) {
+                const int i = c0 + lane;
+                const int d = s_prop[i];
+                const unsigned g = __match_any_sync(0xffffffffu, d >= 0 ? (unsigned)d : (0x80000000u | lane));
+                int within = 0;
+                if (d >= 0) within = s_cnt[d] + __popc(g & md::lanemask_lt());
+                __syncwarp();
+                if (d >= 0 && (g & md::lanemask_lt()) == 0u) s_cnt[d] += __popc(g);
+                __syncwarp();
+                if (d >= 0 && s_base[d] + within < s_rem[d]) {
+                    pred[s_tok[i]] = d;
+                    s_done[i] = 1;
+                }
+            }
+        }
+        if (tile == 0) {
+            for (int d = tid; d < R; d += kRoundThreads) {
+                const int left = s_rem[d] - s_tot[d];
+                rw.rem[d] = left > 0 ? left : 0;
+            }
+            if (tid == 0) *rw.rounds += 1;
+        }
+        if (!grid_barrier(rw, n_ctas, status)) return;
+    }
+}
+
 }  // namespace
 
 extern "C" size_t md_token_shuffle_workspace_size(int64_t T, int E, int R)
@@ -843,5 +1051,88 @@ extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx
     k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, R, pw.keys, pw.tile_hist, nullptr,
                                                          perm, inv);
     md::count_launches(1 + 3 * kRadixPasses + 1 + 3);
+    return md::launch_status();
+}
+
+extern "C" size_t md_token_shuffle_rounds_workspace_size(int64_t T, int E, int R)
+{
+    if (T < 0 || E < 1 || R < 1) return 0;
+    return shuf_layout(T, E, R, nullptr, nullptr) + round_layout(T, R, nullptr, nullptr);
+}
+
+extern "C" int md_token_shuffle_rounds(const int32_t *idx_l, int k, const uint32_t *C,
+                                       const int32_t *expert_to_rank_next, int64_t T, int E, int R,
+                                       int32_t *pred_rank, int32_t *perm, int32_t *inv,
+                                       int32_t *rounds, void *workspace, size_t workspace_bytes,
+                                       int32_t *dev_status, void *stream)
+{
+    if (T < 0 || E < 1 || R < 1 || k < 1 || k > MD_MAX_TOPK) return MD_ERR_ARG;
+    if (E > MD_MAX_EXPERTS || R > MD_MAX_RANKS || T >= ((int64_t)1 << 31)) return MD_ERR_UNSUPPORTED;
+    if (E > 32767) return MD_ERR_UNSUPPORTED;
+    if (T % R != 0) return MD_ERR_ARG;
+    if (!C || !expert_to_rank_next) return MD_ERR_ARG;
+    if (T > 0 && (!idx_l || !pred_rank || !perm || !inv)) return MD_ERR_ARG;
+    const size_t need_s = shuf_layout(T, E, R, nullptr, nullptr);
+    const size_t need = need_s + round_layout(T, R, nullptr, nullptr);
+    if (!workspace || workspace_bytes < need) return MD_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MD_ERR_ARG;
+    const int n_tiles = (int)((T + kTile - 1) / kTile);
+    // every CTA must be resident at once (cooperative launch)
+    const size_t rsm = (size_t)E * R;
+    if (cudaFuncSetAttribute(k_shuf_rounds, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsm) !=
+        cudaSuccess)
+        return MD_ERR_CUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_shuf_rounds, kRoundThreads, rsm) !=
+        cudaSuccess)
+        return MD_ERR_CUDA;
+    if (T > 0 && (int64_t)per_sm * md::sm_count() < n_tiles) return MD_ERR_UNSUPPORTED;
+    cudaStream_t s = md::as_stream(stream);
+    int rc = md::clear_status(dev_status, s);
+    if (rc != MD_OK) return rc;
+    ShufWs ws;
+    shuf_layout(T, E, R, &ws, workspace);
+    RoundWs rw;
+    round_layout(T, R, &rw, static_cast<char *>(workspace) + need_s);
+    md::count_launches(1);
+    if (cudaMemsetAsync(rw.bar, 0, 256 * 3, s) != cudaSuccess) return MD_ERR_CUDA;  // bar, abort, rounds
+    if (T == 0) {
+        if (rounds) {
+            md::count_launches(1);
+            if (cudaMemsetAsync(rounds, 0, sizeof(int32_t), s) != cudaSuccess) return MD_ERR_CUDA;
+        }
+        return MD_OK;
+    }
+    const int64_t Tr = T / R;
+    k_shuf_prefs<<<E, 256, 0, s>>>(C, expert_to_rank_next, E, R, ws, dev_status);
+    k_shuf_class<<<(E + 255) / 256, 256, 0, s>>>(E, ws);
+    const int nbk0 = E + 1;
+    k_bucket_hist<<<n_tiles, 256, nbk0 * sizeof(int), s>>>(0, T, idx_l, k, ws.cls, E, nullptr, nbk0,
+                                                          ws.keys, ws.tile_hist);
+    k_bucket_scan<<<1, kScanThreads, nbk0 * sizeof(int), s>>>(ws.tile_hist, n_tiles, nbk0);
+    k_bucket_scatter<<<n_tiles, 32, nbk0 * sizeof(int), s>>>(0, T, nbk0, ws.keys, ws.tile_hist,
+                                                            ws.order, nullptr, nullptr);
+    const int32_t *order = ws.order;
+    int kk = k;
+    int64_t TT = T, TTr = Tr;
+    int EE = E, RR = R;
+    void *args[] = {(void *)&order, (void *)&idx_l, (void *)&kk, (void *)&ws, (void *)&rw,
+                    (void *)&TT, (void *)&EE, (void *)&RR, (void *)&TTr, (void *)&pred_rank,
+                    (void *)&dev_status};
+    if (cudaLaunchCooperativeKernel((const void *)k_shuf_rounds, dim3(n_tiles), dim3(kRoundThreads),
+                                    args, rsm, s) != cudaSuccess)
+        return MD_ERR_CUDA;
+    k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
+                                                       ws.keys, ws.tile_hist);
+    k_bucket_scan<<<1, kScanThreads, R * sizeof(int), s>>>(ws.tile_hist, n_tiles, R);
+    k_bucket_scatter<<<n_tiles, 32, R * sizeof(int), s>>>(1, T, R, ws.keys, ws.tile_hist, nullptr,
+                                                         perm, inv);
+    md::count_launches(9);
+    if (rounds) {
+        md::count_launches(1);
+        if (cudaMemcpyAsync(rounds, rw.rounds, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+            return MD_ERR_CUDA;
+    }
     return md::launch_status();
 }

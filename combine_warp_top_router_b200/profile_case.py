@@ -4,7 +4,7 @@ profiling a single kernel under ncu on a small case.
     python -m combine_warp_top_router_b200.profile_case --steps layout,permute \
         --workload zipf_pairs_e128_k8 --T 16384 --reps 3
 
-Steps: topk, layout, permute, combine, wire, expand, coselect, place, shuffle,
+Steps: topk, layout, permute, combine, wire, expand, coselect, place, shuffle, shuffle_rounds,
 shuffle_pair (three_layer_e128_k6 only), gather.
 Every listed step runs once as warm-up and then `reps` times.
 """
@@ -74,6 +74,8 @@ def main():
                 md.md_place_correlated(W, R)
             elif s == "shuffle":
                 md.md_token_shuffle(idx, C, w.expert_to_rank, R)
+            elif s == "shuffle_rounds":
+                md.md_token_shuffle_rounds(idx, C, w.expert_to_rank, R)
             elif s == "gather":
                 md.md_gather_rows(w.x, torch.arange(T, dtype=torch.int32, device=dev).flip(0))
             else:

@@ -353,6 +353,31 @@ int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
                      void *stream);
 
 /*
+ * md_token_shuffle_rounds -- md_token_shuffle with a rounds-based parallel
+ * capacity assignment in place of the sequential visit.  Priorities and
+ * preference lists are md_token_shuffle's.  In each round every unassigned
+ * token proposes to the first rank of its list that was not full when the
+ * round began, and each rank accepts its highest-priority proposers up to
+ * its remaining capacity; rounds repeat until every token is placed (at most
+ * R + 1).  The result can differ from the sequential visit: a token turned
+ * away by a full rank competes for its next choice one round later.
+ *
+ *   rounds  int32 [1] device, out (may be NULL): rounds that placed a token
+ *   other arguments as md_token_shuffle; the workspace is
+ *   md_token_shuffle_rounds_workspace_size bytes.
+ *   All ceil(T/1024) CTAs of the assignment must be resident at once
+ *   (cooperative launch): larger T returns MD_ERR_UNSUPPORTED.  Its grid
+ *   barriers are bounded waits (MD_ERR_TIMEOUT).
+ */
+size_t md_token_shuffle_rounds_workspace_size(int64_t T, int E, int R);
+
+int md_token_shuffle_rounds(const int32_t *idx_l, int k, const uint32_t *C,
+                            const int32_t *expert_to_rank_next, int64_t T, int E, int R,
+                            int32_t *pred_rank, int32_t *perm, int32_t *inv, int32_t *rounds,
+                            void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                            void *stream);
+
+/*
  * md_token_shuffle_pair -- md_token_shuffle with the pair-based prediction
  * and its single-expert fallback ("Expert Coupling ...", Method 2,
  * Prediction: a pair-based lookup over the two preceding layers, falling

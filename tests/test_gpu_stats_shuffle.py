@@ -245,3 +245,48 @@ def test_placement_outside_the_compact_path(kind, refine_mode, seed_mode):
                               refine_mode)
     torch.cuda.synchronize()
     assert np.array_equal(p.cpu().numpy(), oracle.place_two_level(W, R, 1, seed_mode, refine_mode))
+
+
+# ------------------------------------------------ rounds-based assignment
+def _rounds_both(a, C, p, R):
+    pred, perm, inv, rounds = md.md_token_shuffle_rounds(
+        i32(a), torch.from_numpy(C.view(np.int32)).to(DEV), i32(p), R)
+    torch.cuda.synchronize()
+    return ((pred.cpu().numpy(), perm.cpu().numpy(), inv.cpu().numpy(), int(rounds.item())),
+            oracle.token_shuffle_rounds(a, C, p, R))
+
+
+@pytest.mark.parametrize("name,T,R", [("two_layer_e128_k6", 8192, 16), ("two_layer_e128_k6", 4096, 4),
+                                      ("full_e256_k8", 8192, 64), ("iid_e64_k6", 16 * 37, 16),
+                                      ("two_layer_e128_k6", 65536, 16)])
+def test_rounds_match_oracle(name, T, R):
+    w, a, b = _two_layer(name, T)
+    _, C = oracle.coselect(a, b, w.E, T_fit=min(T, 4096))
+    C[5, :] = 0
+    p = shuffled_placement(w.E, R, 4)
+    got, want = _rounds_both(a, C, p, R)
+    for g, o in zip(got, want):
+        assert np.array_equal(g, o)
+
+
+@pytest.mark.parametrize("E,k,R,T", [(64, 2, 64, 64 * 40), (128, 6, 16, 16 * 700), (1024, 8, 64, 64 * 80),
+                                     (32, 1, 4, 4 * 1000), (16, 3, 2, 2 * 2500)])
+def test_rounds_skewed_counts(E, k, R, T):
+    rng = np.random.default_rng(E + R)
+    C = rng.integers(0, 3, size=(E, E)).astype(np.uint32)
+    hot = rng.choice(E, size=max(1, E // 16), replace=False)
+    C[:, hot] += 40
+    C[rng.choice(E, size=max(1, E // 10), replace=False), :] = 0
+    a = oracle.route_topk(synth.normal_f32(T, E, 3, 7).numpy(), k)[0]
+    p = shuffled_placement(E, R, 9)
+    got, want = _rounds_both(a, C, p, R)
+    for g, o in zip(got, want):
+        assert np.array_equal(g, o)
+
+
+def test_rounds_hand_example():
+    C = np.array([[10, 0, 0, 0], [6, 3, 1, 0], [1, 5, 4, 0], [2, 2, 0, 3]], np.uint32)
+    p = np.array([0, 1, 2, 2], np.int32)
+    a = np.array([[0], [0], [1], [2], [2], [3]], np.int32)
+    got, want = _rounds_both(a, C, p, 3)
+    assert got[0].tolist() == [0, 0, 2, 1, 1, 2] and got[3] == 2
