@@ -777,19 +777,36 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *p)
     return v;
 }
 
+__device__ __forceinline__ unsigned atom_add_acq_rel_u32(unsigned *p, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void atom_add_release_u32(unsigned *p, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_relaxed_u32(unsigned *p, unsigned v)
+{
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // All CTAs of the (cooperative, hence co-resident) grid meet here; false if
-// a wait ran out somewhere.
+// a wait ran out somewhere.  The block barrier before thread 0's release
+// (and after its acquire) carries every thread's global writes across.
 __device__ bool grid_barrier(RoundWs rw, unsigned n_ctas, int32_t *status)
 {
     __shared__ int s_ok;
     __syncthreads();
     if (threadIdx.x == 0) {
         const unsigned gen = ld_acquire_u32(rw.bar + 1);
-        __threadfence();
-        if (atomicAdd(rw.bar, 1u) + 1u == n_ctas) {
-            atomicExch(rw.bar, 0u);
-            __threadfence();
-            atomicAdd(rw.bar + 1, 1u);
+        if (atom_add_acq_rel_u32(rw.bar, 1u) + 1u == n_ctas) {
+            st_relaxed_u32(rw.bar, 0u);          // ordered before the release below
+            atom_add_release_u32(rw.bar + 1, 1u);
         } else {
             long long n = 0;
             while (ld_acquire_u32(rw.bar + 1) == gen) {
@@ -798,10 +815,9 @@ __device__ bool grid_barrier(RoundWs rw, unsigned n_ctas, int32_t *status)
                     atomicExch(rw.abort, 1);
                     break;
                 }
-                __nanosleep(64);
+                if ((n & 63) == 0) __nanosleep(32);
             }
         }
-        __threadfence();
         s_ok = *(volatile int32_t *)rw.abort == 0;
     }
     __syncthreads();
@@ -818,6 +834,8 @@ __global__ void __launch_bounds__(kRoundThreads)
     __shared__ short s_key[kTile];            // its top-1 expert, or -1 for an empty row
     __shared__ signed char s_prop[kTile];     // this round's proposal (-1: none)
     __shared__ unsigned char s_done[kTile];   // placed in an earlier round
+    __shared__ short s_rank[kTile];           // place among its warp's proposers of its rank
+    __shared__ int s_wcnt[kRoundThreads / 32][MD_MAX_RANKS];  // proposals per warp and rank
     __shared__ int s_cnt[MD_MAX_RANKS], s_rem[MD_MAX_RANKS], s_base[MD_MAX_RANKS], s_tot[MD_MAX_RANKS];
     __shared__ unsigned long long s_full;
     __shared__ int s_any;
@@ -908,20 +926,35 @@ __global__ void __launch_bounds__(kRoundThreads)
         }
         __syncthreads();
         if (!s_any) break;  // every token placed (the same on every CTA)
-        if (wp == 0) {
-            for (int c0 = 0; c0 < kTile; c0 += 32) {
-                const int i = c0 + lane;
-                const int d = s_prop[i];
-                const unsigned g = __match_any_sync(0xffffffffu, d >= 0 ? (unsigned)d : (0x80000000u | lane));
-                int within = 0;
-                if (d >= 0) within = s_cnt[d] + __popc(g & md::lanemask_lt());
-                __syncwarp();
-                if (d >= 0 && (g & md::lanemask_lt()) == 0u) s_cnt[d] += __popc(g);
-                __syncwarp();
-                if (d >= 0 && s_base[d] + within < s_rem[d]) {
-                    pred[s_tok[i]] = d;
-                    s_done[i] = 1;
-                }
+        // warp w ranks positions [w*128, w*128+128) in order; then a prefix
+        // over the warps per rank gives each proposer its place in the tile
+        constexpr int kPerWarp = kTile / (kRoundThreads / 32);
+        for (int d = lane; d < R; d += 32) s_wcnt[wp][d] = 0;
+        __syncwarp();
+        for (int c0 = wp * kPerWarp; c0 < (wp + 1) * kPerWarp; c0 += 32) {
+            const int i = c0 + lane;
+            const int d = s_prop[i];
+            const unsigned g = __match_any_sync(0xffffffffu, d >= 0 ? (unsigned)d : (0x80000000u | lane));
+            if (d >= 0) s_rank[i] = (short)(s_wcnt[wp][d] + __popc(g & md::lanemask_lt()));
+            __syncwarp();
+            if (d >= 0 && (g & md::lanemask_lt()) == 0u) s_wcnt[wp][d] += __popc(g);
+            __syncwarp();
+        }
+        __syncthreads();
+        for (int d = tid; d < R; d += kRoundThreads) {
+            int run = 0;
+            for (int w2 = 0; w2 < kRoundThreads / 32; ++w2) {
+                const int c = s_wcnt[w2][d];
+                s_wcnt[w2][d] = run;
+                run += c;
+            }
+        }
+        __syncthreads();
+        for (int i = tid; i < kTile; i += kRoundThreads) {
+            const int d = s_prop[i];
+            if (d >= 0 && s_base[d] + s_wcnt[i / kPerWarp][d] + s_rank[i] < s_rem[d]) {
+                pred[s_tok[i]] = d;
+                s_done[i] = 1;
             }
         }
         if (tile == 0) {
