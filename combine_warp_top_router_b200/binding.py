@@ -526,6 +526,7 @@ def md_token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_ob
     if idx_prev.shape != idx_l.shape:
         raise ValueError("idx_prev and idx_l differ in shape")
     _room(C2, "C2", E * E * E)
+    need = int(lib().md_token_shuffle_pair_workspace_size(T, E, R))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
     rc = lib().md_token_shuffle_pair(_ptr(idx_prev), _ptr(idx_l), k, _ptr(C), _ptr(C2),
