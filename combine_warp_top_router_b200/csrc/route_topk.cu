@@ -4,6 +4,10 @@
 // is routed to its top-k of E experts; Method 1: the routing probabilities
 // ride with the dispatched rows.
 //
+// Two kernels.  E in {64, 128, 256} with k in {1, 2, 4, 6, 8} (16-byte
+// aligned logits) takes k_route_topk_tpt, one thread per token (described
+// below it).  Every other shape takes k_route_topk:
+//
 // One warp per token.  Lane L holds M of the token's E logits as order-
 // preserving 32-bit keys (element index increases with the register slot);
 // keys compare exactly like the fp32 logits with -0.0 folded onto +0.0, and
@@ -239,6 +243,236 @@ void launch_k(const float *logits, int64_t T, int E, int k, int gate_mode, int32
     }
 }
 
+// ---------------------------------------------------------------- thread per token
+// E in {64, 128, 256}, k in {1, 2, 4, 6, 8}: one thread per token, so the
+// selection needs no cross-lane steps.  A warp stages its 32 consecutive rows
+// (contiguous in memory) in shared memory with 16-byte async copies.  Lane L
+// reads its row's 16-byte chunks in the order (c + L) mod E/4, which puts the
+// 8 lanes of a shared-memory phase on distinct banks.
+//   1. Threshold.  Chunk iteration c belongs to group c mod 16; the k-th
+//      largest of the 16 group maxima is at or below the k-th largest logit
+//      (k group maxima are k distinct elements at or above it).
+//   2. Candidates.  Elements at or above the threshold (about 10 for k = 8)
+//      are compacted into a per-lane list of expert indices.
+//   3. Selection.  Candidates become exact 64-bit keys (order-preserving
+//      logit key, then the complement of the expert index, so that equal
+//      logits go to the lower index).  Batches of 8 are sorted by a 19-
+//      comparator network and merged into the running sorted top 8: the
+//      pairwise maxima of two sorted lists, one reversed, are the union's top 8
+//      as a bitonic sequence, which a 12-comparator bitonic merge sorts.
+// The gates are computed as in the warp kernel, one token per thread.
+constexpr int kTptGroups = 16;
+
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(md::smem_addr(dst_smem)), "l"(src)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// descending compare-exchange
+__device__ __forceinline__ void cx(uint64_t &a, uint64_t &b)
+{
+    const uint64_t hi = a > b ? a : b;
+    b = a > b ? b : a;
+    a = hi;
+}
+
+__device__ __forceinline__ void cx(float &a, float &b)
+{
+    const float hi = fmaxf(a, b);
+    b = fminf(a, b);
+    a = hi;
+}
+
+// Batcher's odd-even merge sort of 8, descending
+template <typename V>
+__device__ __forceinline__ void sort8(V (&a)[8])
+{
+    cx(a[0], a[1]); cx(a[2], a[3]); cx(a[4], a[5]); cx(a[6], a[7]);
+    cx(a[0], a[2]); cx(a[1], a[3]); cx(a[4], a[6]); cx(a[5], a[7]);
+    cx(a[1], a[2]); cx(a[5], a[6]); cx(a[0], a[4]); cx(a[3], a[7]);
+    cx(a[1], a[5]); cx(a[2], a[6]);
+    cx(a[1], a[4]); cx(a[3], a[6]);
+    cx(a[2], a[4]); cx(a[3], a[5]);
+    cx(a[3], a[4]);
+}
+
+// sorts a bitonic sequence of 8, descending
+__device__ __forceinline__ void bitonic8(uint64_t (&a)[8])
+{
+#pragma unroll
+    for (int d = 4; d >= 1; d >>= 1)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if ((i & d) == 0) cx(a[i], a[i + d]);
+}
+
+__device__ __forceinline__ uint64_t cand_key(float v, int e)
+{
+    return ((uint64_t)float_key(v) << 32) | (uint64_t)(0xffffu - (uint32_t)e);
+}
+
+template <int E>
+constexpr size_t tpt_smem() { return (size_t)32 * E * 4 + (size_t)32 * E; }
+
+// One warp per CTA, one tile of 32 consecutive tokens (one per lane).
+template <int E, int KC>
+__global__ void __launch_bounds__(32)
+    k_route_topk_tpt(const float *__restrict__ logits, int64_t T, int gate_mode,
+                     int32_t *__restrict__ out_idx, float *__restrict__ out_w, int vec_out)
+{
+    constexpr int NCH = E / 4;
+    constexpr int NG = kTptGroups;
+    static_assert(KC >= 1 && KC <= 8 && NCH >= NG && (NCH & (NCH - 1)) == 0, "shape");
+    extern __shared__ __align__(16) unsigned char smem[];
+    float *rows = reinterpret_cast<float *>(smem);                      // [32][E]
+    const int lane = threadIdx.x;
+    uint8_t *lst = smem + (size_t)32 * E * 4 + lane;                    // slot s at lst[32 s]
+    const int64_t t0 = (int64_t)blockIdx.x * 32;
+    const int ntok = (int)(T - t0 < 32 ? T - t0 : 32);
+    {
+        const float4 *src = reinterpret_cast<const float4 *>(logits + t0 * E);
+        float4 *dst = reinterpret_cast<float4 *>(rows);
+        for (int i = lane; i < ntok * NCH; i += 32) cp_async16(dst + i, src + i);
+        cp_async_wait_all();
+        __syncwarp();
+    }
+    const bool live = lane < ntok;
+    const float *row = rows + lane * E;
+    const float4 *row4 = reinterpret_cast<const float4 *>(row);
+
+    // 1-2. threshold and candidate list
+    int n = 0;
+    if (live) {
+        float gm[NG];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const float4 q = row4[(c + lane) & (NCH - 1)];
+            const float m = fmaxf(fmaxf(q.x, q.y), fmaxf(q.z, q.w));
+            gm[c % NG] = c < NG ? m : fmaxf(gm[c % NG], m);
+        }
+        float a[8], b[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            a[i] = gm[i];
+            b[i] = gm[8 + i];
+        }
+        sort8(a);
+        sort8(b);
+        // k-th largest of the union of two descending lists
+        float th = fmaxf(a[KC - 1], b[KC - 1]);
+#pragma unroll
+        for (int i = 1; i < KC; ++i) th = fmaxf(th, fminf(a[i - 1], b[KC - i - 1]));
+
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int ch = (c + lane) & (NCH - 1);
+            const float4 q = row4[ch];
+            const int e0 = ch * 4;
+            if (q.x >= th) { lst[32 * n] = (uint8_t)e0; ++n; }
+            if (q.y >= th) { lst[32 * n] = (uint8_t)(e0 + 1); ++n; }
+            if (q.z >= th) { lst[32 * n] = (uint8_t)(e0 + 2); ++n; }
+            if (q.w >= th) { lst[32 * n] = (uint8_t)(e0 + 3); ++n; }
+        }
+    }
+
+    // 3. sorted top 8 of the candidates, batches of 8
+    const int nmax = (int)__reduce_max_sync(0xffffffffu, (unsigned)n);
+    uint64_t best[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) best[i] = 0ull;
+    for (int s = 0; s < nmax; s += 8) {
+        uint64_t bt[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            uint64_t key = 0ull;  // below every logit's key
+            if (s + j < n) {
+                const int e = lst[32 * (s + j)];
+                key = cand_key(row[e], e);
+            }
+            bt[j] = key;
+        }
+        sort8(bt);
+        if (s == 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) best[i] = bt[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) best[i] = best[i] > bt[7 - i] ? best[i] : bt[7 - i];
+            bitonic8(best);
+        }
+    }
+    if (!live) return;
+
+    const int64_t t = t0 + lane;
+    int sel[KC];
+    double ex[KC];
+    const double m = (double)key_float((uint32_t)(best[0] >> 32));
+    double den = 0.0;
+#pragma unroll
+    for (int r = 0; r < KC; ++r) {
+        sel[r] = (int)(0xffffu - (uint32_t)(best[r] & 0xffffffffu));
+        ex[r] = exp((double)key_float((uint32_t)(best[r] >> 32)) - m);
+        den += ex[r];
+    }
+    if (gate_mode == MD_GATE_FULL_SOFTMAX) {
+        den = 0.0;
+#pragma unroll 4
+        for (int c = 0; c < NCH; ++c) {
+            const float4 q = row4[(c + lane) & (NCH - 1)];
+            den += exp((double)q.x - m) + exp((double)q.y - m) + exp((double)q.z - m) +
+                   exp((double)q.w - m);
+        }
+    }
+    float w[KC];
+#pragma unroll
+    for (int r = 0; r < KC; ++r) w[r] = (float)(ex[r] / den);
+    if (vec_out && KC % 4 == 0) {
+#pragma unroll
+        for (int q = 0; q < KC / 4; ++q) {
+            reinterpret_cast<int4 *>(out_idx + t * KC)[q] =
+                make_int4(sel[4 * q], sel[4 * q + 1], sel[4 * q + 2], sel[4 * q + 3]);
+            reinterpret_cast<float4 *>(out_w + t * KC)[q] =
+                make_float4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < KC; ++r) {
+            out_idx[t * KC + r] = sel[r];
+            out_w[t * KC + r] = w[r];
+        }
+    }
+}
+
+template <int E, int KC>
+void launch_tpt(const float *logits, int64_t T, int gate_mode, int32_t *idx, float *w, cudaStream_t s)
+{
+    static std::atomic<uint64_t> attr_done{0};
+    md::once_per_device(attr_done, [] {
+        cudaFuncSetAttribute(k_route_topk_tpt<E, KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tpt_smem<E>());
+    });
+    const int vec = md::aligned16(idx) && md::aligned16(w);
+    const int64_t blocks = (T + 31) / 32;
+    k_route_topk_tpt<E, KC><<<(unsigned)blocks, 32, tpt_smem<E>(), s>>>(logits, T, gate_mode, idx, w, vec);
+    md::count_launches(1);
+}
+
+template <int E>
+bool try_tpt(const float *logits, int64_t T, int k, int gate_mode, int32_t *idx, float *w, cudaStream_t s)
+{
+    switch (k) {
+    case 1: launch_tpt<E, 1>(logits, T, gate_mode, idx, w, s); return true;
+    case 2: launch_tpt<E, 2>(logits, T, gate_mode, idx, w, s); return true;
+    case 4: launch_tpt<E, 4>(logits, T, gate_mode, idx, w, s); return true;
+    case 6: launch_tpt<E, 6>(logits, T, gate_mode, idx, w, s); return true;
+    case 8: launch_tpt<E, 8>(logits, T, gate_mode, idx, w, s); return true;
+    default: return false;
+    }
+}
+
 }  // namespace
 
 extern "C" int md_route_topk(const float *logits, int64_t T, int E, int k, int gate_mode,
@@ -250,6 +484,13 @@ extern "C" int md_route_topk(const float *logits, int64_t T, int E, int k, int g
     if (T == 0) return MD_OK;
     if (!logits || !topk_idx || !topk_w) return MD_ERR_ARG;
     cudaStream_t s = md::as_stream(stream);
+    if (md::aligned16(logits)) {
+        bool done = false;
+        if (E == 64) done = try_tpt<64>(logits, T, k, gate_mode, topk_idx, topk_w, s);
+        else if (E == 128) done = try_tpt<128>(logits, T, k, gate_mode, topk_idx, topk_w, s);
+        else if (E == 256) done = try_tpt<256>(logits, T, k, gate_mode, topk_idx, topk_w, s);
+        if (done) return md::launch_status();
+    }
     const bool vec = (E % 128 == 0) && md::aligned16(logits);
     if (vec) {
         switch (E / 128) {

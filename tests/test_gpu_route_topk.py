@@ -58,6 +58,42 @@ def test_ties_and_signed_zero(E):
         _compare(lg, k, 0)
 
 
+@pytest.mark.parametrize("E", [64, 128, 256])
+@pytest.mark.parametrize("k", [1, 2, 4, 6, 8])
+def test_per_token_kernel_ties_and_many_candidates(E, k):
+    # E in {64, 128, 256} with k <= 8 takes the one-thread-per-token kernel.
+    # Integer logits tie heavily, so many tokens have far more than 16
+    # candidates at or above the threshold (several batches of 8); rows of
+    # equal logits leave every element a candidate.  T = 32*13 + 7 leaves a
+    # ragged last warp.
+    rng = np.random.default_rng(100 * E + k)
+    T = 32 * 13 + 7
+    lg = rng.integers(-3, 2, size=(T, E)).astype(np.float32)
+    lg[rng.random(lg.shape) < 0.1] = -0.0
+    lg[1] = 1.0
+    lg[2] = -np.inf
+    lg[2, E - 1] = 0.0
+    lg[3] = rng.standard_normal(E).astype(np.float32)
+    for mode in (0, 1):
+        _compare(lg, k, mode)
+
+
+@pytest.mark.parametrize("E,k", [(128, 8), (64, 6), (256, 4)])
+def test_per_token_kernel_unaligned_outputs(E, k):
+    T = 100
+    lg_np = synth.normal_f32(T, E, 5, 1).numpy()
+    lg = torch.from_numpy(lg_np).to(DEV)
+    raw_i = torch.full((T * k + 1,), -9, dtype=torch.int32, device=DEV)
+    raw_w = torch.full((T * k + 1,), -9.0, dtype=torch.float32, device=DEV)
+    idx, w = md.md_route_topk(lg, k, 0, topk_idx=raw_i[1:].view(T, k),
+                            topk_w=raw_w[1:].view(T, k))
+    torch.cuda.synchronize()
+    oi, ow = oracle.route_topk(lg_np, k, 0)
+    assert np.array_equal(idx.cpu().numpy(), oi)
+    assert np.allclose(w.cpu().numpy(), ow, rtol=1e-6, atol=0)
+    assert int(raw_i[0].item()) == -9 and float(raw_w[0].item()) == -9.0
+
+
 def test_k1_gate_is_one_and_empty_batch():
     lg = synth.normal_f32(100, 64, 3, 1).numpy()
     _, w = _compare(lg, 1, 0)
