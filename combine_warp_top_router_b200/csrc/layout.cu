@@ -9,44 +9,45 @@
 // dispatcher sends one row per distinct (token, destination rank) pair.
 //
 // Rows are stable-sorted buckets: conventional rows by (p[e], e, t), dedup
-// rows by (d, t).  Two kernels, one thread per token, the token's k experts in
-// registers (k is a template parameter for the common values):
-//   k_layout_hist  bucket totals (assignments per expert, the send matrix)
-//                  in shared-memory histograms, flushed to the workspace.
-//   k_layout_rank  one tile of tokens per CTA, tiles in atomic-ticket order.
-//                  Every CTA turns the totals into bucket bases.  Inside the
-//                  tile, each warp marks which of its lanes hit each bucket
-//                  (a 32-bit set per bucket, built with shared atomicOr), so a
-//                  pair's rank among the warp's earlier tokens is a popcount.
-//                  The CTA publishes its bucket counts and gets the counts of
-//                  all earlier tiles by a single-pass decoupled lookback with
-//                  bounded waits; rows are staged in shared memory in bucket
-//                  order and written out in runs.
+// rows by (d, t).  One cooperative kernel, k_layout, one token per thread
+// (the token's k experts in registers; k is a template parameter for the
+// common values).  CTA c owns a contiguous run of 512-token tiles.
+//   A. Every CTA counts its tokens per bucket (shared-memory histograms) and
+//      the send-matrix rows of the source ranks it covers, writes them to the
+//      workspace and stamps its arrival word with this call's epoch.
+//   B. After every stamp is seen (a bounded wait), each CTA reads the count
+//      table: bucket totals give the bucket bases, the counts of CTAs before
+//      it give its start inside each bucket.  Each CTA also sums a slice of
+//      the send matrix.
+//   C. Tile by tile, each warp marks which of its lanes hit each bucket (a
+//      32-bit set per bucket, built with shared atomicOr), so a pair's rank
+//      among the warp's earlier tokens is a popcount; rows are staged in
+//      shared memory in bucket order and written out in runs.
+// Nothing in the workspace has to start at zero: the arrival words are
+// compared with a per-call epoch, and every count is written before it is read.
 #include "common.cuh"
 
 namespace {
 
-constexpr int kHistThreads = 256;  // one token per thread
 constexpr int kRankThreads = 512;  // one token per thread
 constexpr int kRankWarps = kRankThreads / 32;
-constexpr int kStageRows = 4096;   // output rows a rank tile can stage
-constexpr int kLookBatch = 8;      // buckets a warp looks back on at once
-constexpr unsigned long long kFlagA = 1ull << 62;  // tile aggregate published
-constexpr unsigned long long kFlagP = 2ull << 62;  // tile inclusive prefix published
-constexpr unsigned long long kValMask = (1ull << 62) - 1;
+constexpr int kStageRows = 4096;   // output rows a tile can stage
+constexpr int kMaxCtas = 256;      // CTAs of one launch; the workspace is sized for it
 constexpr long long kPollLimit = 1ll << 22;
 
+std::atomic<unsigned long long> g_epoch{0};
+
 struct Ws {
-    long long poll_limit;         // bound of every lookback wait
-    int skip_tile;                // test hook: this tile publishes nothing (-1: none)
-    unsigned int *ctrl;           // [0] rank tile ticket
-    int *hist_e;                  // [E]   assignments per expert
-    int *send;                    // [R*R] rows per (source, destination)
-    unsigned long long *tiles;    // [NB][n_tiles] lookback words, bucket-major
+    long long poll_limit;         // bound of the arrival wait
+    int skip_cta;                 // test hook: this CTA never stamps its arrival (-1: none)
+    unsigned long long epoch;     // this call's stamp
+    unsigned long long *flags;    // [kMaxCtas] arrival words
+    int *cnt;                     // [NB][kMaxCtas] bucket counts per CTA
+    int *part;                    // [(kMaxCtas + R) * R] send rows: CTA c, source s at row c + s
 };
 
-// tokens per rank tile: one per thread, fewer when k is large so that the
-// tile's rows fit the staging area
+// tokens per tile: one per thread, fewer when k is large so that the tile's
+// rows fit the staging area
 int tile_tokens(int k)
 {
     if (k <= kStageRows / kRankThreads) return kRankThreads;
@@ -56,7 +57,7 @@ int tile_tokens(int k)
 }
 
 struct Plan {
-    size_t off_hist, off_send, off_tiles, total;
+    size_t off_flags, off_cnt, off_part, total;
     int tile_tok, n_tiles, nb;
 };
 
@@ -65,16 +66,16 @@ Plan plan(int64_t T, int E, int k, int R, int mode)
     Plan p;
     p.tile_tok = tile_tokens(k);
     p.n_tiles = (int)((T + p.tile_tok - 1) / p.tile_tok);
-    if (p.n_tiles < 1) p.n_tiles = 1;  // tile 0 also writes the count outputs
+    if (p.n_tiles < 1) p.n_tiles = 1;  // CTA 0 also writes the count outputs
     p.nb = E + (mode == MD_DEDUP ? R : 0);
-    size_t o = 256;
-    p.off_hist = o;
-    o += md::align_up((size_t)E * 4, 256);
-    p.off_send = o;
-    o += md::align_up((size_t)R * R * 4, 256);
-    p.off_tiles = o;
-    o += md::align_up((size_t)p.n_tiles * p.nb * 8, 256);
-    p.total = o;  // all of it must start at zero
+    size_t o = 0;
+    p.off_flags = o;
+    o += md::align_up((size_t)kMaxCtas * 8, 256);
+    p.off_cnt = o;
+    o += md::align_up((size_t)kMaxCtas * p.nb * 4, 256);
+    p.off_part = o;
+    o += md::align_up((size_t)(kMaxCtas + R) * R * 4, 256);
+    p.total = o;
     return p;
 }
 
@@ -83,12 +84,24 @@ Ws carve(void *ws, const Plan &p)
     char *b = static_cast<char *>(ws);
     Ws w;
     w.poll_limit = md::hook_poll_limit(kPollLimit);
-    w.skip_tile = md::hook_layout_skip_tile();
-    w.ctrl = reinterpret_cast<unsigned int *>(b);
-    w.hist_e = reinterpret_cast<int *>(b + p.off_hist);
-    w.send = reinterpret_cast<int *>(b + p.off_send);
-    w.tiles = reinterpret_cast<unsigned long long *>(b + p.off_tiles);
+    w.skip_cta = md::hook_layout_skip_tile();
+    w.epoch = g_epoch.fetch_add(1) + 1;
+    w.flags = reinterpret_cast<unsigned long long *>(b + p.off_flags);
+    w.cnt = reinterpret_cast<int *>(b + p.off_cnt);
+    w.part = reinterpret_cast<int *>(b + p.off_part);
     return w;
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ int warp_incl_scan(int v, int lane)
@@ -101,102 +114,6 @@ __device__ __forceinline__ int warp_incl_scan(int v, int lane)
     return v;
 }
 
-// Clear the workspace (counters, totals, lookback words) and the status word.
-__global__ void __launch_bounds__(256) k_layout_zero(uint4 *__restrict__ ws, size_t n16,
-                                                     int32_t *status)
-{
-    for (size_t i = (size_t)blockIdx.x * 256 + threadIdx.x; i < n16; i += (size_t)gridDim.x * 256)
-        ws[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = MD_OK;
-    asm volatile("griddepcontrol.launch_dependents;");
-}
-
-// --------------------------------------------------------------- totals
-// KC > 0: the token's k experts live in registers (k known at compile time);
-// KC = 0: they are staged in shared memory with an odd row stride.
-template <int KC>
-__global__ void __launch_bounds__(kHistThreads, 2)
-    k_layout_hist(const int32_t *__restrict__ idx, int64_t T, int E, int k, int R,
-                  const int32_t *__restrict__ p_g, int mode, Ws ws, int32_t *status)
-{
-    extern __shared__ int smem[];
-    int *s_p = smem;             // [E]
-    int *s_hist = s_p + E;       // [E]
-    int *s_send = s_hist + E;    // [R*R]
-    int *s_idx = s_send + R * R; // [kHistThreads * (k | 1)]  (KC == 0 only)
-
-    const int K = KC ? KC : k;
-    const int tid = threadIdx.x;
-    for (int e = tid; e < E; e += kHistThreads) {
-        s_p[e] = p_g[e];
-        s_hist[e] = 0;
-    }
-    for (int i = tid; i < R * R; i += kHistThreads) s_send[i] = 0;
-    const int64_t Tr = T / R;
-    const int64_t t0 = (int64_t)blockIdx.x * kHistThreads;
-    const bool have = t0 + tid < T;
-    const int64_t t = have ? t0 + tid : t0;
-    int reg[KC ? KC : 1];
-    const int ks = K | 1;
-    if (KC) {
-#pragma unroll
-        for (int j = 0; j < (KC ? KC : 1); ++j) reg[j] = have ? __ldg(idx + t * K + j) : -1;
-    } else {
-        for (int j = 0; j < K; ++j) s_idx[tid * ks + j] = have ? __ldg(idx + t * K + j) : -1;
-    }
-    // the loads above overlap the clearing kernel; status and workspace are
-    // touched only after it has completed
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    __syncthreads();
-    auto ex = [&](int j) -> int { return KC ? reg[j] : s_idx[tid * ks + j]; };
-
-    // rank of every slot, looked up once (-1: invalid expert or placement)
-    int dr[KC ? KC : 1];
-    if (KC) {
-#pragma unroll
-        for (int j = 0; j < (KC ? KC : 1); ++j) {
-            const int e = ex(j);
-            int d = (e >= 0 && e < E) ? s_p[e] : -1;
-            dr[j] = (d >= 0 && d < R) ? d : -1;
-        }
-    }
-    auto rk = [&](int j) -> int {
-        if (KC) return dr[j];
-        const int e = ex(j);
-        const int d = (e >= 0 && e < E) ? s_p[e] : -1;
-        return (d >= 0 && d < R) ? d : -1;
-    };
-
-    // shared-memory histograms
-    const int src = (int)(t / Tr);
-#pragma unroll
-    for (int j = 0; j < (KC ? KC : MD_MAX_TOPK); ++j) {
-        if (!KC && j >= K) break;
-        int e = ex(j);
-        int d = rk(j);
-        if (have && d < 0) md::report(status, MD_ERR_DATA);
-        if (d < 0) e = -1;
-        bool rep = true;
-#pragma unroll
-        for (int j2 = 0; j2 < (KC ? KC : MD_MAX_TOPK); ++j2) {
-            if (j2 >= j) break;
-            if (e >= 0 && ex(j2) == e) md::report(status, MD_ERR_DATA);  // expert twice in one token
-            if (rk(j2) == d) rep = false;
-        }
-        if (e >= 0) {
-            atomicAdd(&s_hist[e], 1);
-            if (mode == MD_CONV || rep) atomicAdd(&s_send[src * R + d], 1);
-        }
-    }
-    asm volatile("griddepcontrol.launch_dependents;");
-    __syncthreads();
-    for (int e = tid; e < E; e += kHistThreads)
-        if (s_hist[e]) atomicAdd(&ws.hist_e[e], s_hist[e]);
-    for (int i = tid; i < R * R; i += kHistThreads)
-        if (s_send[i]) atomicAdd(&ws.send[i], s_send[i]);
-}
-
-// --------------------------------------------------------------- ranks
 // A token's k outputs are contiguous: vector stores where k allows.
 template <int KC>
 __device__ __forceinline__ void store_row(int32_t *dst, const int (&v)[KC ? KC : MD_MAX_TOPK], int K)
@@ -220,84 +137,187 @@ __device__ __forceinline__ void store_row(int32_t *dst, const int (&v)[KC ? KC :
 
 template <int KC>
 __global__ void __launch_bounds__(kRankThreads, 1)
-    k_layout_rank(const int32_t *__restrict__ idx, int64_t T, int E, int k, int R,
-                  const int32_t *__restrict__ p_g, int mode, int tile_tok, Ws ws,
-                  int32_t *__restrict__ row_of_slot, int32_t *__restrict__ assign_row,
-                  int32_t *__restrict__ row_token, uint32_t *__restrict__ row_mask,
-                  int64_t row_cap, int32_t *__restrict__ expert_counts,
-                  int32_t *__restrict__ send_counts, int32_t *__restrict__ expert_offsets,
-                  int32_t *__restrict__ rank_offsets, int32_t *__restrict__ n_rows,
-                  int32_t *status)
+    k_layout(const int32_t *__restrict__ idx, int64_t T, int E, int k, int R,
+             const int32_t *__restrict__ p_g, int mode, int tile_tok, int n_tiles, int tpc, Ws ws,
+             int32_t *__restrict__ row_of_slot, int32_t *__restrict__ assign_row,
+             int32_t *__restrict__ row_token, uint32_t *__restrict__ row_mask, int64_t row_cap,
+             int32_t *__restrict__ expert_counts, int32_t *__restrict__ send_counts,
+             int32_t *__restrict__ expert_offsets, int32_t *__restrict__ rank_offsets,
+             int32_t *__restrict__ n_rows, int32_t *status)
 {
     constexpr int KM = KC ? KC : MD_MAX_TOPK;
     const int K = KC ? KC : k;
     extern __shared__ int smem[];
     const bool dedup = mode == MD_DEDUP;
     const int NB = E + (dedup ? R : 0);
-    const int n_tiles = gridDim.x;
+    const int G = gridDim.x, cta = blockIdx.x;
     int *s_p = smem;                        // [E] placement
-    int *s_he = s_p + E;                    // [E] assignments per expert (all tiles)
+    int *s_he = s_p + E;                    // [E] assignments per expert (all CTAs)
     int *s_base = s_he + E;                 // [NB] first row of each bucket
-    int *s_pref = s_base + NB;              // [NB] tile total, then first row of the tile
-    int *s_toff = s_pref + NB;              // [NB] tile-local start of each output bucket
+    int *s_run = s_base + NB;               // [NB] this CTA's next row in each bucket
+    int *s_tcnt = s_run + NB;               // [NB] bucket totals, then the tile's bucket counts
+    int *s_toff = s_tcnt + NB;              // [NB] tile-local start of each output bucket
     int *s_cnt = s_toff + NB;               // [16][NB] rows of earlier warps in the tile
     unsigned *s_bits = reinterpret_cast<unsigned *>(s_cnt + kRankWarps * NB);  // [16][NB]
     int *s_otok = reinterpret_cast<int *>(s_bits + kRankWarps * NB);           // [kStageRows]
     int *s_omsk = s_otok + kStageRows;
     int *s_opos = s_omsk + kStageRows;
     int *s_cs = s_opos + kStageRows;        // [E/32][R] per chunk and rank: sum, then start
+    int *s_acnt = s_cnt;                    // phase A: [NB] this CTA's bucket counts
+    int *s_send = s_otok;                   // phase A: [R*R] this CTA's send counts
     __shared__ int s_rt[2][MD_MAX_RANKS + 1];  // rank totals -> offsets: conventional, dedup
     __shared__ int s_per_rank[MD_MAX_RANKS];
-    __shared__ int s_tile, s_timeout, s_nrows;
+    __shared__ int s_timeout, s_nrows;
 
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-    if (tid == 0) {
-        s_tile = (int)atomicAdd(&ws.ctrl[0], 1u);
-        s_timeout = 0;
-    }
+    const int tile_lo = cta * tpc;
+    const int tile_hi = tile_lo + tpc < n_tiles ? tile_lo + tpc : n_tiles;
+    const int64_t Tr = R > 0 && T > 0 ? T / R : 1;
+    // the status word is cleared before this CTA stamps its arrival, and every
+    // report comes after the arrival wait
+    if (cta == 0 && tid == 0 && status) *status = MD_OK;
+    if (tid == 0) s_timeout = 0;
     for (int e = tid; e < E; e += kRankThreads) s_p[e] = p_g[e];
+    for (int i = tid; i < NB; i += kRankThreads) s_acnt[i] = 0;
+    for (int i = tid; i < R * R; i += kRankThreads) s_send[i] = 0;
     for (int i = tid; i < 2 * (MD_MAX_RANKS + 1); i += kRankThreads) (&s_rt[0][0])[i] = 0;
     for (int d = tid; d < R; d += kRankThreads) s_per_rank[d] = 0;
-    for (int i = tid; i < kRankWarps * NB; i += kRankThreads) s_bits[i] = 0u;
     for (int i = tid; i < ((E + 31) >> 5) * R; i += kRankThreads) s_cs[i] = 0;
-    __syncthreads();
-    const int tile = s_tile;
-    const int64_t t0 = (int64_t)tile * tile_tok;
-    const bool have = tid < tile_tok && t0 + tid < T;
-    const int64_t t = t0 + tid;
-
-    // the token's experts: issued now, used after the bucket bases
-    int e[KM];
+    // the first tile's experts: used in A and again in C
+    int e0[KM];
+    {
+        const int64_t t = (int64_t)tile_lo * tile_tok + tid;
+        const bool have = tile_lo < tile_hi && tid < tile_tok && t < T;
 #pragma unroll
-    for (int j = 0; j < KM; ++j)
-        if (KC || j < K) e[j] = have ? __ldg(idx + t * K + j) : -1;
+        for (int j = 0; j < KM; ++j)
+            if (KC || j < K) e0[j] = have ? __ldg(idx + t * K + j) : -1;
+    }
+    // tokens t_first .. t_last; when they all come from one source rank, its
+    // send row follows from the bucket counts
+    const int64_t t_first = (int64_t)tile_lo * tile_tok;
+    const int64_t t_last = ((int64_t)tile_hi * tile_tok < T ? (int64_t)tile_hi * tile_tok : T) - 1;
+    const int s_lo = t_first <= t_last ? (int)(t_first / Tr) : 0;
+    const int s_hi = t_first <= t_last ? (int)(t_last / Tr) : -1;
+    const bool one_src = s_lo == s_hi;
+    __syncthreads();
 
-    // everything above overlaps the histogram kernel (programmatic dependent
-    // launch); its totals are read only after it has completed
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // ---- A. bucket counts and send rows of this CTA's tokens
+    bool bad = false;
+    for (int tile = tile_lo; tile < tile_hi; ++tile) {
+        const int64_t t = (int64_t)tile * tile_tok + tid;
+        if (tid >= tile_tok || t >= T) continue;
+        int e[KM], d[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            if (KC || j < K) e[j] = tile == tile_lo ? e0[j] : __ldg(idx + t * K + j);
+        const int src = (int)(t / Tr);
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            if (!KC && j >= K) break;
+            int ee = e[j];
+            int dd = (ee >= 0 && ee < E) ? s_p[ee] : -1;
+            if (dd >= R) dd = -1;
+            if (dd < 0) { bad = true; ee = -1; }
+            e[j] = ee;
+            d[j] = dd;
+            bool rep = true;  // the token's first slot on rank dd
+#pragma unroll
+            for (int j2 = 0; j2 < KM; ++j2) {
+                if (j2 >= j) break;
+                if (ee >= 0 && e[j2] == ee) bad = true;  // expert twice in one token
+                if (d[j2] == dd) rep = false;
+            }
+            if (ee >= 0) {
+                atomicAdd(&s_acnt[ee], 1);
+                if (dedup && rep) atomicAdd(&s_acnt[E + dd], 1);
+                if (!one_src && (!dedup || rep)) atomicAdd(&s_send[src * R + dd], 1);
+            }
+        }
+    }
+    __syncthreads();
+    if (one_src) {
+        if (dedup) {
+            for (int dd = tid; dd < R; dd += kRankThreads) s_send[s_lo * R + dd] = s_acnt[E + dd];
+        } else {
+            for (int x = tid; x < E; x += kRankThreads) {
+                const int dd = s_p[x];
+                if (dd >= 0 && dd < R && s_acnt[x]) atomicAdd(&s_send[s_lo * R + dd], s_acnt[x]);
+            }
+        }
+        __syncthreads();
+    }
+    for (int b = tid; b < NB; b += kRankThreads) ws.cnt[(size_t)b * kMaxCtas + cta] = s_acnt[b];
+    for (int i = tid; i < (s_hi - s_lo + 1) * R; i += kRankThreads) {
+        const int s = s_lo + i / R, dd = i % R;
+        ws.part[(size_t)(cta + s) * R + dd] = s_send[s * R + dd];
+    }
+    __syncthreads();
+    if (tid == 0 && cta != ws.skip_cta) st_release_u64(ws.flags + cta, ws.epoch);
+    // every CTA's counts are in once its stamp carries this call's epoch
+    if (tid < G) {
+        long long polls = 0;
+        while (ld_acquire_u64(ws.flags + tid) != ws.epoch) {
+            if (++polls > ws.poll_limit) {
+                s_timeout = 1;
+                break;
+            }
+            if (polls > 32) __nanosleep(32);
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    if (s_timeout) {  // positions unknown: leave outputs, status says why
+        if (tid == 0) md::report(status, MD_ERR_TIMEOUT);
+        return;
+    }
+    if (bad) md::report(status, MD_ERR_DATA);
 
-    // ---- bucket bases from the totals (every CTA; tile 0 also writes them out).
-    // Conventional order is (p[e], e): per 32-expert chunk and rank, the sum of
-    // the chunk's experts on that rank; a scan over chunks per rank; then a
-    // prefix among the chunk's own lanes.  All totals are loaded in one round.
+    // ---- B. bucket totals and this CTA's start in each bucket: a bucket's
+    // counts of all CTAs are contiguous, one warp reads them in one pass, for
+    // 4 buckets at a time
+    for (int b0 = w * 4; b0 < NB; b0 += kRankWarps * 4) {
+        int v[4][kMaxCtas / 32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int i = 0; i < kMaxCtas / 32; ++i) {
+                const int c2 = lane + 32 * i;
+                v[q][i] = b0 + q < NB && c2 < G ? __ldcg(ws.cnt + (size_t)(b0 + q) * kMaxCtas + c2) : 0;
+            }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            int tot = 0, pre = 0;
+#pragma unroll
+            for (int i = 0; i < kMaxCtas / 32; ++i) {
+                tot += v[q][i];
+                pre += lane + 32 * i < cta ? v[q][i] : 0;
+            }
+            tot = (int)__reduce_add_sync(0xffffffffu, (unsigned)tot);
+            pre = (int)__reduce_add_sync(0xffffffffu, (unsigned)pre);
+            if (lane == 0 && b0 + q < NB) {
+                s_tcnt[b0 + q] = tot;
+                s_run[b0 + q] = pre;
+            }
+        }
+    }
+    __syncthreads();
+
+    // bucket bases from the totals.  Conventional order is (p[e], e): per
+    // 32-expert chunk and rank, the sum of the chunk's experts on that rank; a
+    // scan over chunks per rank; then a prefix among the chunk's own lanes.
     for (int x = tid; x < E; x += kRankThreads) {
-        const int he = __ldcg(ws.hist_e + x);
+        const int he = s_tcnt[x];
         s_he[x] = he;
         const int d = s_p[x];
         if (d >= 0 && d < R) {
             atomicAdd(&s_cs[(x >> 5) * R + d], he);
             atomicAdd(&s_per_rank[d], 1);
-        } else if (tile == 0) {
+        } else if (cta == 0) {
             md::report(status, MD_ERR_DATA);
         }
     }
-    if (dedup)  // column sums of the send matrix: one warp per destination
-        for (int dd = w; dd < R; dd += kRankWarps) {
-            const int a = __ldcg(ws.send + lane * R + dd);
-            const int b = lane + 32 < R ? __ldcg(ws.send + (lane + 32) * R + dd) : 0;
-            const int sum = (int)__reduce_add_sync(0xffffffffu, (unsigned)((lane < R ? a : 0) + b));
-            if (lane == 0) s_rt[1][dd] = sum;
-        }
+    if (dedup)
+        for (int dd = tid; dd < R; dd += kRankThreads) s_rt[1][dd] = s_tcnt[E + dd];
     __syncthreads();
     const int nchunk = (E + 31) >> 5;
     for (int dd = tid; dd < R; dd += kRankThreads) {  // rank totals (conventional)
@@ -348,12 +368,12 @@ __global__ void __launch_bounds__(kRankThreads, 1)
     if (dedup)
         for (int dd = tid; dd < R; dd += kRankThreads) s_base[E + dd] = s_rt[1][dd];
     __syncthreads();
-    if (tile == 0) {
+    for (int b = tid; b < NB; b += kRankThreads) s_run[b] += s_base[b];
+    if (cta == 0) {
         for (int x = tid; x < E; x += kRankThreads) {
             expert_counts[x] = s_he[x];
             expert_offsets[x] = s_base[x];
         }
-        for (int i = tid; i < R * R; i += kRankThreads) send_counts[i] = __ldcg(ws.send + i);
         for (int d = tid; d <= R; d += kRankThreads) rank_offsets[d] = s_rt[1][d];
         for (int d = tid; d < R; d += kRankThreads)
             if (s_per_rank[d] != E / R) md::report(status, MD_ERR_DATA);
@@ -362,224 +382,167 @@ __global__ void __launch_bounds__(kRankThreads, 1)
             *n_rows = s_rt[1][R];
         }
     }
-
-    // ---- per-token: ranks, which slot carries each dedup row, row masks
-    int d[KM];
-    int jr[KM];
-    unsigned msk[KM];
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        if (!KC && j >= K) break;
-        int ee = e[j];
-        int dd = (ee >= 0 && ee < E) ? s_p[ee] : -1;
-        if (dd >= R) dd = -1;
-        if (dd < 0) ee = -1;
-        e[j] = ee;
-        d[j] = dd;
+    // a slice of the send matrix: source s was counted by the CTAs that own
+    // tokens s*T/R .. (s+1)*T/R - 1
+    for (int i = cta * kRankThreads + tid; i < R * R; i += G * kRankThreads) {
+        int sum = 0;
+        if (T > 0) {
+            const int s = i / R, dd = i % R;
+            const int c_lo = (int)((int64_t)s * Tr / tile_tok) / tpc;
+            const int c_hi = (int)(((int64_t)s + 1) * Tr - 1) / tile_tok / tpc;
+            for (int c2 = c_lo; c2 <= c_hi; ++c2) sum += __ldcg(ws.part + (size_t)(c2 + s) * R + dd);
+        }
+        send_counts[i] = sum;
     }
-    if (dedup) {
+    __syncthreads();
+
+    // ---- C. rows, tile by tile
+    const unsigned lt = md::lanemask_lt();
+    unsigned *wb = s_bits + w * NB;
+    const int *wc = s_cnt + w * NB;
+    const int ob0 = dedup ? E : 0;
+    for (int tile = tile_lo; tile < tile_hi; ++tile) {
+        for (int i = tid; i < kRankWarps * NB; i += kRankThreads) s_bits[i] = 0u;
+        const int64_t t = (int64_t)tile * tile_tok + tid;
+        const bool have = tid < tile_tok && t < T;
+        int e[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            if (KC || j < K) e[j] = e0[j];
+        if (tile + 1 < tile_hi) {  // the next tile's experts load while this one is ranked
+            const int64_t tn = t + tile_tok;
+            const bool hn = tid < tile_tok && tn < T;
+#pragma unroll
+            for (int j = 0; j < KM; ++j)
+                if (KC || j < K) e0[j] = hn ? __ldg(idx + tn * K + j) : -1;
+        }
+        __syncthreads();
+
+        // per-token: ranks, which slot carries each dedup row, row masks
+        int d[KM];
+        int jr[KM];
+        unsigned msk[KM];
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
             if (!KC && j >= K) break;
-            jr[j] = j;
-            msk[j] = 0u;
+            int ee = e[j];
+            int dd = (ee >= 0 && ee < E) ? s_p[ee] : -1;
+            if (dd >= R) dd = -1;
+            if (dd < 0) ee = -1;
+            e[j] = ee;
+            d[j] = dd;
+        }
+        if (dedup) {
 #pragma unroll
-            for (int j2 = KM - 1; j2 >= 0; --j2) {
-                if (j2 >= K) continue;
-                if (d[j2] == d[j] && j2 < j) jr[j] = j2;
-                if (d[j2] == d[j]) msk[j] |= 1u << j2;
+            for (int j = 0; j < KM; ++j) {
+                if (!KC && j >= K) break;
+                jr[j] = j;
+                msk[j] = 0u;
+#pragma unroll
+                for (int j2 = KM - 1; j2 >= 0; --j2) {
+                    if (j2 >= K) continue;
+                    if (d[j2] == d[j] && j2 < j) jr[j] = j2;
+                    if (d[j2] == d[j]) msk[j] |= 1u << j2;
+                }
             }
         }
-    }
-    // mark this lane in the bucket sets of its warp
-    unsigned *wb = s_bits + w * NB;
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        if (!KC && j >= K) break;
-        if (d[j] < 0) continue;
-        atomicOr(wb + e[j], 1u << lane);
-        if (dedup && jr[j] == j) atomicOr(wb + E + d[j], 1u << lane);
-    }
-    __syncthreads();
-
-    // ---- per-bucket tile totals and rows of earlier warps; the totals are
-    // published at once so that later tiles can start their lookback
-    for (int b = tid; b < NB; b += kRankThreads) {
-        int run = 0;
-#pragma unroll
-        for (int w2 = 0; w2 < kRankWarps; ++w2) {
-            const int c = __popc(s_bits[w2 * NB + b]);
-            s_cnt[w2 * NB + b] = run;
-            run += c;
-        }
-        s_pref[b] = run;
-        if (tile != ws.skip_tile)
-            md::st_relaxed_u64(ws.tiles + (size_t)b * n_tiles + tile,
-                               (tile == 0 ? kFlagP : kFlagA) | (unsigned long long)run);
-    }
-    __syncthreads();
-    // tile-local start of each output bucket (the mode's buckets, in order)
-    const int ob0 = dedup ? E : 0;
-    if (w == 0) {
-        int run = 0;
-        for (int b0 = ob0; b0 < NB; b0 += 32) {
-            const int b = b0 + lane;
-            const int c = b < NB ? s_pref[b] : 0;
-            const int incl = warp_incl_scan(c, lane);
-            if (b < NB) s_toff[b] = run + incl - c;
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) s_nrows = run;
-    }
-    __syncthreads();
-
-    // ---- tile-local ranks (bucket << 16 | rank inside the tile's bucket run);
-    // output rows are staged in shared memory in bucket order
-    const unsigned lt = md::lanemask_lt();
-    const int *wc = s_cnt + w * NB;
-    int ar[KM], rs[KM];
-#pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        if (!KC && j >= K) break;
-        ar[j] = -1;
-        rs[j] = -1;
-        if (d[j] < 0) continue;
-        const int x = e[j];
-        const int within = wc[x] + __popc(wb[x] & lt);
-        ar[j] = (x << 16) | within;
-        if (!dedup) {
-            rs[j] = ar[j];
-            const int o = s_toff[x] + within;
-            s_otok[o] = (int)t;
-            s_omsk[o] = (int)(1u << j);
-            s_opos[o] = ar[j];
-        } else if (jr[j] == j) {  // first slot of this token on rank d: owns the row
-            const int b = E + d[j];
-            const int wd = wc[b] + __popc(wb[b] & lt);
-            rs[j] = (b << 16) | wd;
-            const int o = s_toff[b] + wd;
-            s_otok[o] = (int)t;
-            s_omsk[o] = (int)msk[j];
-            s_opos[o] = rs[j];
-        }
-    }
-    if (dedup) {  // every slot takes the row of its rank's first slot
+        // mark this lane in the bucket sets of its warp
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
             if (!KC && j >= K) break;
             if (d[j] < 0) continue;
-            int r = rs[j];
-#pragma unroll
-            for (int j2 = 0; j2 < KM; ++j2)
-                if (j2 < j && jr[j] == j2) r = rs[j2];
-            rs[j] = r;
+            atomicOr(wb + e[j], 1u << lane);
+            if (dedup && jr[j] == j) atomicOr(wb + E + d[j], 1u << lane);
         }
-    }
+        __syncthreads();
 
-    // ---- decoupled lookback over earlier tiles.  The words of one bucket are
-    // contiguous over tiles.  A warp keeps up to kLookBatch buckets in flight
-    // and moves all their windows back together: lane L reads tiles top-2L and
-    // top-2L-1, so one round of loads covers 64 earlier tiles of every bucket
-    // in the batch.  Counts fit 31 bits, so window sums are one warp reduce.
-    for (int b0 = w; b0 < NB; b0 += kRankWarps * kLookBatch) {
-        int excl[kLookBatch];
-        unsigned pending = 0;  // bit q: bucket b0 + 16 q still looking back
+        // per-bucket tile counts and rows of earlier warps
+        for (int b = tid; b < NB; b += kRankThreads) {
+            int run = 0;
 #pragma unroll
-        for (int q = 0; q < kLookBatch; ++q) {
-            excl[q] = 0;
-            if (tile > 0 && b0 + q * kRankWarps < NB) pending |= 1u << q;
-        }
-        int top = tile - 1;
-        long long polls = 0;
-        while (pending) {
-            unsigned long long v[kLookBatch][2];
-#pragma unroll
-            for (int q = 0; q < kLookBatch; ++q) {
-                const unsigned long long *col = ws.tiles + (size_t)(b0 + q * kRankWarps) * n_tiles;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int j = top - 2 * lane - u;
-                    v[q][u] = ((pending >> q) & 1u) && j >= 0 ? md::ld_relaxed_u64(col + j) : kFlagP;
-                }
+            for (int w2 = 0; w2 < kRankWarps; ++w2) {
+                const int c = __popc(s_bits[w2 * NB + b]);
+                s_cnt[w2 * NB + b] = run;
+                run += c;
             }
-#pragma unroll
-            for (int q = 0; q < kLookBatch; ++q) {
-                if (!((pending >> q) & 1u)) continue;
-                const unsigned long long *col = ws.tiles + (size_t)(b0 + q * kRankWarps) * n_tiles;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    // a word not yet published: bounded wait
-                    while ((v[q][u] >> 62) == 0ull) {
-                        if (++polls > ws.poll_limit) {
-                            md::report(status, MD_ERR_TIMEOUT);
-                            s_timeout = 1;
-                            v[q][u] = kFlagP;
-                            break;
-                        }
-                        __nanosleep(64);
-                        v[q][u] = md::ld_relaxed_u64(col + (top - 2 * lane - u));
-                    }
-                }
-                // nearest inclusive prefix: lane order, then u order
-                const int fp = (v[q][0] >> 62) == 2ull ? 0 : ((v[q][1] >> 62) == 2ull ? 1 : 2);
-                const unsigned pm = __ballot_sync(0xffffffffu, fp < 2);
-                const int stop = pm ? __ffs(pm) - 1 : 32;
-                unsigned part = 0;
-                if (lane < stop) {
-                    part = (unsigned)(v[q][0] & kValMask) + (unsigned)(v[q][1] & kValMask);
-                } else if (lane == stop) {
-                    part = (unsigned)(v[q][0] & kValMask) +
-                           (fp == 1 ? (unsigned)(v[q][1] & kValMask) : 0u);
-                }
-                excl[q] += (int)__reduce_add_sync(0xffffffffu, part);
-                if (pm) pending &= ~(1u << q);
-            }
-            top -= 64;
+            s_tcnt[b] = run;
         }
-#pragma unroll
-        for (int q = 0; q < kLookBatch; ++q) {
-            const int b = b0 + q * kRankWarps;
-            if (b < NB && lane == 0) {
-                if (tile > 0 && tile != ws.skip_tile)
-                    md::st_relaxed_u64(ws.tiles + (size_t)b * n_tiles + tile,
-                                       kFlagP | (unsigned long long)(excl[q] + s_pref[b]));
-                s_pref[b] = s_base[b] + excl[q];
+        __syncthreads();
+        // tile-local start of each output bucket (the mode's buckets, in order)
+        if (w == 0) {
+            int run = 0;
+            for (int b0 = ob0; b0 < NB; b0 += 32) {
+                const int b = b0 + lane;
+                const int c = b < NB ? s_tcnt[b] : 0;
+                const int incl = warp_incl_scan(c, lane);
+                if (b < NB) s_toff[b] = run + incl - c;
+                run += __shfl_sync(0xffffffffu, incl, 31);
             }
+            if (lane == 0) s_nrows = run;
         }
-    }
-    __syncthreads();
-    if (s_timeout) return;  // positions unknown: leave outputs, status says why
+        __syncthreads();
 
-    // ---- global rows: the tile's start in the bucket + the tile-local rank
+        // global rows: this CTA's next row in the bucket + the rank inside the
+        // tile; output rows are staged in shared memory in bucket order
+        int ar[KM], rs[KM];
 #pragma unroll
-    for (int j = 0; j < KM; ++j) {
-        if (!KC && j >= K) break;
-        if (ar[j] >= 0) ar[j] = s_pref[ar[j] >> 16] + (ar[j] & 0xffff);
-        if (rs[j] >= 0) rs[j] = s_pref[rs[j] >> 16] + (rs[j] & 0xffff);
-    }
-    if (have) store_row<KC>(assign_row + t * K, ar, K), store_row<KC>(row_of_slot + t * K, rs, K);
-    for (int o = tid; o < s_nrows; o += kRankThreads) {
-        const int pk = s_opos[o];
-        const int pos = s_pref[pk >> 16] + (pk & 0xffff);
-        if (pos >= 0 && pos < row_cap) {
-            row_token[pos] = s_otok[o];
-            row_mask[pos] = (uint32_t)s_omsk[o];
-        } else {
-            md::report(status, MD_ERR_DATA);
+        for (int j = 0; j < KM; ++j) {
+            if (!KC && j >= K) break;
+            ar[j] = -1;
+            rs[j] = -1;
+            if (d[j] < 0) continue;
+            const int x = e[j];
+            const int within = wc[x] + __popc(wb[x] & lt);
+            ar[j] = s_run[x] + within;
+            if (!dedup) {
+                rs[j] = ar[j];
+                const int o = s_toff[x] + within;
+                s_otok[o] = (int)t;
+                s_omsk[o] = (int)(1u << j);
+                s_opos[o] = ar[j];
+            } else if (jr[j] == j) {  // first slot of this token on rank d: owns the row
+                const int b = E + d[j];
+                const int wd = wc[b] + __popc(wb[b] & lt);
+                rs[j] = s_run[b] + wd;
+                const int o = s_toff[b] + wd;
+                s_otok[o] = (int)t;
+                s_omsk[o] = (int)msk[j];
+                s_opos[o] = rs[j];
+            }
         }
+        if (dedup) {  // every slot takes the row of its rank's first slot
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                if (!KC && j >= K) break;
+                if (d[j] < 0) continue;
+                int r = rs[j];
+#pragma unroll
+                for (int j2 = 0; j2 < KM; ++j2)
+                    if (j2 < j && jr[j] == j2) r = rs[j2];
+                rs[j] = r;
+            }
+        }
+        if (have) store_row<KC>(assign_row + t * K, ar, K), store_row<KC>(row_of_slot + t * K, rs, K);
+        __syncthreads();
+        for (int o = tid; o < s_nrows; o += kRankThreads) {
+            const int pos = s_opos[o];
+            if (pos >= 0 && pos < row_cap) {
+                row_token[pos] = s_otok[o];
+                row_mask[pos] = (uint32_t)s_omsk[o];
+            } else {
+                md::report(status, MD_ERR_DATA);
+            }
+        }
+        for (int b = tid; b < NB; b += kRankThreads) s_run[b] += s_tcnt[b];
+        __syncthreads();
     }
 }
 
-size_t rank_smem(int E, int R, int mode)
+size_t layout_smem(int E, int R, int mode)
 {
     const int NB = E + (mode == MD_DEDUP ? R : 0);
-    return (size_t)(2 * E + (2 * kRankWarps + 3) * NB + 3 * kStageRows + ((E + 31) / 32) * R) *
+    return (size_t)(2 * E + (2 * kRankWarps + 4) * NB + 3 * kStageRows + ((E + 31) / 32) * R) *
            sizeof(int);
-}
-
-size_t hist_smem(int E, int k, int R)
-{
-    return (size_t)(2 * E + R * R + kHistThreads * (k | 1)) * sizeof(int);
 }
 
 int check_layout_args(int64_t T, int E, int k, int R, int mode)
@@ -592,46 +555,65 @@ int check_layout_args(int64_t T, int E, int k, int R, int mode)
     return MD_OK;
 }
 
+constexpr size_t kLayoutSmemMax = (size_t)(2 * 1024 + (2 * kRankWarps + 4) * (1024 + 64) +
+                                           3 * kStageRows + 32 * 64) * sizeof(int);
+
+// CTAs of k_layout<KC> resident per SM with the largest shared-memory size
+// (set once per device)
 template <int KC>
-void set_attrs()
+int layout_per_sm()
 {
-    cudaFuncSetAttribute(k_layout_rank<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-    cudaFuncSetAttribute(k_layout_hist<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize, 100 * 1024);
+    static std::atomic<uint64_t> done{0};
+    static int per_sm[64];
+    md::once_per_device(done, [] {
+        int dev = 0, nb = 0;
+        cudaGetDevice(&dev);
+        if (cudaFuncSetAttribute(k_layout<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kLayoutSmemMax) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_layout<KC>, kRankThreads,
+                                                          kLayoutSmemMax) != cudaSuccess) {
+            cudaGetLastError();
+            nb = 0;
+        }
+        per_sm[dev & 63] = nb;
+    });
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return per_sm[dev & 63];
 }
 
 template <int KC>
-void launch_layout(const int32_t *topk_idx, int64_t T, int E, int k, int R,
-                   const int32_t *expert_to_rank, int mode, const Plan &pl, const Ws &ws,
-                   int32_t *row_of_slot, int32_t *assign_row, int32_t *row_token,
-                   uint32_t *row_mask, int64_t cap, int32_t *send_counts,
-                   int32_t *expert_counts, int32_t *expert_offsets, int32_t *rank_offsets,
-                   int32_t *n_rows, int32_t *dev_status, cudaStream_t s)
+int launch_layout(const int32_t *topk_idx, int64_t T, int E, int k, int R,
+                  const int32_t *expert_to_rank, int mode, const Plan &pl, const Ws &ws,
+                  int32_t *row_of_slot, int32_t *assign_row, int32_t *row_token,
+                  uint32_t *row_mask, int64_t cap, int32_t *send_counts, int32_t *expert_counts,
+                  int32_t *expert_offsets, int32_t *rank_offsets, int32_t *n_rows,
+                  int32_t *dev_status, cudaStream_t s)
 {
-    // each kernel may start while the previous one drains (programmatic
-    // dependent launch); it waits (griddepcontrol.wait) before using its results
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t hc = {};
-    hc.gridDim = dim3((unsigned)(T > 0 ? (T + kHistThreads - 1) / kHistThreads : 1));
-    hc.blockDim = dim3(kHistThreads);
-    hc.dynamicSmemBytes = hist_smem(E, k, R);
-    hc.stream = s;
-    hc.attrs = attr;
-    hc.numAttrs = 1;
-    cudaLaunchKernelEx(&hc, k_layout_hist<KC>, topk_idx, T, E, k, R, expert_to_rank, mode, ws,
-                       dev_status);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)pl.n_tiles);
-    cfg.blockDim = dim3(kRankThreads);
-    cfg.dynamicSmemBytes = rank_smem(E, R, mode);
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, k_layout_rank<KC>, topk_idx, T, E, k, R, expert_to_rank, mode,
-                       pl.tile_tok, ws, row_of_slot, assign_row, row_token, row_mask, cap,
-                       expert_counts, send_counts, expert_offsets, rank_offsets, n_rows,
-                       dev_status);
+    const size_t smem = layout_smem(E, R, mode);
+    const int per_sm = layout_per_sm<KC>();
+    if (per_sm < 1 || smem > kLayoutSmemMax) return MD_ERR_UNSUPPORTED;
+    // every CTA waits for all the others: the grid must be resident at once
+    int resident = md::sm_count() * per_sm;
+    if (resident > kMaxCtas) resident = kMaxCtas;
+    const int tpc = (pl.n_tiles + resident - 1) / resident;
+    const int G = (pl.n_tiles + tpc - 1) / tpc;
+    int tile_tok = pl.tile_tok, n_tiles = pl.n_tiles, mode_ = mode, k_ = k, E_ = E, R_ = R;
+    int64_t T_ = T, cap_ = cap;
+    Ws ws_ = ws;
+    void *args[] = {(void *)&topk_idx, &T_,          &E_,         &k_,          &R_,
+                    (void *)&expert_to_rank, &mode_, &tile_tok,  &n_tiles,     (void *)&tpc,
+                    &ws_,        (void *)&row_of_slot, (void *)&assign_row, (void *)&row_token,
+                    (void *)&row_mask, &cap_, (void *)&expert_counts, (void *)&send_counts,
+                    (void *)&expert_offsets, (void *)&rank_offsets, (void *)&n_rows,
+                    (void *)&dev_status};
+    md::count_launches(1);
+    if (cudaLaunchCooperativeKernel((const void *)k_layout<KC>, dim3((unsigned)G), dim3(kRankThreads),
+                                    args, smem, s) != cudaSuccess) {
+        cudaGetLastError();
+        return MD_ERR_CUDA;
+    }
+    return MD_OK;
 }
 
 }  // namespace
@@ -661,31 +643,25 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
     if (!workspace || workspace_bytes < pl.total) return MD_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MD_ERR_ARG;
     cudaStream_t s = md::as_stream(stream);
-    const Ws ws = carve(workspace, pl);
-
-    static std::atomic<uint64_t> attr_done{0};
-    md::once_per_device(attr_done, [] {
-        set_attrs<0>();
-        set_attrs<1>();
-        set_attrs<2>();
-        set_attrs<4>();
-        set_attrs<6>();
-        set_attrs<8>();
-    });
-    {
-        const size_t n16 = pl.total / 16;
-        int zb = (int)((n16 + 255) / 256);
-        if (zb > md::sm_count()) zb = md::sm_count();
-        k_layout_zero<<<zb < 1 ? 1 : zb, 256, 0, s>>>(static_cast<uint4 *>(workspace), n16,
-                                                     dev_status);
+    Ws ws = carve(workspace, pl);
+    cudaStreamCaptureStatus cst = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cst) != cudaSuccess) {
+        cudaGetLastError();
+        cst = cudaStreamCaptureStatusNone;
+    }
+    if (cst == cudaStreamCaptureStatusActive) {
+        // a graph replays the launch with the same arguments: the arrival
+        // words are cleared inside the graph and the epoch is fixed
         md::count_launches(1);
+        if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 8, s) != cudaSuccess) return MD_ERR_CUDA;
+        ws.epoch = 1;
     }
 
     const int64_t cap = mode == MD_CONV ? T * k : T * (int64_t)(k < R ? k : R);
 #define MD_LAYOUT(KC)                                                                            \
-    launch_layout<KC>(topk_idx, T, E, k, R, expert_to_rank, mode, pl, ws, row_of_slot,          \
-                      assign_row, row_token, row_mask, cap, send_counts, expert_counts,         \
-                      expert_offsets, rank_offsets, n_rows, dev_status, s)
+    rc = launch_layout<KC>(topk_idx, T, E, k, R, expert_to_rank, mode, pl, ws, row_of_slot,     \
+                           assign_row, row_token, row_mask, cap, send_counts, expert_counts,    \
+                           expert_offsets, rank_offsets, n_rows, dev_status, s)
     // the specialised kernels store a token's k outputs as vectors
     const bool vec_ok = md::aligned16(assign_row) && md::aligned16(row_of_slot);
     switch (vec_ok ? k : 0) {
@@ -697,8 +673,7 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
     default: MD_LAYOUT(0); break;
     }
 #undef MD_LAYOUT
-    md::count_launches(2);
-    return md::launch_status();
+    return rc;
 }
 
 // ------------------------------------------------------------------------
@@ -756,8 +731,8 @@ extern "C" int md_dispatch_layout_noalloc(const int32_t *topk_idx, int64_t T, in
     if (plan(T, E, k, R, mode).total > kNoAllocScratchBytes) return MD_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     if ((rc = scratch_for_current_device(&scratch)) != MD_OK) return rc;
-    // The shared array keeps the previous call's contents; md_dispatch_layout
-    // clears the part that must start at zero on the stream before using it.
+    // The shared array keeps the previous call's contents; nothing in it has to
+    // start at zero (the arrival words are compared with a per-call epoch).
     return md_dispatch_layout(topk_idx, T, E, k, R, expert_to_rank, mode, row_of_slot, assign_row,
                               row_token, row_mask, send_counts, expert_counts, expert_offsets,
                               rank_offsets, n_rows, scratch, kNoAllocScratchBytes, dev_status,

@@ -130,7 +130,14 @@ int md_route_topk(const float *logits, int64_t T, int E, int k, int gate_mode,
  *   rank_offsets    int32 [R+1]    first row of rank d in this mode; [R] = n_rows
  *   n_rows          int32 [1]      rows in this mode (T*k for MD_CONV)
  *   workspace       >= md_dispatch_layout_workspace_size(...) bytes, 256-B
- *                   aligned; contents on entry do not matter.
+ *                   aligned; contents on entry do not matter.  The size does
+ *                   not grow with T (at most about 1.2 MiB, at E=1024, R=64).
+ *   One cooperative launch: all its CTAs (at most one per SM) must be
+ *   resident at once, so a GPU shared with a running kernel that holds SMs
+ *   may delay it; MD_ERR_CUDA if the launch is refused.  Every CTA waits for
+ *   the others' counts with a bounded wait (MD_ERR_TIMEOUT in dev_status if
+ *   it runs out; the outputs are then not written).  Safe in CUDA graph
+ *   capture: a capturing stream also records a clear of the arrival words.
  *   Limits: T % R == 0, E % R == 0, 1 <= k <= min(E, 32), E <= 1024,
  *   R <= 64, T*k < 2^31.
  */
@@ -157,16 +164,15 @@ int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int k, int R,
  * fixed array of MD_NOALLOC_LAYOUT_SCRATCH_BYTES (4 MiB) compiled into the
  * library, which every GPU that loads the library holds until the process
  * exits.  The caller still passes all inputs and outputs.
- *   - Problems whose workspace would exceed that size return
- *     MD_ERR_UNSUPPORTED (md_dispatch_layout_workspace_size tells the need;
- *     T=262144, E=256, k=8, R=64 dedup needs about 2.6 MiB).
+ *   - Every shape within md_dispatch_layout's limits fits: the workspace
+ *     does not grow with T and is at most about 1.2 MiB.
  *   - The first call on each device looks up the array's device address with
  *     cudaGetSymbolAddress (with that device current) and caches it; make
  *     that first call before any stream capture.
  *   - Every call on a device shares the one array, which keeps the previous
- *     call's contents; each call clears what must start at zero on its
- *     stream.  Calls that overlap on the GPU (other streams, other threads)
- *     race on it and must be serialised by the caller.
+ *     call's contents; nothing in it has to start at zero.  Calls that
+ *     overlap on the GPU (other streams, other threads) race on it and must
+ *     be serialised by the caller.
  *   - Results are identical to md_dispatch_layout's.
  */
 #define MD_NOALLOC_LAYOUT_SCRATCH_BYTES ((size_t)4 << 20)

@@ -48,3 +48,15 @@ def test_host_only_calls():
                               None) == binding.MD_ERR_ARG                    # T % R != 0
     assert L.md_dedup_expand(None, 0, 12, None, None, 4, 2, 8, None, None,
                              None) == binding.MD_ERR_ARG                     # H % 8 != 0
+
+
+def test_layout_workspace_does_not_grow_with_tokens():
+    # the layout's scratch is per CTA and per bucket, not per tile, so it is
+    # the same for every T and fits the no-alloc entry point's fixed array
+    L = binding.lib()
+    cap = L.md_dispatch_layout_noalloc_max_scratch()
+    for E, k, R, mode in ((128, 8, 16, 1), (256, 8, 64, 1), (1024, 32, 64, 1), (1024, 32, 64, 0)):
+        sizes = {L.md_dispatch_layout_workspace_size(T, E, k, R, mode)
+                 for T in (R, 64 * R, 1 << 16, 1 << 20, (1 << 26) // k)}
+        assert len(sizes) == 1
+        assert 0 < sizes.pop() <= cap

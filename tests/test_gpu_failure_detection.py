@@ -1,8 +1,8 @@
 """Failure detection without a GPU fault: every device-side wait is bounded.
 
-md_set_test_hooks shortens the poll limit and leaves one lookback publish (the
-dispatch layout) or one bulk-copy load (the dedup expand) out, so that a wait
-runs out.  The call must end with MD_ERR_TIMEOUT in its status word -- no
+md_set_test_hooks shortens the poll limit and leaves one CTA's arrival stamp
+(the dispatch layout) or one bulk-copy load (the dedup expand) out, so that a
+wait runs out.  The call must end with MD_ERR_TIMEOUT in its status word -- no
 trap, no hang -- and the next call, with the hooks cleared, must be exact."""
 import numpy as np
 import pytest
@@ -29,8 +29,8 @@ def _routes(T):
 
 
 @pytest.mark.parametrize("mode", [0, 1])
-def test_layout_lookback_wait_runs_out(hooks, mode):
-    w, idx = _routes(8192)                    # 16 tiles of 512 tokens
+def test_layout_arrival_wait_runs_out(hooks, mode):
+    w, idx = _routes(8192)                    # 16 tiles of 512 tokens, one per CTA
     p = w.expert_to_rank.numpy()
     hooks(poll_limit=4096, layout_skip_tile=0)
     st = md.new_status(DEV)

@@ -155,3 +155,45 @@ def test_layout_unaligned_outputs(mode):
     md.md_dispatch_layout(i32(idx), E, R, i32(p), mode, out=L)
     torch.cuda.synchronize()
     assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), T, k)
+
+
+def test_layout_replays_in_cuda_graph():
+    # A captured layout replays with new inputs: the capture also records the
+    # clear of the arrival words, so every replay waits for its own counts.
+    from combine_warp_top_router_b200 import binding
+    name, T, R, E, k = "zipf_pairs_e128_k8", 4096, 16, 128, 8
+    p = synth.contiguous_placement(E, R).numpy()
+    runs = [_routes(name, T, seed=s) for s in (0, 1, 2)]
+    static_idx = i32(runs[0])
+    pg = i32(p)
+    L = md.alloc_layout(T, E, k, R, 1, DEV)
+    ws = binding.alloc_workspace(binding.dispatch_layout_workspace_size(T, E, k, R, 1), DEV)
+    st = md.new_status(DEV)
+    md.md_dispatch_layout(static_idx, E, R, pg, 1, out=L, workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        md.md_dispatch_layout(static_idx, E, R, pg, 1, out=L, workspace=ws, dev_status=st)
+    for idx in (runs[1], runs[2], runs[0], runs[1]):
+        static_idx.copy_(torch.from_numpy(idx))
+        L.row_token.fill_(POISON)
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(st.item()) == md.MD_OK
+        assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, 1), T, k)
+    del g
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("T", [512 * 148 * 3 + 64, 512 * 300])
+def test_layout_several_tiles_per_cta(T, mode):
+    # more tiles than resident CTAs: each CTA walks a run of tiles and carries
+    # its bucket starts from one tile to the next (T = 512*148*3 + 64 leaves a
+    # short last tile; R = 8 divides both sizes)
+    E, k, R = 64, 6, 8
+    lg = synth.normal_f32(T, E, 21, 1).numpy()
+    idx = oracle.route_topk(lg, k)[0]
+    p = shuffled_placement(E, R, 9)
+    L, st = gpu_layout(idx, E, R, p, mode)
+    assert st == md.MD_OK
+    assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), T, k)

@@ -90,11 +90,19 @@ def test_noalloc_matches_workspace_entry_point_twice(name, T, mode):
         _same(got, want)
 
 
-def test_noalloc_rejects_sizes_beyond_its_scratch():
+def test_noalloc_takes_sizes_whose_old_scratch_need_was_larger():
+    # the workspace does not grow with T: a million tokens (E=256, k=8, R=64,
+    # about 5 MB of per-tile scratch in a per-tile lookback design) fits
+    T, E, k, R = 1 << 20, 256, 8, 64
     lib = binding.lib()
-    T, E, k, R = 1 << 21, 1024, 32, 64
-    assert lib.md_dispatch_layout_workspace_size(T, E, k, R, md.MD_DEDUP) > \
+    assert lib.md_dispatch_layout_workspace_size(T, E, k, R, md.MD_DEDUP) <= \
         lib.md_dispatch_layout_noalloc_max_scratch()
-    rc = lib.md_dispatch_layout_noalloc(None, T, E, k, R, None, md.MD_DEDUP, None, None, None,
-                                        None, None, None, None, None, None, None, None)
-    assert rc == md.MD_ERR_UNSUPPORTED
+    stream = torch.cuda.current_stream()
+    p = synth.contiguous_placement(E, R, DEV)
+    status = torch.full((1,), 77, dtype=torch.int32, device=DEV)
+    idx, _ = md.md_route_topk(synth.normal_f32(T, E, 5, 1, DEV), k)
+    got = _noalloc(idx, E, R, p, md.MD_DEDUP, status, stream)
+    want = _with_workspace(idx, E, R, p, md.MD_DEDUP, stream)
+    torch.cuda.synchronize()
+    assert int(status.item()) == md.MD_OK
+    _same(got, want)
