@@ -40,8 +40,8 @@ std::atomic<unsigned long long> g_epoch{0};
 struct Ws {
     long long poll_limit;         // bound of the arrival wait
     int skip_cta;                 // test hook: this CTA never stamps its arrival (-1: none)
-    unsigned long long epoch;     // this call's stamp
-    unsigned long long *flags;    // [kMaxCtas] arrival words
+    unsigned epoch;               // this call's stamp (never 0)
+    unsigned *flags;              // [kMaxCtas] arrival words
     int *cnt;                     // [NB][kMaxCtas] bucket counts per CTA
     int *part;                    // [(kMaxCtas + R) * R] send rows: CTA c, source s at row c + s
 };
@@ -70,7 +70,7 @@ Plan plan(int64_t T, int E, int k, int R, int mode)
     p.nb = E + (mode == MD_DEDUP ? R : 0);
     size_t o = 0;
     p.off_flags = o;
-    o += md::align_up((size_t)kMaxCtas * 8, 256);
+    o += md::align_up((size_t)kMaxCtas * 4, 256);
     p.off_cnt = o;
     o += md::align_up((size_t)kMaxCtas * p.nb * 4, 256);
     p.off_part = o;
@@ -85,23 +85,28 @@ Ws carve(void *ws, const Plan &p)
     Ws w;
     w.poll_limit = md::hook_poll_limit(kPollLimit);
     w.skip_cta = md::hook_layout_skip_tile();
-    w.epoch = g_epoch.fetch_add(1) + 1;
-    w.flags = reinterpret_cast<unsigned long long *>(b + p.off_flags);
+    do {
+        w.epoch = (unsigned)(g_epoch.fetch_add(1) + 1);
+    } while (w.epoch == 0u);
+    w.flags = reinterpret_cast<unsigned *>(b + p.off_flags);
     w.cnt = reinterpret_cast<int *>(b + p.off_cnt);
     w.part = reinterpret_cast<int *>(b + p.off_part);
     return w;
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p)
+__device__ __forceinline__ uint4 ld_relaxed_v4(const unsigned *p)
 {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    uint4 v;
+    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
     return v;
 }
 
-__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v)
+__device__ __forceinline__ void st_relaxed_u32(unsigned *p, unsigned v)
 {
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
 __device__ __forceinline__ int warp_incl_scan(int v, int lane)
@@ -252,16 +257,27 @@ __global__ void __launch_bounds__(kRankThreads, 1)
         ws.part[(size_t)(cta + s) * R + dd] = s_send[s * R + dd];
     }
     __syncthreads();
-    if (tid == 0 && cta != ws.skip_cta) st_release_u64(ws.flags + cta, ws.epoch);
-    // every CTA's counts are in once its stamp carries this call's epoch
-    if (tid < G) {
+    if (tid == 0 && cta != ws.skip_cta) {
+        __threadfence();
+        st_relaxed_u32(ws.flags + cta, ws.epoch);
+    }
+    // every CTA's counts are in once its stamp carries this call's epoch; one
+    // warp reads all stamps, four per 16-byte load
+    if (w == 0) {
         long long polls = 0;
-        while (ld_acquire_u64(ws.flags + tid) != ws.epoch) {
+        for (;;) {
+            bool ok = true;
+            for (int i = lane * 4; i < G; i += 128) {
+                const uint4 v = ld_relaxed_v4(ws.flags + i);
+                ok = ok && v.x == ws.epoch && (i + 1 >= G || v.y == ws.epoch) &&
+                     (i + 2 >= G || v.z == ws.epoch) && (i + 3 >= G || v.w == ws.epoch);
+            }
+            if (__all_sync(0xffffffffu, ok)) break;
             if (++polls > ws.poll_limit) {
-                s_timeout = 1;
+                if (lane == 0) s_timeout = 1;
                 break;
             }
-            if (polls > 32) __nanosleep(32);
+            if (polls > 16) __nanosleep(32);
         }
         __threadfence();
     }
@@ -382,9 +398,9 @@ __global__ void __launch_bounds__(kRankThreads, 1)
             *n_rows = s_rt[1][R];
         }
     }
-    // a slice of the send matrix: source s was counted by the CTAs that own
-    // tokens s*T/R .. (s+1)*T/R - 1
-    for (int i = cta * kRankThreads + tid; i < R * R; i += G * kRankThreads) {
+    // entries cta, cta + G, ... of the send matrix: source s was counted by the
+    // CTAs that own tokens s*T/R .. (s+1)*T/R - 1
+    for (int i = cta + G * tid; i < R * R; i += G * kRankThreads) {
         int sum = 0;
         if (T > 0) {
             const int s = i / R, dd = i % R;
@@ -653,7 +669,7 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
         // a graph replays the launch with the same arguments: the arrival
         // words are cleared inside the graph and the epoch is fixed
         md::count_launches(1);
-        if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 8, s) != cudaSuccess) return MD_ERR_CUDA;
+        if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 4, s) != cudaSuccess) return MD_ERR_CUDA;
         ws.epoch = 1;
     }
 
