@@ -80,19 +80,6 @@ __device__ __forceinline__ unsigned lanemask_lt()
     return m;
 }
 
-// Relaxed 64-bit loads / stores at GPU scope for cross-CTA flags.
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p)
-{
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v)
-{
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
 // 16-byte streaming load (read once) and store (written once).
 __device__ __forceinline__ uint4 ld_stream(const uint4 *p)
 {
