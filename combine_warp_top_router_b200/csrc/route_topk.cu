@@ -376,6 +376,12 @@ __global__ void __launch_bounds__(32)
             if (q.z >= th) { lst[32 * n] = (uint8_t)(e0 + 2); ++n; }
             if (q.w >= th) { lst[32 * n] = (uint8_t)(e0 + 3); ++n; }
         }
+        // fewer than k candidates happens only with NaN logits (outside the
+        // contract): take every element, so the indices stay valid and distinct
+        if (n < KC) {
+            for (int e = 0; e < E; ++e) lst[32 * e] = (uint8_t)e;
+            n = E;
+        }
     }
 
     // 3. sorted top 8 of the candidates, batches of 8

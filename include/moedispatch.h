@@ -88,7 +88,9 @@ uint64_t md_launch_count(void);
  * is routed to its top-k of E experts; Method 1: the routing probabilities
  * travel with the dispatched rows.
  *
- *   logits    float32 [T, E]   raw router logits (no NaN; -inf allowed)
+ *   logits    float32 [T, E]   raw router logits (no NaN; -inf allowed; with
+ *                              NaN the order is unspecified, but every token
+ *                              still gets k distinct experts in [0, E))
  *   topk_idx  int32   [T, k]   out: experts by logit descending; equal
  *                              logits (-0.0 == +0.0) by lower expert index
  *   topk_w    float32 [T, k]   out: gate weights.  MD_GATE_TOPK_SOFTMAX:

@@ -112,3 +112,24 @@ def test_full_size_sampled():
     oi, ow = oracle.route_topk(lg[rows], 8)
     assert np.array_equal(idx.cpu().numpy()[rows], oi)
     assert np.allclose(gw.cpu().numpy()[rows], ow, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("E,k", [(128, 8), (64, 6), (256, 2), (40, 5)])
+def test_nan_rows_give_valid_distinct_experts(E, k):
+    # NaN logits are outside the contract; the router must still return k
+    # distinct experts in [0, E) for every token, and the same ones each time
+    rng = np.random.default_rng(E + k)
+    T = 96
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    lg[0] = np.nan                                  # all NaN
+    lg[1, : E - k + 1] = np.nan                     # fewer than k numbers
+    lg[2, ::3] = np.nan                             # scattered NaN
+    lg[3] = -np.nan
+    gi, _ = _run(lg, k, 0)
+    gi2, _ = _run(lg, k, 0)
+    assert np.array_equal(gi, gi2)
+    assert gi.min() >= 0 and gi.max() < E
+    assert all(len(set(r)) == k for r in gi.tolist())
+    # rows without NaN are unaffected
+    oi, _ = oracle.route_topk(lg[4:], k, 0)
+    assert np.array_equal(gi[4:], oi)
