@@ -536,47 +536,75 @@ def run_rows(args, md, device, stream, peak):
 
 
 def run_e2e(args, md, w, mode, device, stream, idx, gates, L, wsp, buf, status, dist):
-    """Same step through host buffers: pinned inputs -> HBM, path, result -> host."""
+    """Same step through host buffers: pinned inputs -> HBM, path, result -> host.
+
+    Steps are pipelined over two device buffer sets, as a serving loop would
+    run them: the inputs of step i+1 copy in (one copy stream) while step i
+    computes and step i-1's result copies out (another copy stream).  Every
+    step still moves all of its own inputs in and its result out."""
     T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
     h_logits = w.logits.cpu().pin_memory()
     h_x = w.x.cpu().pin_memory()
     h_y = w.y.cpu().pin_memory()
-    h_out = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
-    d_logits = torch.empty_like(w.logits)
-    d_x = torch.empty_like(w.x)
-    d_y = torch.empty_like(w.y)
-    d_out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+    h_out = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    d_in = [(w.logits, w.x, w.y)] + [(torch.empty_like(w.logits), torch.empty_like(w.x),
+                                      torch.empty_like(w.y))]
+    d_out = [torch.empty(T, H, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    s_in = torch.cuda.Stream(device)
+    s_out = torch.cuda.Stream(device)
     steps = max(1, min(args.steps, args.e2e_steps))
+    ev = lambda: torch.cuda.Event()
+    in_done = [ev(), ev()]      # inputs of set b are in HBM
+    used = [ev(), ev()]         # the step on set b no longer reads its inputs
+    out_done = [ev(), ev()]     # the result of set b is on the host
 
-    def step():
-        d_logits.copy_(h_logits, non_blocking=True)
-        d_x.copy_(h_x, non_blocking=True)
-        d_y.copy_(h_y, non_blocking=True)
+    def step(i):
+        b = i % 2
+        d_logits, d_x, d_y = d_in[b]
+        s_in.wait_event(used[b])
+        with torch.cuda.stream(s_in):
+            d_logits.copy_(h_logits, non_blocking=True)
+            d_x.copy_(h_x, non_blocking=True)
+            d_y.copy_(h_y, non_blocking=True)
+        in_done[b].record(s_in)
+        stream.wait_event(in_done[b])
+        stream.wait_event(out_done[b])
         md.md_route_topk(d_logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream)
         md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp,
                               dev_status=status, stream=stream)
         md.md_dispatch_permute(d_x, L.row_of_slot, out=buf, stream=stream)
-        md.md_combine(d_y, L.assign_row, idx, gates, out=d_out, stream=stream)
-        h_out.copy_(d_out, non_blocking=True)
+        md.md_combine(d_y, L.assign_row, idx, gates, out=d_out[b], stream=stream)
+        used[b].record(stream)
+        s_out.wait_event(used[b])
+        with torch.cuda.stream(s_out):
+            h_out[b].copy_(d_out[b], non_blocking=True)
+        out_done[b].record(s_out)
 
-    with torch.cuda.stream(stream):
-        step()
-    stream.synchronize()
+    for e in used + out_done:
+        e.record(stream)
+    for i in range(2):
+        step(i)
+    torch.cuda.synchronize()
     barrier(dist, device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(steps):
-            step()
-        e1.record(stream)
-    stream.synchronize()
+    e0.record(s_in)
+    for i in range(steps):
+        step(i)
+    s_in.wait_stream(s_out)
+    s_in.wait_stream(stream)
+    e1.record(s_in)
+    torch.cuda.synchronize()
     ms = max_over_ranks(dist, e0.elapsed_time(e1), device)
+    # the last step's result is the step's own output
+    assert torch.equal(h_out[(steps - 1) % 2], d_out[(steps - 1) % 2].cpu())
     ws = dist.get_world_size() if dist is not None else 1
     h2d = (h_logits.numel() * 4 + h_x.numel() * 2 + h_y.numel() * 2)
     return {"value": round(T * steps * ws / (ms * 1e-3) / 1e6, 4), "unit": UNIT,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(h_out.numel() * 2),
-            "steps": steps, "note": "pinned host buffers; copies on the compute stream"}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(h_out[0].numel() * 2),
+            "steps": steps,
+            "note": "pinned host buffers; two device buffer sets, inputs of the next step "
+                    "copy in while the result of the previous one copies out"}
 
 
 # -------------------------------------------------------- oracle (CPU) arm
