@@ -11,7 +11,8 @@
 // Rows are stable-sorted buckets: conventional rows by (p[e], e, t), dedup
 // rows by (d, t).  One cooperative kernel, k_layout, one token per thread
 // (the token's k experts in registers; k is a template parameter for the
-// common values).  CTA c owns a contiguous run of 512-token tiles.
+// common values).  CTA c owns a contiguous run of tiles (512 tokens each,
+// fewer when k > 8).
 //   A. Every CTA counts its tokens per bucket (shared-memory histograms) and
 //      the send-matrix rows of the source ranks it covers, writes them to the
 //      workspace and stamps its arrival word with this call's epoch.
@@ -25,6 +26,8 @@
 //      shared memory in bucket order and written out in runs.
 // Nothing in the workspace has to start at zero: the arrival words are
 // compared with a per-call epoch, and every count is written before it is read.
+// A graph replays one epoch, so a capturing stream also records a clear of
+// the arrival words and the epoch is fixed at 1.
 #include "common.cuh"
 
 namespace {
