@@ -735,8 +735,9 @@ __global__ void __launch_bounds__(32)
 // launch: CTA c owns positions [c*1024, (c+1)*1024) of the priority order.
 // Phase 1 counts the tile's proposals per rank; after a grid barrier, phase
 // 2 places each proposer among the proposers of its rank (earlier tiles
-// first, then tile order, one warp with __match_any_sync) and accepts it if
-// that place is inside the remaining capacity; after a second barrier the
+// first, then tile order: each warp ranks its 128 positions with
+// __match_any_sync, then a prefix over the warps) and accepts it if that
+// place is inside the remaining capacity; after a second barrier the
 // next round starts.  At most R + 1 rounds.  The grid barrier waits are
 // bounded (MD_ERR_TIMEOUT, and every CTA then stops).
 constexpr int kRoundThreads = 256;
