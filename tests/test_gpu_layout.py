@@ -185,11 +185,13 @@ def test_layout_replays_in_cuda_graph():
 
 
 @pytest.mark.parametrize("mode", [0, 1])
-@pytest.mark.parametrize("T", [512 * 148 * 3 + 64, 512 * 300])
+@pytest.mark.parametrize("T", [512 * 148 * 3 + 64, 512 * 300, 512 * 148, 512 * 149])
 def test_layout_several_tiles_per_cta(T, mode):
     # more tiles than resident CTAs: each CTA walks a run of tiles and carries
     # its bucket starts from one tile to the next (T = 512*148*3 + 64 leaves a
-    # short last tile; R = 8 divides both sizes)
+    # short last tile).  512*148 tiles launch one CTA per SM, so the arrival
+    # wait reads more than 128 stamps; 512*149 gives two tiles per CTA.  R = 8
+    # divides every size.
     E, k, R = 64, 6, 8
     lg = synth.normal_f32(T, E, 21, 1).numpy()
     idx = oracle.route_topk(lg, k)[0]
