@@ -2,15 +2,23 @@
 
 One step = one pass of the per-layer hot path over one batch:
     md_route_topk -> md_dispatch_layout (dedup) -> md_dispatch_permute -> md_combine
-on the workload "zipf_pairs_e128_k8" (T=65536 tokens, hidden 2048 bf16, E=128,
-top-8, 16 virtual EP ranks, correlated Zipf(1.1) pair logits, contiguous
-placement).  Inputs are synthetic, seeded, resident in HBM, and larger than L2.
+on the workload "full_e256_k8": T=262144 tokens, hidden 2048 bf16, E=256,
+top-8 (softmax over the selected logits), 64 virtual EP ranks, correlated
+Zipf(1.1) group logits with a x4 expert-load skew.  The expert placement is
+the correlated one, fitted once before the timed steps (co-selection counts W
+over all tokens, then best single swaps from contiguous placement), as the
+pages refit it only every ~1000 steps.  Inputs are synthetic, seeded, resident
+in HBM, and each step moves ~17 GB, far more than the 126 MB L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
 
 Under torchrun each rank runs an independent replica on its own GPU (the
 virtual EP ranks live inside one GPU; nothing is sharded), times K steps with
-CUDA events, and rank 0 prints one JSON line with the max over ranks.
+CUDA events, and rank 0 prints one JSON line with the max over ranks.  The
+`rows` object times every other workload of the path on its own (config-2
+conventional and dedup dispatch, the L2-flushed small config, the top-2
+H=4096 config at EP 8 and 32, the token shuffle and the dedup dispatch after
+it, placement modes, routing statistics, the full E=256 pipeline).
 --impl reference times the CPU oracle on the host instead (bounded samples).
 """
 from __future__ import annotations
@@ -19,6 +27,7 @@ import argparse
 import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -33,10 +42,21 @@ sys.path.insert(0, ROOT)
 
 METRIC = "dispatch+combine Mtokens/s at 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
 UNIT = "Mtokens/s"
-WORKLOAD = "zipf_pairs_e128_k8"
+WORKLOAD = "full_e256_k8"
 NOMINAL_HBM_GBS = 8000.0    # B200 HBM3e, nominal (context only; the roofline uses the measured peak)
 FALLBACK_HBM_GBS = 6650.0
-CPU_TOKENS_PER_S_GUESS = 16000.0  # oracle, one core, this workload's shape
+CPU_TOKENS_PER_S_GUESS = 12000.0  # oracle, one core, this workload's shape
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 # ------------------------------------------------------------- environment
@@ -152,13 +172,15 @@ def algorithmic_bytes(T, H, k, E, n_rows):
     }
 
 
-def kernel_traffic(name, launches_units, units_per_launch):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current source of the kernel; else None."""
+def kernel_traffic(name, workload, units_per_launch):
+    """DRAM bytes per launch from the committed ncu record of this kernel on
+    this workload's shape, if it was taken on the current source of the kernel;
+    else None.  The record holds bytes per token of a smaller capture of the
+    same (E, k, H, R) workload; every token moves the same rows."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
-            rec = json.load(f).get(name)
+            rec = json.load(f).get(f"{name}@{workload}")
     except Exception:
         return None
     if not rec:
@@ -171,6 +193,25 @@ def kernel_traffic(name, launches_units, units_per_launch):
     if digest != rec.get("source_sha256_16"):
         return None
     return rec["dram_bytes_per_unit"] * units_per_launch
+
+
+def hbm_peak():
+    peaks = measured_peaks()
+    if peaks and "hbm_gbs" in peaks:
+        return float(peaks["hbm_gbs"]), "of measured"
+    return FALLBACK_HBM_GBS, "of fallback"
+
+
+def gbps(nbytes, ms, peak):
+    a = nbytes / (ms * 1e-3) / 1e9
+    return {"GBps": round(a, 1), "frac": round(a / peak, 3),
+            "frac_of_nominal_8TBps": round(a / NOMINAL_HBM_GBS, 3)}
+
+
+def fit_placement(md, idx, E, R, T_fit, seed_mode, stream=None):
+    """Correlated placement from the co-selection counts of tokens [0, T_fit)."""
+    W, _ = md.md_coselect_stats(idx, None, E, T_fit=T_fit, stream=stream)
+    return md.md_place_correlated(W, R, seed_mode=seed_mode, stream=stream), W
 
 
 # -------------------------------------------------------------- native arm
@@ -186,15 +227,22 @@ def run_native(args):
     md.lib()  # fail loudly if the library is missing
 
     w = synth.make_workload(WORKLOAD, seed=args.seed, device=device)
+    w.logits_next = None  # the headline step routes one layer
+    torch.cuda.empty_cache()
     T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
     mode = md.MD_DEDUP if args.dispatch == "dedup" else md.MD_CONV
     stream = torch.cuda.Stream(device)
-    cap = T * k if mode == md.MD_CONV else T * min(k, R)
+    # the placement: fitted once, before the timed steps
+    with torch.cuda.stream(stream):
+        idx0, _ = md.md_route_topk(w.logits, k, stream=stream)
+        p, _ = fit_placement(md, idx0, E, R, w.fit_tokens, md.MD_SEED_CONTIGUOUS, stream)
+    stream.synchronize()
+    del idx0
     idx = torch.empty(T, k, dtype=torch.int32, device=device)
     gates = torch.empty(T, k, dtype=torch.float32, device=device)
     L = md.alloc_layout(T, E, k, R, mode, device)
     wsp = md.alloc_workspace(md.dispatch_layout_workspace_size(T, E, k, R, mode), device)
-    buf = torch.empty(cap, H, dtype=torch.bfloat16, device=device)
+    buf = torch.empty(L.row_capacity, H, dtype=torch.bfloat16, device=device)
     out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
     status = md.new_status(device)
     torch.cuda.synchronize()
@@ -205,8 +253,8 @@ def run_native(args):
         md.md_route_topk(w.logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp,
-                              dev_status=status, stream=stream)
+        md.md_dispatch_layout(idx, E, R, p, mode, out=L, workspace=wsp, dev_status=status,
+                              stream=stream)
         if ev is not None:
             ev[2].record(stream)
         md.md_dispatch_permute(w.x, L.row_of_slot, out=buf, stream=stream)
@@ -244,24 +292,22 @@ def run_native(args):
     total_ms_max = max_over_ranks(dist, total_ms, device)
     n_rows = int(L.n_rows.item())
     md.check_status(status, "layout status")
+    contiguous = synth.contiguous_placement(E, R, device)
+    n_rows_contiguous = int(md.md_dispatch_layout(idx, E, R, contiguous, mode).n_rows.item())
 
     # end to end through host buffers: inputs copied in, the result copied out
-    e2e = run_e2e(args, md, w, mode, device, stream, idx, gates, L, wsp, buf, status, dist)
+    e2e = run_e2e(args, md, w, p, mode, device, stream, idx, gates, L, wsp, buf, status, dist)
+    torch.cuda.synchronize()
 
     if rank != 0:
         return None
-    peaks = measured_peaks()
-    peak = float(peaks["hbm_gbs"]) if peaks and "hbm_gbs" in peaks else FALLBACK_HBM_GBS
-    peak_src = "of measured" if peaks and "hbm_gbs" in peaks else "of fallback"
+    peak, peak_src = hbm_peak()
     ab = algorithmic_bytes(T, H, k, E, n_rows)
-    kernels = {n: {"us": round(per[n] * 1e3, 2), "bytes": ab[n],
-                   "GBps": round(ab[n] / (per[n] * 1e-3) / 1e9, 1),
-                   "frac": round(ab[n] / (per[n] * 1e-3) / 1e9 / peak, 3),
-                   "frac_of_nominal_8TBps": round(ab[n] / (per[n] * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 3)}
+    kernels = {n: {"us": round(per[n] * 1e3, 2), "bytes": ab[n], **gbps(ab[n], per[n], peak)}
                for n in per}
     dom = max(("dispatch_permute", "combine"), key=lambda n: per[n])
     achieved = ab[dom] / (per[dom] * 1e-3) / 1e9
-    traffic = kernel_traffic(dom, args.steps, T)
+    traffic = kernel_traffic(dom, WORKLOAD, T)
     value = T * args.steps * ws / (total_ms_max * 1e-3) / 1e6
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": ws,
@@ -269,25 +315,35 @@ def run_native(args):
         "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
         "dispatch_combine_excl_router": round(
             T * ws / ((per["dispatch_layout"] + per["dispatch_permute"] + per["combine"]) * 1e-3) / 1e6, 3),
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes of the pages' E=256 top-8 model)",
         "config": {"workload": WORKLOAD, "T": T, "H": H, "E": E, "top_k": k, "ep_ranks": R,
                    "dispatch": args.dispatch, "combine": "fused", "gates": "topk_softmax",
-                   "placement": "contiguous", "parallelism": f"replicas x{ws}",
-                   "l2": "not flushed: every step moves >2.6 GB through HBM, 20x the 126 MB L2",
-                   "dedup_rows_per_token": round(n_rows / T, 4)},
+                   "placement": "correlated: W over all tokens, best single swaps from "
+                                "contiguous, fitted once before the timed steps",
+                   "parallelism": f"replicas x{ws}",
+                   "l2": "not flushed: every step moves ~17 GB through HBM, >100x the 126 MB L2",
+                   "dedup_rows_per_token": round(n_rows / T, 4),
+                   "dedup_rows_per_token_contiguous": round(n_rows_contiguous / T, 4)},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "peak_source": peak_src,
+                     "frac_of_nominal_8TBps": round(achieved / NOMINAL_HBM_GBS, 4),
                      "traffic": None if traffic is None else int(traffic),
                      "algorithmic_bytes_per_launch": ab[dom]},
+        "step_roofline": {"bytes_per_step": sum(ab.values()),
+                          "achieved_GBps": round(sum(ab.values()) / (total_ms_max / args.steps * 1e-3) / 1e9, 1),
+                          "frac": round(sum(ab.values()) / (total_ms_max / args.steps * 1e-3) / 1e9 / peak, 4)},
         "kernels": kernels,
         "gpu_launches": int(launches),
         "e2e": e2e,
         "clocks": clk.summary(),
     }
+    del buf, out, L, wsp
+    w.y = None
+    w.x = None
+    torch.cuda.empty_cache()
     if args.rows:
-        del w, buf, out
-        torch.cuda.empty_cache()
         line["rows"] = run_rows(args, md, device, stream, peak)
     line["cpu_baseline"] = cpu_baseline(args)
     return line
@@ -312,17 +368,29 @@ def _time(fn, stream, reps):
     return e0.elapsed_time(e1) / reps
 
 
+def _remote_rows(send_counts):
+    """Rows that leave their source rank: the off-diagonal sum of the send matrix."""
+    sc = send_counts.to(torch.int64)
+    return int(sc.sum().item() - sc.diagonal().sum().item())
+
+
 def run_rows(args, md, device, stream, peak):
-    """Every step of the path on the workload it belongs to (one GPU)."""
+    """Every other workload of the path, each on its own (one GPU)."""
+    rows = {}
+    rows.update(rows_config2(args, md, device, stream, peak))
+    rows.update(rows_config1(args, md, device, stream, peak))
+    rows.update(rows_config3(args, md, device, stream, peak))
+    rows.update(rows_config4(args, md, device, stream, peak))
+    rows.update(rows_config5_planning(args, md, device, stream, peak))
+    return rows
+
+
+def rows_config2(args, md, device, stream, peak):
+    """zipf_pairs_e128_k8: conventional and dedup dispatch, wire combine, expand."""
     from combine_warp_top_router_b200 import synth
     rows = {}
     reps = args.row_reps
-
-    def gbps(nbytes, ms):
-        return {"GBps": round(nbytes / (ms * 1e-3) / 1e9, 1), "frac": round(nbytes / (ms * 1e-3) / 1e9 / peak, 3)}
-
-    # conventional dispatch and the two-stage (wire) combine, same workload as the headline
-    w = synth.make_workload(WORKLOAD, seed=args.seed, device=device)
+    w = synth.make_workload("zipf_pairs_e128_k8", seed=args.seed, device=device)
     T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
     idx, gates = md.md_route_topk(w.logits, k)
     for name, mode in (("conv", md.MD_CONV), ("dedup", md.MD_DEDUP)):
@@ -339,9 +407,9 @@ def run_rows(args, md, device, stream, peak):
                        stream, reps)
         pb = T * (2 * H + 4 * k) + n * 2 * H
         cb = T * (2 * H * (k + 1) + 12 * k)
-        r = {"rows_per_token": round(n / T, 4), "layout_us": round(t_lay * 1e3, 2),
-             "permute_us": round(t_perm * 1e3, 2), "permute": gbps(pb, t_perm),
-             "combine_us": round(t_comb * 1e3, 2), "combine": gbps(cb, t_comb),
+        r = {"T": T, "rows_per_token": round(n / T, 4), "layout_us": round(t_lay * 1e3, 2),
+             "permute_us": round(t_perm * 1e3, 2), "permute": gbps(pb, t_perm, peak),
+             "combine_us": round(t_comb * 1e3, 2), "combine": gbps(cb, t_comb, peak),
              "dispatch_combine_Mtokens_per_s": round(T / ((t_lay + t_perm + t_comb) * 1e-3) / 1e6, 2)}
         if mode == md.MD_DEDUP:
             z = torch.empty(L.row_capacity, H, dtype=torch.bfloat16, device=device)
@@ -350,7 +418,7 @@ def run_rows(args, md, device, stream, peak):
                                                  stream=stream), stream, reps)
             wb = T * (2 * H * k + 2 * H + 16 * k) + n * 2 * H
             r["combine_wire_us"] = round(t_wire * 1e3, 2)
-            r["combine_wire"] = gbps(wb, t_wire)
+            r["combine_wire"] = gbps(wb, t_wire, peak)
             del z
             # receiver side: dedup rows -> one row per (token, expert), expert-grouped
             xc = torch.empty(T * k, H, dtype=torch.bfloat16, device=device)
@@ -358,84 +426,216 @@ def run_rows(args, md, device, stream, peak):
                                                      stream=stream), stream, reps)
             eb = n * 2 * H + T * k * (2 * H + 8)
             r["dedup_expand_us"] = round(t_exp * 1e3, 2)
-            r["dedup_expand"] = gbps(eb, t_exp)
+            r["dedup_expand"] = gbps(eb, t_exp, peak)
             del xc
         rows[f"zipf_pairs_e128_k8_{name}"] = r
         del L, wsp, buf, out
     t_topk = _time(lambda: md.md_route_topk(w.logits, k, topk_idx=idx, topk_w=gates, stream=stream),
                    stream, reps)
-    rows["route_topk_e128_k8"] = {"us": round(t_topk * 1e3, 2), **gbps(T * (4 * E + 8 * k), t_topk)}
+    rows["route_topk_e128_k8"] = {"us": round(t_topk * 1e3, 2), **gbps(T * (4 * E + 8 * k), t_topk, peak)}
     del w, idx, gates
     torch.cuda.empty_cache()
+    return rows
 
-    # token shuffle on the two-layer workload (C fitted on the first 4096 tokens)
+
+def rows_config1(args, md, device, stream, peak):
+    """iid_e64_k6 (T=4096, 117 MB per kernel, about the size of L2): every
+    step is timed on its own with L2 flushed before it (a write of twice the
+    L2 size), and the median over the steps is reported."""
+    from combine_warp_top_router_b200 import synth
+    w = synth.make_workload("iid_e64_k6", seed=args.seed, device=device)
+    T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
+    mode = md.MD_CONV
+    idx = torch.empty(T, k, dtype=torch.int32, device=device)
+    gates = torch.empty(T, k, dtype=torch.float32, device=device)
+    L = md.alloc_layout(T, E, k, R, mode, device)
+    wsp = md.alloc_workspace(md.dispatch_layout_workspace_size(T, E, k, R, mode), device)
+    buf = torch.empty(L.row_capacity, H, dtype=torch.bfloat16, device=device)
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+    l2 = int(getattr(torch.cuda.get_device_properties(device), "L2_cache_size", 126 << 20))
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+    parts = ("route_topk", "dispatch_layout", "dispatch_permute", "combine")
+    calls = (
+        lambda: md.md_route_topk(w.logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream),
+        lambda: md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp,
+                                      stream=stream),
+        lambda: md.md_dispatch_permute(w.x, L.row_of_slot, out=buf, stream=stream),
+        lambda: md.md_combine(w.y, L.assign_row, idx, gates, out=out, stream=stream),
+    )
+    torch.cuda.synchronize()
+    times = {n: [] for n in parts + ("step",)}
+    n_steps = max(20, args.row_reps)
+    with torch.cuda.stream(stream):
+        for i in range(3 + n_steps):
+            flush.fill_(i & 0xff)
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+            ev[0].record(stream)
+            for j, c in enumerate(calls):
+                c()
+                ev[j + 1].record(stream)
+            stream.synchronize()
+            if i >= 3:
+                for j, n in enumerate(parts):
+                    times[n].append(ev[j].elapsed_time(ev[j + 1]))
+                times["step"].append(ev[0].elapsed_time(ev[-1]))
+    med = {n: statistics.median(v) for n, v in times.items()}
+    n = int(L.n_rows.item())
+    ab = algorithmic_bytes(T, H, k, E, n)
+    r = {"T": T, "H": H, "E": E, "top_k": k, "ep_ranks": R, "dispatch": "conv",
+         "placement": "contiguous", "l2": f"flushed before every step ({2 * l2 >> 20} MiB write)",
+         "steps": n_steps, "median_step_us": round(med["step"] * 1e3, 2),
+         "Mtokens_per_s": round(T / (med["step"] * 1e-3) / 1e6, 2),
+         "dispatch_combine_excl_router": round(
+             T / ((med["dispatch_layout"] + med["dispatch_permute"] + med["combine"]) * 1e-3) / 1e6, 2)}
+    for nme in parts:
+        r[nme] = {"us": round(med[nme] * 1e3, 2), **gbps(ab[nme], med[nme], peak)}
+    del w, idx, gates, L, wsp, buf, out, flush
+    torch.cuda.empty_cache()
+    return {"iid_e64_k6_l2_flushed": r}
+
+
+def rows_config3(args, md, device, stream, peak):
+    """boost_pairs_e128_k2 (T=65536, H=4096, top-2) at EP 8 and 32: placement
+    fitted on tokens [0, 4096) (greedy pair seed, then best single swaps),
+    dedup dispatch and fused combine; rows per token against contiguous."""
+    from combine_warp_top_router_b200 import synth
+    rows = {}
+    reps = args.row_reps
+    w = synth.make_workload("boost_pairs_e128_k2", seed=args.seed, device=device)
+    T, H, E, k = w.T, w.H, w.E, w.k
+    idx, gates = md.md_route_topk(w.logits, k)
+    for R in (8, 32):
+        p, _ = fit_placement(md, idx, E, R, w.fit_tokens, md.MD_SEED_GREEDY_PAIRS)
+        mode = md.MD_DEDUP
+        L = md.alloc_layout(T, E, k, R, mode, device)
+        wsp = md.alloc_workspace(md.dispatch_layout_workspace_size(T, E, k, R, mode), device)
+        buf = torch.empty(L.row_capacity, H, dtype=torch.bfloat16, device=device)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+        t_lay = _time(lambda: md.md_dispatch_layout(idx, E, R, p, mode, out=L, workspace=wsp,
+                                                      stream=stream), stream, reps)
+        n = int(L.n_rows.item())
+        t_perm = _time(lambda: md.md_dispatch_permute(w.x, L.row_of_slot, out=buf, stream=stream),
+                       stream, reps)
+        t_comb = _time(lambda: md.md_combine(w.y, L.assign_row, idx, gates, out=out, stream=stream),
+                       stream, reps)
+        Lc = md.md_dispatch_layout(idx, E, R, synth.contiguous_placement(E, R, device), mode)
+        ab = algorithmic_bytes(T, H, k, E, n)
+        rows[f"boost_pairs_e128_k2_ep{R}"] = {
+            "T": T, "H": H, "rows_per_token": round(n / T, 4),
+            "rows_per_token_contiguous": round(int(Lc.n_rows.item()) / T, 4),
+            "remote_rows_per_token": round(_remote_rows(L.send_counts) / T, 4),
+            "remote_rows_per_token_contiguous": round(_remote_rows(Lc.send_counts) / T, 4),
+            "layout_us": round(t_lay * 1e3, 2),
+            "permute_us": round(t_perm * 1e3, 2), "permute": gbps(ab["dispatch_permute"], t_perm, peak),
+            "combine_us": round(t_comb * 1e3, 2), "combine": gbps(ab["combine"], t_comb, peak),
+            "dispatch_combine_Mtokens_per_s": round(T / ((t_lay + t_perm + t_comb) * 1e-3) / 1e6, 2)}
+        del L, wsp, buf, out, Lc
+    del w, idx, gates
+    torch.cuda.empty_cache()
+    return rows
+
+
+def rows_config4(args, md, device, stream, peak):
+    """The token shuffle and the dedup dispatch after it.  Single form on
+    two_layer_e128_k6, pair form on three_layer_e128_k6; counts fitted on
+    tokens [0, 4096); contiguous placement at layer l+1.  After the shuffle the
+    layer-(l+1) top-k rows are gathered into the shuffled order and the dedup
+    layout runs with src = the token's new block."""
+    from combine_warp_top_router_b200 import synth
+    rows = {}
+    reps = args.row_reps
+
+    def after_shuffle(nxt, inv, E, R, p_next):
+        """dedup rows and remote rows per token at l+1 in the given token order"""
+        T = nxt.shape[0]
+        ordered = nxt if inv is None else md.md_gather_rows(nxt, inv)
+        L = md.md_dispatch_layout(ordered, E, R, p_next, md.MD_DEDUP)
+        return {"rows_per_token": round(int(L.n_rows.item()) / T, 4),
+                "remote_rows_per_token": round(_remote_rows(L.send_counts) / T, 4)}
+
+    # single-expert prediction
     w = synth.make_workload("two_layer_e128_k6", seed=args.seed, device=device)
+    T, E, R = w.T, w.E, w.R
     a, _ = md.md_route_topk(w.logits, w.k)
     b, _ = md.md_route_topk(w.logits_next, w.k)
-    _, C = md.md_coselect_stats(a, b, w.E, T_fit=w.fit_tokens, want_W=False)
-    sws = md.alloc_workspace(int(md.lib().md_token_shuffle_workspace_size(w.T, w.E, w.R)), device)
-    pred = torch.empty(w.T, dtype=torch.int32, device=device)
+    _, C = md.md_coselect_stats(a, b, E, T_fit=w.fit_tokens, want_W=False)
+    sws = md.alloc_workspace(int(md.lib().md_token_shuffle_workspace_size(T, E, R)), device)
+    pred = torch.empty(T, dtype=torch.int32, device=device)
     perm = torch.empty_like(pred)
     inv = torch.empty_like(pred)
-    t_sh = _time(lambda: md.md_token_shuffle(a, C, w.expert_to_rank, w.R, pred, perm, inv,
+    t_sh = _time(lambda: md.md_token_shuffle(a, C, w.expert_to_rank, R, pred, perm, inv,
                                              workspace=sws, stream=stream), stream, reps)
     xs = torch.empty_like(w.x)
     t_g = _time(lambda: md.md_gather_rows(w.x, inv, out=xs, stream=stream), stream, reps)
-    loc_before = float((torch.arange(w.T, device=device) // (w.T // w.R)).eq(
-        w.expert_to_rank[b.long()].T).float().mean())
-    bs = b[inv.long()]
-    loc_after = float((torch.arange(w.T, device=device) // (w.T // w.R)).eq(
-        w.expert_to_rank[bs.long()].T).float().mean())
+    bs = torch.empty_like(b)
+    t_gi = _time(lambda: md.md_gather_rows(b, inv, out=bs, stream=stream), stream, reps)
+    Ls = md.alloc_layout(T, E, w.k, R, md.MD_DEDUP, device)
+    lws = md.alloc_workspace(md.dispatch_layout_workspace_size(T, E, w.k, R, md.MD_DEDUP), device)
+    t_lay = _time(lambda: md.md_dispatch_layout(bs, E, R, w.expert_to_rank, md.MD_DEDUP, out=Ls,
+                                                  workspace=lws, stream=stream), stream, reps)
+    none = after_shuffle(b, None, E, R, w.expert_to_rank)
+    single = after_shuffle(b, inv, E, R, w.expert_to_rank)
     # the rounds-based parallel assignment on the same inputs
-    rws = md.alloc_workspace(int(md.lib().md_token_shuffle_rounds_workspace_size(w.T, w.E, w.R)),
-                             device)
+    rws = md.alloc_workspace(int(md.lib().md_token_shuffle_rounds_workspace_size(T, E, R)), device)
     rp, rperm, rinv = torch.empty_like(pred), torch.empty_like(pred), torch.empty_like(pred)
     holder = {}
     t_rd = _time(lambda: holder.__setitem__("r", md.md_token_shuffle_rounds(
-        a, C, w.expert_to_rank, w.R, rp, rperm, rinv, workspace=rws, stream=stream)[3]), stream, reps)
+        a, C, w.expert_to_rank, R, rp, rperm, rinv, workspace=rws, stream=stream)[3]), stream, reps)
     n_rounds = int(holder["r"].item())
-    loc_rounds = float((torch.arange(w.T, device=device) // (w.T // w.R)).eq(
-        w.expert_to_rank[b[rinv.long()].long()].T).float().mean())
+    rounds = after_shuffle(b, rinv, E, R, w.expert_to_rank)
+    loc = lambda order: float((torch.arange(T, device=device) // (T // R)).eq(
+        w.expert_to_rank[order.long()].T).float().mean())
     rows["token_shuffle_e128_k6"] = {
-        "T": w.T, "shuffle_us": round(t_sh * 1e3, 2), "gather_x_us": round(t_g * 1e3, 2),
-        "gather": gbps(2 * w.T * 2 * w.H + 4 * w.T, t_g),
-        "locality_before": round(loc_before, 4), "locality_after": round(loc_after, 4),
+        "T": T, "shuffle_us": round(t_sh * 1e3, 2), "gather_x_us": round(t_g * 1e3, 2),
+        "gather": gbps(2 * T * 2 * w.H + 4 * T, t_g, peak),
+        "gather_topk_us": round(t_gi * 1e3, 2), "layout_after_shuffle_us": round(t_lay * 1e3, 2),
+        "locality_before": round(loc(b), 4), "locality_after": round(loc(b[inv.long()]), 4),
+        "dedup_dispatch_at_next_layer": {"no_shuffle": none, "single": single,
+                                         "rounds": rounds},
         "rounds_variant": {"us": round(t_rd * 1e3, 2), "rounds": n_rounds,
-                           "locality_after": round(loc_rounds, 4)}}
-    del w, a, b, C, sws, xs
+                           "locality_after": round(loc(b[rinv.long()]), 4)}}
+    del w, a, b, C, sws, xs, bs, Ls, lws
     torch.cuda.empty_cache()
 
-    # pair-based shuffle prediction on the three-layer workload (counts fitted
-    # on the first 4096 tokens; a pair row is used when its total reaches 8k)
+    # pair-based prediction on the three-layer workload (a pair row is used
+    # when its total reaches 8k)
     w = synth.make_workload("three_layer_e128_k6", seed=args.seed, device=device, with_rows=False)
+    T, E, R = w.T, w.E, w.R
     g = [md.md_route_topk(lg, w.k)[0] for lg in (w.logits_prev, w.logits, w.logits_next)]
-    C2 = torch.empty(w.E, w.E, w.E, dtype=torch.int32, device=device)
-    t_c2 = _time(lambda: md.md_coselect_pair_stats(g[0], g[1], g[2], w.E, T_fit=w.fit_tokens, C2=C2,
+    C2 = torch.empty(E, E, E, dtype=torch.int32, device=device)
+    t_c2 = _time(lambda: md.md_coselect_pair_stats(g[0], g[1], g[2], E, T_fit=w.fit_tokens, C2=C2,
                                                    stream=stream), stream, reps)
-    _, C = md.md_coselect_stats(g[1], g[2], w.E, T_fit=w.fit_tokens, want_W=False)
-    pws = md.alloc_workspace(int(md.lib().md_token_shuffle_pair_workspace_size(w.T, w.E, w.R)), device)
-    pred = torch.empty(w.T, dtype=torch.int32, device=device)
+    _, C = md.md_coselect_stats(g[1], g[2], E, T_fit=w.fit_tokens, want_W=False)
+    pws = md.alloc_workspace(int(md.lib().md_token_shuffle_pair_workspace_size(T, E, R)), device)
+    pred = torch.empty(T, dtype=torch.int32, device=device)
     perm, inv, use = torch.empty_like(pred), torch.empty_like(pred), torch.empty_like(pred)
     min_obs = 8 * w.k
-    t_sp = _time(lambda: md.md_token_shuffle_pair(g[0], g[1], C, C2, w.expert_to_rank, w.R, min_obs,
+    t_sp = _time(lambda: md.md_token_shuffle_pair(g[0], g[1], C, C2, w.expert_to_rank, R, min_obs,
                                                   pred, perm, inv, use, workspace=pws,
                                                   stream=stream), stream, reps)
     nxt_rank = w.expert_to_rank[g[2].long()]
-    loc_pair = float(pred[:, None].eq(nxt_rank).float().mean())
-    use_share = float(use.float().mean())
-    sp = md.md_token_shuffle(g[1], C, w.expert_to_rank, w.R)[0]
-    loc_single = float(sp[:, None].eq(nxt_rank).float().mean())
-    loc_none = float((torch.arange(w.T, device=device) // (w.T // w.R))[:, None].eq(nxt_rank)
-                     .float().mean())
+    sp, _, sinv = md.md_token_shuffle(g[1], C, w.expert_to_rank, R)
     rows["token_shuffle_pair_e128_k6"] = {
-        "T": w.T, "min_obs": min_obs, "pair_counts_us": round(t_c2 * 1e3, 2),
-        "shuffle_pair_us": round(t_sp * 1e3, 2), "tokens_on_pair_rows": round(use_share, 4),
-        "locality_no_shuffle": round(loc_none, 4), "locality_single": round(loc_single, 4),
-        "locality_pair": round(loc_pair, 4)}
+        "T": T, "min_obs": min_obs, "pair_counts_us": round(t_c2 * 1e3, 2),
+        "shuffle_pair_us": round(t_sp * 1e3, 2), "tokens_on_pair_rows": round(float(use.float().mean()), 4),
+        "locality_no_shuffle": round(float((torch.arange(T, device=device) // (T // R))[:, None]
+                                           .eq(nxt_rank).float().mean()), 4),
+        "locality_single": round(float(sp[:, None].eq(nxt_rank).float().mean()), 4),
+        "locality_pair": round(float(pred[:, None].eq(nxt_rank).float().mean()), 4),
+        "dedup_dispatch_at_next_layer": {"no_shuffle": after_shuffle(g[2], None, E, R, w.expert_to_rank),
+                                         "single": after_shuffle(g[2], sinv, E, R, w.expert_to_rank),
+                                         "pair": after_shuffle(g[2], inv, E, R, w.expert_to_rank)}}
     del w, g, C2, C, pws
     torch.cuda.empty_cache()
+    return rows
 
-    # the full pipeline at full size: T=262144, E=256, k=8, R=64
+
+def rows_config5_planning(args, md, device, stream, peak):
+    """The E=256 workload's planning steps: the full pipeline with co-selection
+    counts and placement inside every step, placement modes, routing statistics."""
+    from combine_warp_top_router_b200 import synth
+    rows = {}
+    reps = args.row_reps
     w = synth.make_workload("full_e256_k8", seed=args.seed, device=device)
     T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
     a = torch.empty(T, k, dtype=torch.int32, device=device)
@@ -482,12 +682,13 @@ def run_rows(args, md, device, stream, peak):
         pipeline()
     stream.synchronize()
     evs = []
+    n_runs = max(1, reps // 5)
     with torch.cuda.stream(stream):
-        for _ in range(max(1, reps // 5)):
+        for _ in range(n_runs):
             pipeline(evs)
     stream.synchronize()
     for name, e0, e1 in evs:
-        parts[name] = parts.get(name, 0.0) + e0.elapsed_time(e1) / max(1, reps // 5)
+        parts[name] = parts.get(name, 0.0) + e0.elapsed_time(e1) / n_runs
     total = sum(parts.values())
     n = int(L.n_rows.item())
     contiguous = synth.contiguous_placement(E, R, device)
@@ -510,8 +711,8 @@ def run_rows(args, md, device, stream, peak):
 
     # the pages' routing statistics on this workload: Table I columns for both
     # placements, the cross-layer successor share, fitted vs held-out W
-    s_corr = md.table1_row(md.md_rank_stats(a, E, R, p))
-    s_cont = md.table1_row(md.md_rank_stats(a, E, R, contiguous))
+    s_corr = md.table1_row(md.md_rank_stats(a, E, R, p).cpu())
+    s_cont = md.table1_row(md.md_rank_stats(a, E, R, contiguous).cpu())
     Wf, Cf = md.md_coselect_stats(a[:4096], b[:4096], E)
     Wh, _ = md.md_coselect_stats(a[4096:8192], None, E)
     num, den = md.md_successor_share(Cf, Wf)
@@ -528,93 +729,134 @@ def run_rows(args, md, device, stream, peak):
         "parts_us": {kk: round(v * 1e3, 1) for kk, v in parts.items()},
         "rows_per_token_correlated": round(n / T, 4),
         "rows_per_token_contiguous": round(int(Lc.n_rows.item()) / T, 4),
-        "permute": gbps(T * (2 * H + 4 * k) + n * 2 * H, parts["dispatch_permute"]),
-        "combine": gbps(T * (2 * H * (k + 1) + 12 * k), parts["combine"])}
+        "permute": gbps(T * (2 * H + 4 * k) + n * 2 * H, parts["dispatch_permute"], peak),
+        "combine": gbps(T * (2 * H * (k + 1) + 12 * k), parts["combine"], peak)}
     del w, buf, out
     torch.cuda.empty_cache()
     return rows
 
 
-def run_e2e(args, md, w, mode, device, stream, idx, gates, L, wsp, buf, status, dist):
-    """Same step through host buffers: pinned inputs -> HBM, path, result -> host.
+def _pinned_copy(t):
+    h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+    h.copy_(t)
+    return h
+
+
+def run_e2e(args, md, w, p, mode, device, stream, idx, gates, L, wsp, buf, status, dist):
+    """The same step through host buffers: pinned inputs -> HBM, the path, the
+    result -> host.  Two forms:
+
+    * main: every input of the timed step (logits, x and the expert outputs y)
+      is copied in each step, and the combined rows are copied out;
+    * y_on_device: only logits and x are copied in; the expert outputs are made
+      on the device by identity experts (the receiver-side expand of the dedup
+      rows, md_dedup_expand, gives each (token, expert) its row), so the step
+      is router -> layout -> permute -> expand -> combine.
 
     Steps are pipelined over two device buffer sets, as a serving loop would
     run them: the inputs of step i+1 copy in (one copy stream) while step i
     computes and step i-1's result copies out (another copy stream).  Every
     step still moves all of its own inputs in and its result out."""
     T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
-    h_logits = w.logits.cpu().pin_memory()
-    h_x = w.x.cpu().pin_memory()
-    h_y = w.y.cpu().pin_memory()
-    h_out = [torch.empty(T, H, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    d_in = [(w.logits, w.x, w.y)] + [(torch.empty_like(w.logits), torch.empty_like(w.x),
-                                      torch.empty_like(w.y))]
+    h_logits = _pinned_copy(w.logits)
+    h_x = _pinned_copy(w.x)
+    h_out = [torch.empty(T, H, dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
     d_out = [torch.empty(T, H, dtype=torch.bfloat16, device=device) for _ in range(2)]
     s_in = torch.cuda.Stream(device)
     s_out = torch.cuda.Stream(device)
     steps = max(1, min(args.steps, args.e2e_steps))
-    ev = lambda: torch.cuda.Event()
-    in_done = [ev(), ev()]      # inputs of set b are in HBM
-    used = [ev(), ev()]         # the step on set b no longer reads its inputs
-    out_done = [ev(), ev()]     # the result of set b is on the host
-
-    def step(i):
-        b = i % 2
-        d_logits, d_x, d_y = d_in[b]
-        s_in.wait_event(used[b])
-        with torch.cuda.stream(s_in):
-            d_logits.copy_(h_logits, non_blocking=True)
-            d_x.copy_(h_x, non_blocking=True)
-            d_y.copy_(h_y, non_blocking=True)
-        in_done[b].record(s_in)
-        stream.wait_event(in_done[b])
-        stream.wait_event(out_done[b])
-        md.md_route_topk(d_logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream)
-        md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp,
-                              dev_status=status, stream=stream)
-        md.md_dispatch_permute(d_x, L.row_of_slot, out=buf, stream=stream)
-        md.md_combine(d_y, L.assign_row, idx, gates, out=d_out[b], stream=stream)
-        used[b].record(stream)
-        s_out.wait_event(used[b])
-        with torch.cuda.stream(s_out):
-            h_out[b].copy_(d_out[b], non_blocking=True)
-        out_done[b].record(s_out)
-
-    for e in used + out_done:
-        e.record(stream)
-    for i in range(2):
-        step(i)
-    torch.cuda.synchronize()
-    barrier(dist, device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(s_in)
-    for i in range(steps):
-        step(i)
-    s_in.wait_stream(s_out)
-    s_in.wait_stream(stream)
-    e1.record(s_in)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(dist, e0.elapsed_time(e1), device)
-    # the last step's result is the step's own output
-    assert torch.equal(h_out[(steps - 1) % 2], d_out[(steps - 1) % 2].cpu())
     ws = dist.get_world_size() if dist is not None else 1
-    h2d = (h_logits.numel() * 4 + h_x.numel() * 2 + h_y.numel() * 2)
+
+    def measure(y_from_host):
+        h_y = _pinned_copy(w.y) if y_from_host else None
+        d_in = [(w.logits, w.x, w.y)] + [(torch.empty_like(w.logits), torch.empty_like(w.x),
+                                          torch.empty_like(w.y))]
+        ev = lambda: torch.cuda.Event()
+        in_done = [ev(), ev()]      # inputs of set b are in HBM
+        used = [ev(), ev()]         # the step on set b no longer reads its inputs
+        out_done = [ev(), ev()]     # the result of set b is on the host
+
+        def step(i):
+            b = i % 2
+            d_logits, d_x, d_y = d_in[b]
+            s_in.wait_event(used[b])
+            with torch.cuda.stream(s_in):
+                d_logits.copy_(h_logits, non_blocking=True)
+                d_x.copy_(h_x, non_blocking=True)
+                if y_from_host:
+                    d_y.copy_(h_y, non_blocking=True)
+            in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            stream.wait_event(out_done[b])
+            md.md_route_topk(d_logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream)
+            md.md_dispatch_layout(idx, E, R, p, mode, out=L, workspace=wsp, dev_status=status,
+                                  stream=stream)
+            md.md_dispatch_permute(d_x, L.row_of_slot, out=buf, stream=stream)
+            if not y_from_host:
+                md.md_dedup_expand(buf, L.row_of_slot, L.assign_row, out=d_y, stream=stream)
+            md.md_combine(d_y, L.assign_row, idx, gates, out=d_out[b], stream=stream)
+            used[b].record(stream)
+            s_out.wait_event(used[b])
+            with torch.cuda.stream(s_out):
+                h_out[b].copy_(d_out[b], non_blocking=True)
+            out_done[b].record(s_out)
+
+        for e in used + out_done:
+            e.record(stream)
+        for i in range(2):
+            step(i)
+        torch.cuda.synchronize()
+        barrier(dist, device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(s_in)
+        for i in range(steps):
+            step(i)
+        s_in.wait_stream(s_out)
+        s_in.wait_stream(stream)
+        e1.record(s_in)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(dist, e0.elapsed_time(e1), device)
+        # the last step's result is the step's own output
+        assert torch.equal(h_out[(steps - 1) % 2], d_out[(steps - 1) % 2].cpu())
+        h2d = h_logits.numel() * 4 + h_x.numel() * 2 + (w.y.numel() * 2 if y_from_host else 0)
+        del d_in, h_y
+        torch.cuda.empty_cache()
+        return ms, h2d
+
+    if mode != md.MD_DEDUP:
+        raise SystemExit("the end-to-end leg expects the dedup dispatch")
+    ms, h2d = measure(True)       # first: it copies the synthetic y to the host
+    ms_y, h2d_y = measure(False)  # then the expand overwrites the device y
+    d2h = int(h_out[0].numel() * 2)
     return {"value": round(T * steps * ws / (ms * 1e-3) / 1e6, 4), "unit": UNIT,
-            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(h_out[0].numel() * 2),
-            "steps": steps,
-            "note": "pinned host buffers; two device buffer sets, inputs of the next step "
-                    "copy in while the result of the previous one copies out"}
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": d2h, "steps": steps,
+            "note": "pinned host buffers; logits, x and the expert outputs y copied in every "
+                    "step, the combined rows copied out; two device buffer sets, inputs of the "
+                    "next step copy in while the result of the previous one copies out",
+            "y_on_device": {
+                "value": round(T * steps * ws / (ms_y * 1e-3) / 1e6, 4), "unit": UNIT,
+                "h2d_bytes_per_step": int(h2d_y), "d2h_bytes_per_step": d2h,
+                "note": "logits and x copied in; identity experts on the device (md_dedup_expand "
+                        "of the dedup rows) make y; router -> layout -> permute -> expand -> "
+                        "combine; result copied out"}}
 
 
 # -------------------------------------------------------- oracle (CPU) arm
 
 def oracle_sample(T_s, seed):
-    """Inputs for a T_s-token sample of the workload (same recipe, E, k, R, H)."""
+    """Inputs for a T_s-token sample of the headline workload (same recipe, E, k,
+    R, H), with the oracle's own correlated placement fitted on the sample
+    (untimed, as the GPU arm fits its placement before timing)."""
+    import oracle
     from combine_warp_top_router_b200 import synth
     w = synth.make_workload(WORKLOAD, seed=seed, device="cpu", T=T_s)
     bits = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
-    return (w.logits.numpy(), bits(w.x), bits(w.y), w.expert_to_rank.numpy(), w.E, w.k, w.R)
+    lg = w.logits.numpy()
+    idx = oracle.route_topk(lg, w.k)[0]
+    W, _ = oracle.coselect(idx, None, w.E)
+    p = oracle.place_correlated(W, w.R)
+    return (lg, bits(w.x), bits(w.y), p, w.E, w.k, w.R)
 
 
 def oracle_step(oracle, inp, dedup=True):
@@ -641,8 +883,9 @@ def cpu_baseline(args):
     dt = time.perf_counter() - t0
     out = {"value": round(T_s * reps / dt / 1e6, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
            "sample": f"{reps} x {T_s}-token sample of the same workload recipe "
-                     f"(E=128, top-8, 16 ranks, H=2048), single-threaded C oracle, "
-                     f"{dt:.1f} s", "host_cores": os.cpu_count()}
+                     f"(E=256, top-8, 64 ranks, H=2048, correlated placement fitted on the "
+                     f"sample), single-threaded C oracle, {dt:.1f} s",
+           "host_cores": os.cpu_count(), "cpu_model": cpu_model()}
     if args.rows:
         out["rows"] = cpu_rows(oracle, args.seed)
     return out
@@ -690,8 +933,10 @@ def run_reference(args):
     if rank != 0:
         return None
     import oracle
+    from combine_warp_top_router_b200 import synth
     oracle.build()
-    R = 16
+    spec = synth.SPECS[WORKLOAD]
+    R = spec["R"]
     # bound the run to about a minute of CPU for K + W steps
     per_step = 60.0 / max(1, args.steps + args.warmup)
     T_s = int(per_step * CPU_TOKENS_PER_S_GUESS) // R * R
@@ -709,11 +954,12 @@ def run_reference(args):
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "T": T_s, "H": 2048, "E": 128, "top_k": 8, "ep_ranks": R,
-                   "dispatch": args.dispatch, "combine": "fused",
+        "config": {"workload": WORKLOAD, "T": T_s, "H": spec["H"], "E": spec["E"],
+                   "top_k": spec["k"], "ep_ranks": R, "dispatch": args.dispatch, "combine": "fused",
+                   "placement": "correlated, fitted on the sample before timing",
                    "note": "each step is a bounded sample of the workload"},
         "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"{T_s}-token sample per step"},
+                         "sample": f"{T_s}-token sample per step", "cpu_model": cpu_model()},
         "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -722,13 +968,13 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--dispatch", choices=["dedup", "conv"], default="dedup")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--cpu-sample-tokens", type=int, default=32768)
+    ap.add_argument("--cpu-sample-tokens", type=int, default=16384)
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
     ap.add_argument("--rows", action=argparse.BooleanOptionalAction, default=True,
                     help="also time every step of the path on its own workload")

@@ -58,6 +58,8 @@ _SIGNATURES = {
     "md_place_two_level": ([_P, _I, _I, _I, _I, _I, _P, _P, _S, _P, _P], _I),
     "md_successor_share": ([_P, _P, _I, _P, _P, _P], _I),
     "md_count_sums": ([_P, _P, _L, _P, _P], _I),
+    "md_table1_row": ([_P, _I, _P], _I),
+    "md_pearson_from_sums": ([_P, _L, _P], _I),
     "md_token_shuffle_pair_workspace_size": ([_L, _I, _I], _S),
     "md_token_shuffle_pair": ([_P, _P, _I, _P, _P, _P, _L, _I, _I, ctypes.c_uint32, _P, _P, _P, _P,
                                _P, _S, _P, _P], _I),
@@ -100,6 +102,21 @@ def launch_count() -> int:
 def _check(rc: int, what: str):
     if rc != MD_OK:
         raise MoeDispatchError(rc, what)
+
+
+def _call(name: str, dev, *args) -> int:
+    """Call entry point `name` with `dev` as the current CUDA device.
+
+    The CUDA runtime launches on the calling thread's current device, and the
+    library looks up per-device state (kernel attributes, the allocation-free
+    scratch array) for that device, so tensors on another device are handled
+    by making their device current for the call."""
+    fn = getattr(lib(), name)
+    dev = torch.device(dev)
+    if dev.index is None or torch.cuda.current_device() == dev.index:
+        return fn(*args)
+    with torch.cuda.device(dev):
+        return fn(*args)
 
 
 def _ptr(t):
@@ -160,7 +177,7 @@ def md_route_topk(logits, k, gate_mode=MD_GATE_TOPK_SOFTMAX, topk_idx=None, topk
     _need(topk_w, "topk_w", torch.float32, dev)
     _room(topk_idx, "topk_idx", T * k)
     _room(topk_w, "topk_w", T * k)
-    rc = lib().md_route_topk(_ptr(logits), T, E, k, gate_mode, _ptr(topk_idx), _ptr(topk_w),
+    rc = _call("md_route_topk", dev, _ptr(logits), T, E, k, gate_mode, _ptr(topk_idx), _ptr(topk_w),
                              _stream(stream, dev))
     _check(rc, "md_route_topk")
     return topk_idx, topk_w
@@ -227,7 +244,7 @@ def md_dispatch_layout(topk_idx, E, R, expert_to_rank, mode, out: Layout | None 
     if workspace is None:
         workspace = alloc_workspace(need, dev)
     _need(workspace, "workspace", torch.uint8, dev)
-    rc = lib().md_dispatch_layout(
+    rc = _call("md_dispatch_layout", dev, 
         _ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), mode, _ptr(out.row_of_slot),
         _ptr(out.assign_row), _ptr(out.row_token), _ptr(out.row_mask), _ptr(out.send_counts),
         _ptr(out.expert_counts), _ptr(out.expert_offsets), _ptr(out.rank_offsets),
@@ -249,7 +266,7 @@ def md_dispatch_layout_noalloc(topk_idx, E, R, expert_to_rank, mode, out: Layout
     if out is None:
         out = alloc_layout(T, E, k, R, mode, dev)
     _check_layout(out, T, E, k, R, mode, dev)
-    rc = lib().md_dispatch_layout_noalloc(
+    rc = _call("md_dispatch_layout_noalloc", dev, 
         _ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), mode, _ptr(out.row_of_slot),
         _ptr(out.assign_row), _ptr(out.row_token), _ptr(out.row_mask), _ptr(out.send_counts),
         _ptr(out.expert_counts), _ptr(out.expert_offsets), _ptr(out.rank_offsets),
@@ -272,7 +289,7 @@ def md_dispatch_permute(x, row_of_slot, out_rows=None, out=None, dev_status=None
     _need(out, "out", torch.bfloat16, dev)
     if out.dim() != 2 or out.shape[1] != H:
         raise ValueError(f"out must be [rows, {H}]")
-    rc = lib().md_dispatch_permute(_ptr(x), T, H, k, _ptr(row_of_slot), out.shape[0], _ptr(out),
+    rc = _call("md_dispatch_permute", dev, _ptr(x), T, H, k, _ptr(row_of_slot), out.shape[0], _ptr(out),
                                    _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_dispatch_permute")
     return out
@@ -295,7 +312,7 @@ def md_dedup_expand(wire, row_of_slot, assign_row, out_rows=None, out=None, dev_
     _need(out, "out", torch.bfloat16, dev)
     if out.dim() != 2 or out.shape[1] != H:
         raise ValueError(f"out must be [rows, {H}]")
-    rc = lib().md_dedup_expand(_ptr(wire), wire.shape[0], H, _ptr(row_of_slot), _ptr(assign_row), T,
+    rc = _call("md_dedup_expand", dev, _ptr(wire), wire.shape[0], H, _ptr(row_of_slot), _ptr(assign_row), T,
                                k, out.shape[0], _ptr(out), _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_dedup_expand")
     return out
@@ -322,7 +339,7 @@ def md_combine(y, assign_row, topk_idx, topk_w, mode=MD_COMBINE_FUSED, row_of_sl
         _need(z, "z", torch.bfloat16, dev)
         _room(row_of_slot, "row_of_slot", T * k)
         z_rows = z.shape[0]
-    rc = lib().md_combine(_ptr(y), y.shape[0], _ptr(assign_row), _ptr(topk_idx), _ptr(topk_w), T,
+    rc = _call("md_combine", dev, _ptr(y), y.shape[0], _ptr(assign_row), _ptr(topk_idx), _ptr(topk_w), T,
                           k, H, mode, _ptr(row_of_slot), z_rows, _ptr(z), _ptr(out),
                           _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_combine")
@@ -342,7 +359,7 @@ def md_gather_rows(src, index, out=None, dev_status=None, stream=None):
     _room(out, "out", n * (src[0].numel() if src.shape[0] else out[0].numel()))
     row_bytes = src[0].numel() * src.element_size() if src.shape[0] else \
         out[0].numel() * out.element_size()
-    rc = lib().md_gather_rows(_ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out),
+    rc = _call("md_gather_rows", dev, _ptr(src), src.shape[0], row_bytes, _ptr(index), n, _ptr(out),
                               _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_gather_rows")
     return out
@@ -372,7 +389,7 @@ def md_coselect_stats(idx_l, idx_next, E, T_fit=None, W=None, C=None, accumulate
         if t is not None:
             _need(t, n, torch.int32, dev)
             _room(t, n, E * E)
-    rc = lib().md_coselect_stats(_ptr(idx_l), _ptr(idx_next), T_fit, E, k, _ptr(W), _ptr(C),
+    rc = _call("md_coselect_stats", dev, _ptr(idx_l), _ptr(idx_next), T_fit, E, k, _ptr(W), _ptr(C),
                                  1 if accumulate else 0, _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_coselect_stats")
     return W, C
@@ -392,7 +409,7 @@ def md_place_correlated(W, R, seed_mode=MD_SEED_CONTIGUOUS, refine=True, out=Non
     need = int(lib().md_place_correlated_workspace_size(E, R))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    rc = lib().md_place_correlated(_ptr(W), E, R, seed_mode, 1 if refine else 0, _ptr(out),
+    rc = _call("md_place_correlated", dev, _ptr(W), E, R, seed_mode, 1 if refine else 0, _ptr(out),
                                    _ptr(workspace), workspace.numel(), _ptr(dev_status),
                                    _stream(stream, dev))
     _check(rc, "md_place_correlated")
@@ -415,7 +432,7 @@ def md_place_two_level(W, R, nodes=1, seed_mode=MD_SEED_CONTIGUOUS, refine_mode=
     need = int(lib().md_place_two_level_workspace_size(E, R, nodes))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    rc = lib().md_place_two_level(_ptr(W), E, R, nodes, seed_mode, refine_mode, _ptr(out),
+    rc = _call("md_place_two_level", dev, _ptr(W), E, R, nodes, seed_mode, refine_mode, _ptr(out),
                                   _ptr(workspace), workspace.numel(), _ptr(dev_status),
                                   _stream(stream, dev))
     _check(rc, "md_place_two_level")
@@ -447,7 +464,7 @@ def md_token_shuffle(idx_l, C, expert_to_rank_next, R, pred_rank=None, perm=None
     need = int(lib().md_token_shuffle_workspace_size(T, E, R))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    rc = lib().md_token_shuffle(_ptr(idx_l), k, _ptr(C), _ptr(expert_to_rank_next), T, E, R,
+    rc = _call("md_token_shuffle", dev, _ptr(idx_l), k, _ptr(C), _ptr(expert_to_rank_next), T, E, R,
                                 _ptr(pred_rank), _ptr(perm), _ptr(inv), _ptr(workspace),
                                 workspace.numel(), _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_token_shuffle")
@@ -472,7 +489,7 @@ def md_token_shuffle_rounds(idx_l, C, expert_to_rank_next, R, pred_rank=None, pe
     need = int(lib().md_token_shuffle_rounds_workspace_size(T, E, R))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    rc = lib().md_token_shuffle_rounds(_ptr(idx_l), k, _ptr(C), _ptr(expert_to_rank_next), T, E, R,
+    rc = _call("md_token_shuffle_rounds", dev, _ptr(idx_l), k, _ptr(C), _ptr(expert_to_rank_next), T, E, R,
                                        _ptr(pred_rank), _ptr(perm), _ptr(inv), _ptr(rounds),
                                        _ptr(workspace), workspace.numel(), _ptr(dev_status),
                                        _stream(stream, dev))
@@ -497,7 +514,7 @@ def md_coselect_pair_stats(idx_prev, idx_l, idx_next, E, T_fit=None, C2=None, ac
         raise ValueError("idx_prev, idx_l and idx_next differ in k")
     if min(idx_prev.shape[0], idx_next.shape[0], T) < T_fit:
         raise ValueError("fewer than T_fit rows")
-    rc = lib().md_coselect_pair_stats(_ptr(idx_prev), _ptr(idx_l), _ptr(idx_next), T_fit, E, k,
+    rc = _call("md_coselect_pair_stats", dev, _ptr(idx_prev), _ptr(idx_l), _ptr(idx_next), T_fit, E, k,
                                       _ptr(C2), 1 if accumulate else 0, _ptr(dev_status),
                                       _stream(stream, dev))
     _check(rc, "md_coselect_pair_stats")
@@ -529,7 +546,7 @@ def md_token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_ob
     need = int(lib().md_token_shuffle_pair_workspace_size(T, E, R))
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    rc = lib().md_token_shuffle_pair(_ptr(idx_prev), _ptr(idx_l), k, _ptr(C), _ptr(C2),
+    rc = _call("md_token_shuffle_pair", dev, _ptr(idx_prev), _ptr(idx_l), k, _ptr(C), _ptr(C2),
                                      _ptr(expert_to_rank_next), T, E, R, int(min_obs),
                                      _ptr(pred_rank), _ptr(perm), _ptr(inv), _ptr(use_pair),
                                      _ptr(workspace), workspace.numel(), _ptr(dev_status),
@@ -550,18 +567,20 @@ def md_rank_stats(topk_idx, E, R, expert_to_rank, hist=None, dev_status=None, st
     _need(hist, "hist", torch.int64, dev)
     _room(hist, "hist", k + 1)
     _room(expert_to_rank, "expert_to_rank", E)
-    rc = lib().md_rank_stats(_ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), _ptr(hist),
+    rc = _call("md_rank_stats", dev, _ptr(topk_idx), T, E, k, R, _ptr(expert_to_rank), _ptr(hist),
                              _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_rank_stats")
     return hist
 
 
 def table1_row(hist):
-    """Table I columns from a rank histogram: (same-rank %, ranks per token, dedup %)."""
-    h = [int(v) for v in hist.tolist()]
-    T, k = sum(h), len(h) - 1
-    gpus = sum(d * n for d, n in enumerate(h)) / T
-    return 100.0 * h[1] / T, gpus, 100.0 * (1.0 - gpus / k)
+    """Table I columns from a rank histogram: (same-rank %, ranks per token, dedup %)
+    (md_table1_row on the host)."""
+    h = (ctypes.c_int64 * len(hist))(*[int(v) for v in hist.tolist()])
+    out = (ctypes.c_double * 3)()
+    _check(lib().md_table1_row(ctypes.cast(h, _P), len(hist) - 1, ctypes.cast(out, _P)),
+           "md_table1_row")
+    return out[0], out[1], out[2]
 
 
 def md_successor_share(C, W, stream=None):
@@ -574,7 +593,7 @@ def md_successor_share(C, W, stream=None):
         raise ValueError("C and W must be [E, E]")
     num = torch.empty(E, dtype=torch.int32, device=dev)
     den = torch.empty(E, dtype=torch.int32, device=dev)
-    rc = lib().md_successor_share(_ptr(C), _ptr(W), E, _ptr(num), _ptr(den), _stream(stream, dev))
+    rc = _call("md_successor_share", dev, _ptr(C), _ptr(W), E, _ptr(num), _ptr(den), _stream(stream, dev))
     _check(rc, "md_successor_share")
     return num, den
 
@@ -587,17 +606,26 @@ def md_count_sums(x, y, stream=None):
     if x.numel() != y.numel():
         raise MoeDispatchError("md_count_sums: tables differ in size")
     out = torch.empty(10, dtype=torch.int64, device=dev)
-    rc = lib().md_count_sums(_ptr(x), _ptr(y), x.numel(), _ptr(out), _stream(stream, dev))
+    rc = _call("md_count_sums", dev, _ptr(x), _ptr(y), x.numel(), _ptr(out), _stream(stream, dev))
     _check(rc, "md_count_sums")
     w = [v & (2 ** 64 - 1) for v in out.cpu().tolist()]
     return tuple(w[2 * i] | (w[2 * i + 1] << 64) for i in range(5))
 
 
 def pearson_from_sums(n, sums):
-    """Pearson correlation from the exact sums of md_count_sums."""
-    sx, sy, sxx, syy, sxy = sums
-    vx, vy = n * sxx - sx * sx, n * syy - sy * sy
-    return (n * sxy - sx * sy) / (vx * vy) ** 0.5 if vx > 0 and vy > 0 else float("nan")
+    """Pearson correlation from the exact sums of md_count_sums (md_pearson_from_sums
+    on the host); NaN when a table has zero variance."""
+    words = []
+    for v in sums:
+        v = int(v)
+        words += [v & (2 ** 64 - 1), (v >> 64) & (2 ** 64 - 1)]
+    c = (ctypes.c_uint64 * 10)(*words)
+    r = ctypes.c_double()
+    rc = lib().md_pearson_from_sums(ctypes.cast(c, _P), int(n), ctypes.byref(r))
+    if rc == MD_ERR_DATA:
+        return float("nan")
+    _check(rc, "md_pearson_from_sums")
+    return r.value
 
 
 def md_set_test_hooks(poll_limit=0, layout_skip_tile=-1, expand_skip_unit=-1):

@@ -119,8 +119,11 @@ __global__ void __launch_bounds__(kWarps * 32)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) {
             md::report(status, MD_ERR_TIMEOUT);
+            // wait, again bounded, for the load that timed out and the ones
+            // issued after it; one late beyond both bounds can still land in
+            // shared memory after the block has exited
             if (lane == 0)
-                for (int a = 1; a <= kAhead; ++a)
+                for (int a = 0; a <= kAhead; ++a)
                     if (u + a * nw < U)
                         md::mbar_wait_bounded(&bar[(i + a) % kStages],
                                               (uint32_t)(((i + a) / kStages) & 1), polls);

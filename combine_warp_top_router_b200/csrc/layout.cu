@@ -15,7 +15,7 @@
 // fewer when k > 8).
 //   A. Every CTA counts its tokens per bucket (shared-memory histograms) and
 //      the send-matrix rows of the source ranks it covers, writes them to the
-//      workspace and stamps its arrival word with this call's epoch.
+//      workspace and stamps its arrival word (cleared to 0 before the launch).
 //   B. After every stamp is seen (a bounded wait), each CTA reads the count
 //      table: bucket totals give the bucket bases, the counts of CTAs before
 //      it give its start inside each bucket.  Each CTA also sums a slice of
@@ -24,10 +24,11 @@
 //      32-bit set per bucket, built with shared atomicOr), so a pair's rank
 //      among the warp's earlier tokens is a popcount; rows are staged in
 //      shared memory in bucket order and written out in runs.
-// Nothing in the workspace has to start at zero: the arrival words are
-// compared with a per-call epoch, and every count is written before it is read.
-// A graph replays one epoch, so a capturing stream also records a clear of
-// the arrival words and the epoch is fixed at 1.
+// Nothing in the workspace has to start at zero: every call first clears the
+// arrival words on its stream (a 1 KiB memset, recorded too when the stream is
+// capturing), so a word left over from an earlier call, or from whatever the
+// memory held before, can never pass for this call's arrival; every count is
+// written before it is read.
 #include "common.cuh"
 
 namespace {
@@ -38,12 +39,10 @@ constexpr int kStageRows = 4096;   // output rows a tile can stage
 constexpr int kMaxCtas = 256;      // CTAs of one launch; the workspace is sized for it
 constexpr long long kPollLimit = 1ll << 22;
 
-std::atomic<unsigned long long> g_epoch{0};
-
 struct Ws {
     long long poll_limit;         // bound of the arrival wait
     int skip_cta;                 // test hook: this CTA never stamps its arrival (-1: none)
-    unsigned epoch;               // this call's stamp (never 0)
+    unsigned epoch;               // the arrival stamp (the words are cleared to 0 first)
     unsigned *flags;              // [kMaxCtas] arrival words
     int *cnt;                     // [NB][kMaxCtas] bucket counts per CTA
     int *part;                    // [(kMaxCtas + R) * R] send rows: CTA c, source s at row c + s
@@ -88,9 +87,7 @@ Ws carve(void *ws, const Plan &p)
     Ws w;
     w.poll_limit = md::hook_poll_limit(kPollLimit);
     w.skip_cta = md::hook_layout_skip_tile();
-    do {
-        w.epoch = (unsigned)(g_epoch.fetch_add(1) + 1);
-    } while (w.epoch == 0u);
+    w.epoch = 1u;
     w.flags = reinterpret_cast<unsigned *>(b + p.off_flags);
     w.cnt = reinterpret_cast<int *>(b + p.off_cnt);
     w.part = reinterpret_cast<int *>(b + p.off_part);
@@ -181,9 +178,6 @@ __global__ void __launch_bounds__(kRankThreads, 1)
     const int tile_lo = cta * tpc;
     const int tile_hi = tile_lo + tpc < n_tiles ? tile_lo + tpc : n_tiles;
     const int64_t Tr = R > 0 && T > 0 ? T / R : 1;
-    // the status word is cleared before this CTA stamps its arrival, and every
-    // report comes after the arrival wait
-    if (cta == 0 && tid == 0 && status) *status = MD_OK;
     if (tid == 0) s_timeout = 0;
     for (int e = tid; e < E; e += kRankThreads) s_p[e] = p_g[e];
     for (int i = tid; i < NB; i += kRankThreads) s_acnt[i] = 0;
@@ -264,7 +258,7 @@ __global__ void __launch_bounds__(kRankThreads, 1)
         __threadfence();
         st_relaxed_u32(ws.flags + cta, ws.epoch);
     }
-    // every CTA's counts are in once its stamp carries this call's epoch; one
+    // every CTA's counts are in once its arrival word is stamped; one
     // warp reads all stamps, four per 16-byte load
     if (w == 0) {
         long long polls = 0;
@@ -663,17 +657,15 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return MD_ERR_ARG;
     cudaStream_t s = md::as_stream(stream);
     Ws ws = carve(workspace, pl);
-    cudaStreamCaptureStatus cst = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(s, &cst) != cudaSuccess) {
+    // The status word and the arrival words are cleared on the stream before
+    // the kernel, eagerly and under capture alike (a graph records both
+    // memsets, so every replay waits for its own counts).  Stale arrival words
+    // can therefore never let a CTA pass the wait early.
+    if ((rc = md::clear_status(dev_status, s)) != MD_OK) return rc;
+    md::count_launches(1);
+    if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 4, s) != cudaSuccess) {
         cudaGetLastError();
-        cst = cudaStreamCaptureStatusNone;
-    }
-    if (cst == cudaStreamCaptureStatusActive) {
-        // a graph replays the launch with the same arguments: the arrival
-        // words are cleared inside the graph and the epoch is fixed
-        md::count_launches(1);
-        if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 4, s) != cudaSuccess) return MD_ERR_CUDA;
-        ws.epoch = 1;
+        return MD_ERR_CUDA;
     }
 
     const int64_t cap = mode == MD_CONV ? T * k : T * (int64_t)(k < R ? k : R);
@@ -751,7 +743,8 @@ extern "C" int md_dispatch_layout_noalloc(const int32_t *topk_idx, int64_t T, in
     void *scratch = nullptr;
     if ((rc = scratch_for_current_device(&scratch)) != MD_OK) return rc;
     // The shared array keeps the previous call's contents; nothing in it has to
-    // start at zero (the arrival words are compared with a per-call epoch).
+    // start at zero (md_dispatch_layout clears the arrival words on the stream
+    // before its kernel).
     return md_dispatch_layout(topk_idx, T, E, k, R, expert_to_rank, mode, row_of_slot, assign_row,
                               row_token, row_mask, send_counts, expert_counts, expert_offsets,
                               rank_offsets, n_rows, scratch, kNoAllocScratchBytes, dev_status,

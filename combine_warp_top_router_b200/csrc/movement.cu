@@ -168,8 +168,11 @@ __global__ void __launch_bounds__(kTmaWarps * 32)
         if (!ok) {
             md::report(status, MD_ERR_TIMEOUT);
             if (lane == 0) {
-                // wait, again bounded, for the loads still in flight
-                for (int j = 1; j <= kTmaAhead; ++j)
+                // wait, again bounded, for the loads still in flight: the one
+                // that timed out and the ones issued after it.  A load that
+                // is merely late beyond both bounds can still land in shared
+                // memory after the block has exited.
+                for (int j = 0; j <= kTmaAhead; ++j)
                     if (u + j * nw < U)
                         md::mbar_wait_bounded(&bar[(i + j) % kTmaStages],
                                               (uint32_t)(((i + j) / kTmaStages) & 1), kTmaPolls);

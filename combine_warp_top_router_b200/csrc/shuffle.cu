@@ -1088,6 +1088,38 @@ extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx
     return md::launch_status();
 }
 
+namespace {
+
+// CTAs of k_shuf_rounds resident per SM with rsm bytes of dynamic shared
+// memory; -1 if CUDA refuses.  The shared-memory limit is raised once per
+// device to the largest size (E*R <= 64 KiB); the occupancy query itself is
+// host arithmetic and depends on rsm, so it runs per call.
+int rounds_per_sm(size_t rsm)
+{
+    static std::atomic<uint64_t> done{0};
+    static std::atomic<int> attr_ok[64];
+    md::once_per_device(done, [] {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const bool ok = cudaFuncSetAttribute(k_shuf_rounds, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             MD_MAX_EXPERTS * MD_MAX_RANKS) == cudaSuccess;
+        if (!ok) cudaGetLastError();
+        attr_ok[dev & 63].store(ok ? 1 : 0);
+    });
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_ok[dev & 63].load()) return -1;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_shuf_rounds, kRoundThreads, rsm) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return -1;
+    }
+    return per_sm;
+}
+
+}  // namespace
+
 extern "C" size_t md_token_shuffle_rounds_workspace_size(int64_t T, int E, int R)
 {
     if (T < 0 || E < 1 || R < 1) return 0;
@@ -1113,13 +1145,8 @@ extern "C" int md_token_shuffle_rounds(const int32_t *idx_l, int k, const uint32
     const int n_tiles = (int)((T + kTile - 1) / kTile);
     // every CTA must be resident at once (cooperative launch)
     const size_t rsm = (size_t)E * R;
-    if (cudaFuncSetAttribute(k_shuf_rounds, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsm) !=
-        cudaSuccess)
-        return MD_ERR_CUDA;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_shuf_rounds, kRoundThreads, rsm) !=
-        cudaSuccess)
-        return MD_ERR_CUDA;
+    const int per_sm = rounds_per_sm(rsm);
+    if (per_sm < 0) return MD_ERR_CUDA;
     if (T > 0 && (int64_t)per_sm * md::sm_count() < n_tiles) return MD_ERR_UNSUPPORTED;
     cudaStream_t s = md::as_stream(stream);
     int rc = md::clear_status(dev_status, s);
@@ -1154,8 +1181,10 @@ extern "C" int md_token_shuffle_rounds(const int32_t *idx_l, int k, const uint32
                     (void *)&TT, (void *)&EE, (void *)&RR, (void *)&TTr, (void *)&pred_rank,
                     (void *)&dev_status};
     if (cudaLaunchCooperativeKernel((const void *)k_shuf_rounds, dim3(n_tiles), dim3(kRoundThreads),
-                                    args, rsm, s) != cudaSuccess)
+                                    args, rsm, s) != cudaSuccess) {
+        cudaGetLastError();  // a refused launch must not be blamed on a later call
         return MD_ERR_CUDA;
+    }
     k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
                                                        ws.keys, ws.tile_hist);
     k_bucket_scan<<<1, kScanThreads, R * sizeof(int), s>>>(ws.tile_hist, n_tiles, R);

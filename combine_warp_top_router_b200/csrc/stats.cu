@@ -12,6 +12,8 @@
 //   largest C[e][e'].
 //   Correlation Formation and Stability: the Pearson correlation of two count
 //   tables follows from five exact sums, accumulated in 128 bits by one CTA.
+#include <cmath>
+
 #include "common.cuh"
 
 namespace {
@@ -155,4 +157,59 @@ extern "C" int md_count_sums(const uint32_t *x, const uint32_t *y, int64_t n, ui
     k_count_sums<<<1, 1024, 0, s>>>(x, y, n, reinterpret_cast<unsigned long long *>(sums));
     md::count_launches(1);
     return md::launch_status();
+}
+
+// ------------------------------------------------------------------------
+// Host helpers: the finished statistics from the device counts above.
+// ------------------------------------------------------------------------
+
+// Table I columns ("Expert Coupling ...", Offline Placement and Prediction
+// Statistics) from hist[D] = tokens on exactly D distinct ranks:
+//   out[0] "Same GPU" %  = 100 * hist[1] / T
+//   out[1] "GPUs"        = sum_D D * hist[D] / T   (mean distinct ranks)
+//   out[2] "Dedup" %     = 100 * (1 - GPUs / k)
+// The token count T = sum_D hist[D] and the weighted sum are exact integers.
+extern "C" int md_table1_row(const int64_t *hist, int k, double *out)
+{
+    if (!hist || !out || k < 1 || k > MD_MAX_TOPK) return MD_ERR_ARG;
+    int64_t T = 0, ranks = 0;
+    for (int d = 0; d <= k; ++d) {
+        if (hist[d] < 0) return MD_ERR_ARG;
+        T += hist[d];
+        ranks += (int64_t)d * hist[d];
+    }
+    if (T == 0) return MD_ERR_ARG;
+    const double gpus = (double)ranks / (double)T;
+    out[0] = 100.0 * (double)hist[1] / (double)T;
+    out[1] = gpus;
+    out[2] = 100.0 * (1.0 - gpus / (double)k);
+    return MD_OK;
+}
+
+// Pearson correlation of two count tables of n entries ("Expert Coupling
+// ...", Correlation Formation and Stability) from md_count_sums' exact sums
+// (sx, sy, sxx, syy, sxy as 128-bit (low, high) word pairs):
+//   r = (n sxy - sx sy) / sqrt((n sxx - sx^2) (n syy - sy^2)).
+// With n < 2^31 and 32-bit counts, sx < 2^63 and sxx, sxy < 2^95, so every
+// product and each of the three differences is exact in signed 128 bits; the
+// quotient is taken in long double.  A table with zero variance gives MD_ERR_DATA (r undefined).
+extern "C" int md_pearson_from_sums(const uint64_t *sums, int64_t n, double *r)
+{
+    if (!sums || !r || n < 1) return MD_ERR_ARG;
+    if (n >= ((int64_t)1 << 31)) return MD_ERR_UNSUPPORTED;
+    // n < 2^31 entries below 2^32: sums below 2^63, sums of products below 2^95
+    unsigned __int128 v[5];
+    for (int q = 0; q < 5; ++q) {
+        v[q] = ((unsigned __int128)sums[2 * q + 1] << 64) | sums[2 * q];
+        if (v[q] >> (q < 2 ? 63 : 95)) return MD_ERR_DATA;  // not sums of such counts
+    }
+    const __int128 N = n, sx = (__int128)v[0], sy = (__int128)v[1];
+    const __int128 sxx = (__int128)v[2], syy = (__int128)v[3], sxy = (__int128)v[4];
+    const __int128 cov = N * sxy - sx * sy;
+    const __int128 vx = N * sxx - sx * sx;
+    const __int128 vy = N * syy - sy * sy;
+    if (vx <= 0 || vy <= 0) return MD_ERR_DATA;
+    const long double den = sqrtl((long double)vx) * sqrtl((long double)vy);
+    *r = (double)((long double)cov / den);
+    return MD_OK;
 }

@@ -21,7 +21,9 @@
  *     aligned and H must be a multiple of 8 (16-byte rows).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Each call
  *     only enqueues work on it and returns; results are ready when the
- *     stream reaches that point.
+ *     stream reaches that point.  As for any CUDA runtime launch, the device
+ *     that holds the pointers and the stream must be the calling thread's
+ *     current device.
  *   - The return value reports what can be checked on the host: MD_ERR_ARG
  *     for bad sizes or pointers, MD_ERR_WORKSPACE for a short workspace,
  *     MD_ERR_CUDA when a launch fails.  Nothing is enqueued on an error.
@@ -132,14 +134,17 @@ int md_route_topk(const float *logits, int64_t T, int E, int k, int gate_mode,
  *   rank_offsets    int32 [R+1]    first row of rank d in this mode; [R] = n_rows
  *   n_rows          int32 [1]      rows in this mode (T*k for MD_CONV)
  *   workspace       >= md_dispatch_layout_workspace_size(...) bytes, 256-B
- *                   aligned; contents on entry do not matter.  The size does
- *                   not grow with T (at most about 1.2 MiB, at E=1024, R=64).
+ *                   aligned; contents on entry do not matter: the call clears
+ *                   its arrival words on `stream` before the kernel (one 1 KiB
+ *                   memset) and writes every count before reading it.  The
+ *                   size does not grow with T (at most about 1.2 MiB, at
+ *                   E=1024, R=64).
  *   One cooperative launch: all its CTAs (at most one per SM) must be
  *   resident at once, so a GPU shared with a running kernel that holds SMs
  *   may delay it; MD_ERR_CUDA if the launch is refused.  Every CTA waits for
  *   the others' counts with a bounded wait (MD_ERR_TIMEOUT in dev_status if
  *   it runs out; the outputs are then not written).  Safe in CUDA graph
- *   capture: a capturing stream also records a clear of the arrival words.
+ *   capture: the graph records the clear of the arrival words with the kernel.
  *   Limits: T % R == 0, E % R == 0, 1 <= k <= min(E, 32), E <= 1024,
  *   R <= 64, T*k < 2^31.
  */
@@ -453,12 +458,35 @@ int md_successor_share(const uint32_t *C, const uint32_t *W, int E, uint32_t *nu
 int md_count_sums(const uint32_t *x, const uint32_t *y, int64_t n, uint64_t *sums, void *stream);
 
 /*
+ * Host helpers that finish the statistics above (no device work; HOST
+ * pointers; they may be called without a GPU).
+ *
+ * md_table1_row -- Table I columns ("Expert Coupling ...", Offline Placement
+ *   and Prediction Statistics) from a rank histogram copied to the host:
+ *   hist  int64 [k+1] host (md_rank_stats), T = sum of hist > 0
+ *   out   double [3] host: "Same GPU" % = 100 hist[1] / T, "GPUs" = sum_D D
+ *         hist[D] / T (mean distinct ranks per token), "Dedup" % = 100 (1 -
+ *         GPUs / k).  MD_ERR_ARG for T == 0 or a negative entry.
+ *
+ * md_pearson_from_sums -- the Pearson correlation of two count tables of n
+ *   entries (Correlation Formation and Stability) from md_count_sums' five
+ *   exact sums copied to the host (uint64 [10]):
+ *   r = (n sxy - sx sy) / sqrt((n sxx - sx^2)(n syy - sy^2)), the three
+ *   differences exact in 128 bits, the quotient in long double.
+ *   MD_ERR_DATA when a table has zero variance (r undefined) or the sums
+ *   exceed what n 32-bit counts can give; 1 <= n < 2^31.
+ */
+int md_table1_row(const int64_t *hist, int k, double *out);
+
+int md_pearson_from_sums(const uint64_t *sums, int64_t n, double *r);
+
+/*
  * md_set_test_hooks -- fault injection for tests; not for production use.
  * Every bounded device-side wait gives up after a poll limit and reports
  * MD_ERR_TIMEOUT.  These hooks make such a wait run out on purpose, with no
  * fault: poll_limit > 0 replaces the default limits; layout_skip_tile >= 0
- * makes that md_dispatch_layout tile publish no lookback word, so the tiles
- * after it wait in vain; expand_skip_unit >= 0 makes md_dedup_expand (bulk-copy
+ * makes that md_dispatch_layout CTA stamp no arrival word, so every CTA
+ * waits for it in vain; expand_skip_unit >= 0 makes md_dedup_expand (bulk-copy
  * path) never fill that unit's shared-memory slot.  (0, -1, -1) restores the
  * defaults.  Process-wide; set them only while no other call is in flight.
  */

@@ -43,5 +43,7 @@ def test_algorithmic_bytes_match_the_calls_tensors(T, H, k, E, n_rows):
 
 def test_headline_combine_bytes_per_token():
     import bench
-    # 2H(k+1) + 12k = 36,960 B per token at H=2048, k=8
-    assert bench.algorithmic_bytes(65536, 2048, 8, 128, 0)["combine"] == 65536 * 36960
+    # the headline workload: T=262144, H=2048, E=256, k=8;
+    # 2H(k+1) + 12k = 36,960 B per token
+    assert bench.WORKLOAD == "full_e256_k8"
+    assert bench.algorithmic_bytes(262144, 2048, 8, 256, 0)["combine"] == 262144 * 36960

@@ -199,3 +199,39 @@ def test_layout_several_tiles_per_cta(T, mode):
     L, st = gpu_layout(idx, E, R, p, mode)
     assert st == md.MD_OK
     assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), T, k)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+@pytest.mark.parametrize("fill", ["stamp", "ones_bits", "random"])
+def test_layout_ignores_stale_workspace(fill, mode):
+    # Whatever the workspace holds on entry -- every 32-bit word equal to the
+    # value a CTA stamps on arrival (1), all bits set, or random words such as
+    # a recycled allocation holds -- the layout is the oracle's: the call
+    # clears its arrival words on the stream before the kernel, so no CTA can
+    # pass the arrival wait before every other CTA has published its counts.
+    E, k, R = 128, 8, 16
+    T = 512 * 148 * 2  # two tiles per CTA
+    lg = synth.make_workload("zipf_pairs_e128_k8", seed=4, T=T, with_rows=False).logits.numpy()
+    idx = oracle.route_topk(lg, k)[0]
+    p = shuffled_placement(E, R, 2)
+    O = oracle.dispatch_layout(idx, E, R, p, mode)
+    from combine_warp_top_router_b200 import binding
+    ws = binding.alloc_workspace(binding.dispatch_layout_workspace_size(T, E, k, R, mode), DEV)
+    words = ws.view(torch.int32)
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(17)
+    for rep in range(3):
+        if fill == "stamp":
+            words.fill_(1)
+        elif fill == "ones_bits":
+            words.fill_(-1)
+        else:
+            words.copy_(torch.randint(-2**31, 2**31 - 1, words.shape, generator=gen, device=DEV,
+                                      dtype=torch.int64).to(torch.int32))
+        L = md.alloc_layout(T, E, k, R, mode, DEV)
+        L.row_token.fill_(POISON)
+        st = torch.full((1,), 99, dtype=torch.int32, device=DEV)  # cleared by the call
+        md.md_dispatch_layout(i32(idx), E, R, i32(p), mode, out=L, workspace=ws, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == md.MD_OK
+        assert_layout_equal(L, O, T, k)
