@@ -25,6 +25,7 @@ MD_GATE_TOPK_SOFTMAX, MD_GATE_FULL_SOFTMAX = 0, 1
 MD_COMBINE_FUSED, MD_COMBINE_WIRE = 0, 1
 MD_SEED_CONTIGUOUS, MD_SEED_GREEDY_PAIRS = 0, 1
 MD_REFINE_NONE, MD_REFINE_SWAPS, MD_REFINE_KL = 0, 1, 2
+MD_PERMUTE_AUTO, MD_PERMUTE_BULK, MD_PERMUTE_VECTOR = 0, 1, 2
 
 _lock = threading.Lock()
 _lib = None
@@ -42,6 +43,7 @@ _SIGNATURES = {
     "md_dispatch_layout_noalloc": ([_P, _L, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P,
                                     _P, _P, _P], _I),
     "md_dispatch_permute": ([_P, _L, _I, _I, _P, _L, _P, _P, _P], _I),
+    "md_set_permute_path": ([_I], _I),
     "md_dedup_expand": ([_P, _L, _I, _P, _P, _L, _I, _L, _P, _P, _P], _I),
     "md_combine": ([_P, _L, _P, _P, _P, _L, _I, _I, _I, _P, _L, _P, _P, _P, _P], _I),
     "md_coselect_stats": ([_P, _P, _L, _I, _I, _P, _P, _I, _P, _P], _I),
@@ -293,6 +295,11 @@ def md_dispatch_permute(x, row_of_slot, out_rows=None, out=None, dev_status=None
                                    _ptr(dev_status), _stream(stream, dev))
     _check(rc, "md_dispatch_permute")
     return out
+
+
+def md_set_permute_path(path=MD_PERMUTE_AUTO):
+    """Choose md_dispatch_permute's kernel (tests and tuning; same bits either way)."""
+    _check(lib().md_set_permute_path(int(path)), "md_set_permute_path")
 
 
 def md_dedup_expand(wire, row_of_slot, assign_row, out_rows=None, out=None, dev_status=None,

@@ -19,7 +19,18 @@ long long hook_poll_limit(long long dflt)
 }
 int hook_layout_skip_tile() { return g_layout_skip_tile.load(std::memory_order_relaxed); }
 long long hook_expand_skip_unit() { return g_expand_skip_unit.load(std::memory_order_relaxed); }
+
+static std::atomic<int> g_permute_path{MD_PERMUTE_AUTO};
+int permute_path() { return g_permute_path.load(std::memory_order_relaxed); }
 }  // namespace md
+
+extern "C" int md_set_permute_path(int path)
+{
+    if (path != MD_PERMUTE_AUTO && path != MD_PERMUTE_BULK && path != MD_PERMUTE_VECTOR)
+        return MD_ERR_ARG;
+    md::g_permute_path.store(path, std::memory_order_relaxed);
+    return MD_OK;
+}
 
 extern "C" void md_set_test_hooks(long long poll_limit, int layout_skip_tile,
                                   long long expand_skip_unit)

@@ -21,6 +21,9 @@ long long hook_poll_limit(long long dflt);
 int hook_layout_skip_tile();        // -1: none
 long long hook_expand_skip_unit();  // -1: none
 
+// Kernel choice of md_dispatch_permute (md_set_permute_path).
+int permute_path();
+
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -107,6 +107,7 @@ constexpr int kTmaAhead = 2;
 constexpr int kTmaPiece = 4096;
 constexpr int kTmaMinRowBytes = 1024;
 constexpr long long kTmaPolls = 1ll << 22;
+static_assert(kTmaAhead >= 1 && kTmaAhead < kTmaStages, "ring: loads ahead < stages");
 
 template <int KC>
 __global__ void __launch_bounds__(kTmaWarps * 32)
@@ -313,6 +314,81 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// FUSED with a compile-time k: the same slot order and arithmetic as
+// k_combine<KC, false>, but for small k each thread works on U (token,
+// 16-byte column) items at once and issues all U*KC row loads before the
+// first FMA, so that 8 loads are in flight per thread (with k = 2 a single
+// item keeps only two in flight, and the kernel waits on latency).  From
+// k = 4 on one item per thread measured best.  Items of a group are
+// q = c + g*C for its ng tokens.
+template <int KC>
+constexpr int combine_items() { return KC >= 4 ? 1 : (8 + KC - 1) / KC; }
+
+template <int KC>
+__global__ void __launch_bounds__(kThreads)
+    k_combine_fused(const uint4 *__restrict__ y, int64_t y_rows, const int32_t *__restrict__ assign_row,
+                    const int32_t *__restrict__ idx, const float *__restrict__ w, int64_t T, int C,
+                    uint4 *__restrict__ out, int32_t *status)
+{
+    constexpr int U = combine_items<KC>();
+    __shared__ int s_r[kGroup][KC];
+    __shared__ float s_w[kGroup][KC];
+    const int lane = threadIdx.x & 31, wp = threadIdx.x >> 5;
+
+    for (int64_t g0 = (int64_t)blockIdx.x * kGroup; g0 < T; g0 += (int64_t)gridDim.x * kGroup) {
+        const int ng = (int)(T - g0 < kGroup ? T - g0 : kGroup);
+        // warp wp orders the slots of token g0 + wp by ascending expert
+        if (wp < ng) {
+            const int64_t t = g0 + wp;
+            const bool live = lane < KC;
+            const int e = live ? idx[t * KC + lane] : INT_MAX;
+            int r = live ? assign_row[t * KC + lane] : -1;
+            const float ww = live ? w[t * KC + lane] : 0.0f;
+            int rank = 0;
+#pragma unroll
+            for (int j = 0; j < KC; ++j) {
+                const int ej = __shfl_sync(0xffffffffu, e, j);
+                rank += (ej < e || (ej == e && j < lane)) ? 1 : 0;
+            }
+            if (live) {
+                if (r < 0 || r >= y_rows) {
+                    md::report(status, MD_ERR_DATA);
+                    r = -1;
+                }
+                s_r[wp][rank] = r;
+                s_w[wp][rank] = ww;
+            }
+        }
+        __syncthreads();
+        const int nq = ng * C;
+        for (int q0 = threadIdx.x; q0 < nq; q0 += kThreads * U) {
+            uint4 v[U][KC];
+            int gq[U], cq[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int q = q0 + u * kThreads;
+                gq[u] = q < nq ? q / C : -1;
+                cq[u] = q < nq ? q - gq[u] * C : 0;
+#pragma unroll
+                for (int j = 0; j < KC; ++j) {
+                    const int r = gq[u] >= 0 ? s_r[gq[u]][j] : -1;
+                    v[u][j] = r >= 0 ? md::ld_stream(y + (int64_t)r * C + cq[u]) : make_uint4(0, 0, 0, 0);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (gq[u] < 0) continue;
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j = 0; j < KC; ++j)
+                    if (s_r[gq[u]][j] >= 0) fma_row(acc, s_w[gq[u]][j], v[u][j]);
+                md::st_stream(out + (g0 + gq[u]) * C + cq[u], pack_row(acc));
+            }
+        }
+        __syncthreads();
+    }
+}
+
 // ------------------------------------------------------------------ gather
 __global__ void __launch_bounds__(kThreads)
     k_gather16(const uint4 *__restrict__ src, int64_t src_rows, int C,
@@ -357,12 +433,23 @@ void launch_permute(const void *x, int64_t T, int C, int k, const int32_t *rs, i
                     void *out, int32_t *st, cudaStream_t s)
 {
     const int rowbytes = C * 16;
-    if (rowbytes >= kTmaMinRowBytes) {
-        const int pieces = (rowbytes + kTmaPiece - 1) / kTmaPiece;
+    const int pieces = (rowbytes + kTmaPiece - 1) / kTmaPiece;
+    const int64_t units = T * pieces;
+    // Which kernel: bulk copies need rows of 1 KiB and more.  By shape (the
+    // default), they take the write-heavy calls -- k > 4 slots per token and
+    // at least 8 row pieces per warp of the bulk-copy grid -- where one ring
+    // of 4 warps per SM gave the best write bandwidth.  With k <= 4 a larger
+    // share of the bytes are reads and the ring waits on its loads; with few
+    // pieces per warp its start and drain dominate.  There the vector kernel,
+    // with one warp per token in flight across the whole GPU, measured faster.
+    const int path = md::permute_path();
+    bool bulk = rowbytes >= kTmaMinRowBytes && path != MD_PERMUTE_VECTOR;
+    if (bulk && path == MD_PERMUTE_AUTO)
+        bulk = k > 4 && units >= (int64_t)8 * md::sm_count() * kTmaWarps;
+    if (bulk) {
         const size_t smem = (size_t)kTmaWarps * kTmaStages * kTmaPiece;
         cudaFuncSetAttribute(k_permute_tma<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
-        const int64_t units = T * pieces;
         int64_t blocks = (units + kTmaWarps - 1) / kTmaWarps;
         const int64_t cap = md::sm_count();
         if (blocks > cap) blocks = cap;
@@ -388,6 +475,11 @@ void launch_combine(const void *y, int64_t y_rows, const int32_t *ar, const int3
                     const float *w, int64_t T, int k, int C, const int32_t *rs, int64_t z_rows,
                     void *z, void *out, int32_t *st, cudaStream_t s)
 {
+    if (KC > 0 && !WIRE) {
+        k_combine_fused<KC ? KC : 1><<<grid_for(T, kGroup), kThreads, 0, s>>>(
+            static_cast<const uint4 *>(y), y_rows, ar, idx, w, T, C, static_cast<uint4 *>(out), st);
+        return;
+    }
     k_combine<KC, WIRE><<<grid_for(T, kGroup), kThreads, 0, s>>>(
         static_cast<const uint4 *>(y), y_rows, ar, idx, w, T, k, C, rs, z_rows,
         static_cast<uint4 *>(z), static_cast<uint4 *>(out), st);

@@ -211,6 +211,24 @@ int md_dispatch_permute(const void *x, int64_t T, int H, int k,
                         int32_t *dev_status, void *stream);
 
 /*
+ * md_set_permute_path -- which kernel md_dispatch_permute runs (for tests and
+ * tuning; the result is the same bits either way).
+ *   MD_PERMUTE_AUTO    by shape (default): bulk copies through shared memory
+ *                      for rows of at least 1 KiB when k > 4 and the call has
+ *                      at least 8 row pieces of 4 KiB per warp of its grid;
+ *                      16-byte vector loads and stores otherwise
+ *   MD_PERMUTE_BULK    bulk copies whenever rows are at least 1 KiB
+ *   MD_PERMUTE_VECTOR  16-byte vectors always
+ * Process-wide; MD_ERR_ARG for another value.  Set it only while no
+ * md_dispatch_permute call is being enqueued.
+ */
+#define MD_PERMUTE_AUTO 0
+#define MD_PERMUTE_BULK 1
+#define MD_PERMUTE_VECTOR 2
+
+int md_set_permute_path(int path);
+
+/*
  * md_dedup_expand -- receiver-side expand of deduplicated rows.
  * "Expert Coupling ...", Method 1 (Deduplicating Dispatcher): a rank receives
  * one row per (token, rank) carrying all of the token's experts on that rank;

@@ -17,6 +17,16 @@ pytestmark = pytest.mark.gpu
 POISON_BITS = 0x7FA1  # a NaN pattern no kernel writes
 
 
+@pytest.fixture(params=[md.MD_PERMUTE_BULK, md.MD_PERMUTE_VECTOR, md.MD_PERMUTE_AUTO],
+                ids=["bulk", "vector", "auto"])
+def permute_path(request):
+    """Run a permute test with each of md_dispatch_permute's kernels (the
+    bulk-copy ring only takes rows of 1 KiB and more)."""
+    md.md_set_permute_path(request.param)
+    yield request.param
+    md.md_set_permute_path(md.MD_PERMUTE_AUTO)
+
+
 def _case(name, T, R=None, H=None, mode=None, seed=0, placement="contiguous"):
     w = synth.make_workload(name, seed=seed, T=T, R=R, H=H, mode=mode)
     k, E = w.k, w.E
@@ -39,7 +49,7 @@ CASES = [("iid_e64_k6", 4096, None, None, 0), ("zipf_pairs_e128_k8", 4096, None,
 
 
 @pytest.mark.parametrize("name,T,R,H,mode", CASES)
-def test_permute_matches_oracle(name, T, R, H, mode):
+def test_permute_matches_oracle(name, T, R, H, mode, permute_path):
     w, idx, gates, p, L = _case(name, T, R, H, mode, placement="shuffled")
     n = L["n_rows"]
     cap = n + 5
@@ -85,7 +95,7 @@ def test_combine_wire_matches_oracle(name, T, R, H):
 
 
 @pytest.mark.parametrize("k", [1, 3, 5, 12, 32])
-def test_generic_k(k):
+def test_generic_k(k, permute_path):
     # k values without a specialised kernel (and k = 1)
     T, E, R, H = 256, 64, 4, 40
     lg = synth.normal_f32(T, E, k, 1).numpy()
@@ -113,7 +123,7 @@ def test_generic_k(k):
 # (5 has no specialised kernel)
 @pytest.mark.parametrize("H", [504, 512, 2056, 4104])
 @pytest.mark.parametrize("k", [2, 5, 8, 32])
-def test_permute_row_pieces(H, k):
+def test_permute_row_pieces(H, k, permute_path):
     T, E, R = 300, 64, 4
     idx = oracle.route_topk(synth.normal_f32(T, E, H + k, 1).numpy(), k)[0]
     L = oracle.dispatch_layout(idx, E, R, shuffled_placement(E, R, 6), 1)
@@ -130,7 +140,7 @@ def test_permute_row_pieces(H, k):
 
 
 @pytest.mark.parametrize("H", [16, 1024])
-def test_bad_rows_are_skipped_and_reported(H):
+def test_bad_rows_are_skipped_and_reported(H, permute_path):
     T, k = 64, 2
     x = synth.normal_bf16(T, H, 0, 3).to(DEV)
     rows = torch.arange(T * k, dtype=torch.int32, device=DEV).view(T, k)
@@ -159,6 +169,12 @@ def test_gather_rows():
     ids = torch.randint(0, 50, (T, 6), dtype=torch.int32, device=DEV)  # 24-byte rows
     got2 = md.md_gather_rows(ids, perm)
     assert torch.equal(got2, ids[perm.long()])
+
+
+def test_permute_path_selector_rejects_unknown_values():
+    with pytest.raises(md.MoeDispatchError):
+        md.md_set_permute_path(7)
+    md.md_set_permute_path(md.MD_PERMUTE_AUTO)
 
 
 def test_full_size_sampled():
