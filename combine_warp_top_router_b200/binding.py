@@ -44,6 +44,10 @@ _SIGNATURES = {
                                     _P, _P, _P], _I),
     "md_dispatch_permute": ([_P, _L, _I, _I, _P, _L, _P, _P, _P], _I),
     "md_set_permute_path": ([_I], _I),
+    "md_exchange_plan": ([_P, _I, _I, _P, _P], _I),
+    "md_dispatch_exchange": ([_P, _L, _I, _I, _P, _P, _P, _I, _I, _P, _P, _L, _P, _P, _P], _I),
+    "md_combine_partials": ([_P, _L, _P, _P, _P, _L, _I, _I, _P, _P, _P], _I),
+    "md_combine_exchange": ([_P, _L, _I, _I, _P, _P, _I, _I, _P, _P, _P, _P, _P], _I),
     "md_dedup_expand": ([_P, _L, _I, _P, _P, _L, _I, _L, _P, _P, _P], _I),
     "md_combine": ([_P, _L, _P, _P, _P, _L, _I, _I, _I, _P, _L, _P, _P, _P, _P], _I),
     "md_coselect_stats": ([_P, _P, _L, _I, _I, _P, _P, _I, _P, _P], _I),
@@ -560,6 +564,129 @@ def md_token_shuffle_pair(idx_prev, idx_l, C, C2, expert_to_rank_next, R, min_ob
                                      _stream(stream, dev))
     _check(rc, "md_token_shuffle_pair")
     return pred_rank, perm, inv, use_pair
+
+
+# ------------------------------------------------------- EP exchange
+
+class md_peer_rows(ctypes.Structure):
+    """One rank's exchange buffers as this rank addresses them (include/moedispatch.h)."""
+    _fields_ = [("rows", ctypes.c_void_p), ("token", ctypes.c_void_p),
+                ("slot_idx", ctypes.c_void_p), ("slot_w", ctypes.c_void_p),
+                ("row_base", ctypes.c_int64), ("rows_cap", ctypes.c_int64)]
+
+
+@dataclass
+class PeerRows:
+    """Buffers of one destination rank: tensors on this device, or raw device
+    addresses (ints) of another GPU's memory mapped into this process."""
+    rows: object
+    row_base: int
+    rows_cap: int
+    token: object = None
+    slot_idx: object = None
+    slot_w: object = None
+
+
+def _addr(v):
+    if v is None:
+        return None
+    if isinstance(v, torch.Tensor):
+        return v.data_ptr()
+    return int(v)
+
+
+def _peer_table(peers):
+    arr = (md_peer_rows * len(peers))()
+    for i, q in enumerate(peers):
+        arr[i] = md_peer_rows(_addr(q.rows), _addr(q.token), _addr(q.slot_idx), _addr(q.slot_w),
+                              int(q.row_base), int(q.rows_cap))
+    return arr
+
+
+def md_exchange_plan(src_rank_offsets, me):
+    """(dst_row_base [R], recv_offsets [R+1]) of rank `me` from every source's
+    layout rank_offsets, gathered ([R, R+1], row s = source s), on the host."""
+    rows = [[int(v) for v in r] for r in src_rank_offsets.tolist()] \
+        if hasattr(src_rank_offsets, "tolist") else [[int(v) for v in r] for r in src_rank_offsets]
+    R = len(rows)
+    if any(len(r) != R + 1 for r in rows):
+        raise ValueError("src_rank_offsets must be [R, R+1]")
+    flat = (ctypes.c_int64 * (R * (R + 1)))(*[v for r in rows for v in r])
+    base = (ctypes.c_int64 * R)()
+    recv = (ctypes.c_int64 * (R + 1))()
+    _check(lib().md_exchange_plan(ctypes.cast(flat, _P), R, int(me), ctypes.cast(base, _P),
+                                  ctypes.cast(recv, _P)), "md_exchange_plan")
+    return list(base), list(recv)
+
+
+def md_dispatch_exchange(x, topk_idx, topk_w, expert_to_rank, E, row_of_slot, rank_offsets,
+                         token_base, peers, dev_status=None, stream=None):
+    """Write this rank's dispatch rows (and their metadata) into the R
+    destination ranks' buffers `peers` (a list of PeerRows)."""
+    _need(x, "x", torch.bfloat16)
+    dev = x.device
+    _need(topk_idx, "topk_idx", torch.int32, dev)
+    if topk_w is not None:
+        _need(topk_w, "topk_w", torch.float32, dev)
+    _need(expert_to_rank, "expert_to_rank", torch.int32, dev)
+    _need(row_of_slot, "row_of_slot", torch.int32, dev)
+    _need(rank_offsets, "rank_offsets", torch.int32, dev)
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    R = len(peers)
+    _room(rank_offsets, "rank_offsets", R + 1)
+    _room(row_of_slot, "row_of_slot", T * k)
+    tab = _peer_table(peers)
+    rc = _call("md_dispatch_exchange", dev, _ptr(x), T, H, k, _ptr(topk_idx), _ptr(topk_w),
+               _ptr(expert_to_rank), E, R, _ptr(row_of_slot), _ptr(rank_offsets), int(token_base),
+               ctypes.cast(tab, _P), _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_dispatch_exchange")
+
+
+def md_combine_partials(y, y_row, slot_idx, slot_w, out=None, dev_status=None, stream=None):
+    """Return rows of a receiving rank: z[i] = bf16(sum over carried slots, by
+    ascending expert, of slot_w * y[y_row])."""
+    _need(y, "y", torch.bfloat16)
+    dev = y.device
+    _need(y_row, "y_row", torch.int32, dev)
+    _need(slot_idx, "slot_idx", torch.int32, dev)
+    _need(slot_w, "slot_w", torch.float32, dev)
+    n, k = y_row.shape
+    H = y.shape[1]
+    if slot_idx.shape != (n, k) or slot_w.shape != (n, k):
+        raise ValueError("y_row, slot_idx and slot_w differ in shape")
+    if out is None:
+        out = torch.empty(n, H, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _room(out, "out", n * H)
+    rc = _call("md_combine_partials", dev, _ptr(y), y.shape[0], _ptr(y_row), _ptr(slot_idx),
+               _ptr(slot_w), n, k, H, _ptr(out), _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_combine_partials")
+    return out
+
+
+def md_combine_exchange(peers, topk_idx, expert_to_rank, E, row_of_slot, rank_offsets, H,
+                        out=None, dev_status=None, stream=None):
+    """out[t] = bf16(fp32 sum, by ascending rank, of the return rows of t read
+    from the R ranks' buffers `peers`)."""
+    _need(topk_idx, "topk_idx", torch.int32)
+    dev = topk_idx.device
+    _need(expert_to_rank, "expert_to_rank", torch.int32, dev)
+    _need(row_of_slot, "row_of_slot", torch.int32, dev)
+    _need(rank_offsets, "rank_offsets", torch.int32, dev)
+    T, k = topk_idx.shape
+    R = len(peers)
+    _room(rank_offsets, "rank_offsets", R + 1)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    _room(out, "out", T * H)
+    tab = _peer_table(peers)
+    rc = _call("md_combine_exchange", dev, ctypes.cast(tab, _P), T, H, k, _ptr(topk_idx),
+               _ptr(expert_to_rank), E, R, _ptr(row_of_slot), _ptr(rank_offsets), _ptr(out),
+               _ptr(dev_status), _stream(stream, dev))
+    _check(rc, "md_combine_exchange")
+    return out
 
 
 # ------------------------------------------------------------ statistics

@@ -448,6 +448,113 @@ int md_gather_rows(const void *src, int64_t src_rows, int64_t row_bytes, const i
                    int64_t n_out, void *dst, int32_t *dev_status, void *stream);
 
 /*
+ * Expert-parallel exchange between real ranks (one process per GPU).
+ * "Expert Coupling ...", The Communication Bottleneck: dispatch and combine
+ * are the two all-to-alls of each MoE layer; Method 1: a dedup row carries
+ * the token's expert IDs and routing probabilities for its rank.  "DODOCO
+ * ...", send_matrices.csv: source s sends send_counts[s][d] rows to rank d,
+ * and combine returns the transposed volumes.
+ *
+ * Each rank lays out its own T_r tokens with md_dispatch_layout (rows
+ * ordered (d, t)); its send row is rank_offsets[d+1] - rank_offsets[d].
+ * After an all-gather of the R rank_offsets (the caller's collective),
+ * md_exchange_plan places this rank's block in every destination: rank d
+ * receives source 0's rows, then source 1's, ...  For MD_DEDUP layouts that
+ * is the (d, global token) order of a single-GPU layout of all tokens; for
+ * MD_CONV the rows arrive by (source, expert, token), and the receiver
+ * groups them by expert for its GEMM (md_dedup_expand or its own order).  The data kernels
+ * write or read the other ranks' buffers through plain device pointers
+ * (peer pointers over NVLink, e.g. from symmetric memory or IPC handles, or
+ * local memory); the caller orders them against the peers (a barrier
+ * before md_combine_exchange reads what the peers wrote).  No load or store
+ * uses multicast.
+ *
+ * md_peer_rows: one rank's buffers as seen by this rank (pointers on the
+ * device, the struct itself in host memory):
+ *   rows      bf16 [rows_cap, H]: dispatch receive rows (md_dispatch_exchange
+ *             writes them) or combine return rows (md_combine_exchange reads)
+ *   token     int32 [rows_cap] or NULL: global token id of each received row
+ *   slot_idx  int32 [rows_cap, k] or NULL: per slot of the token, its expert
+ *             if this row carries it (its expert sits on that rank), else -1
+ *   slot_w    float [rows_cap, k] or NULL: the carried slots' gates, else 0
+ *   row_base  first row of this source's block in those buffers
+ *             (md_exchange_plan's dst_row_base[d])
+ *   rows_cap  rows the buffers hold; a row outside [0, rows_cap) is skipped
+ *             and reported (MD_ERR_DATA)
+ */
+typedef struct md_peer_rows {
+    void *rows;
+    int32_t *token;
+    int32_t *slot_idx;
+    float *slot_w;
+    int64_t row_base;
+    int64_t rows_cap;
+} md_peer_rows;
+
+/*
+ * md_exchange_plan -- host helper (no device work; HOST pointers).
+ *   src_rank_offsets  int64 [R, R+1]: every source rank's rank_offsets from
+ *                     md_dispatch_layout of its own tokens, gathered (row s =
+ *                     source s); source s sends rank_offsets_s[d+1] -
+ *                     rank_offsets_s[d] rows to rank d (its send-matrix row)
+ *   me                this rank
+ *   dst_row_base      int64 [R] out: first row of my block on rank d, the
+ *                     rows all sources before me send to d
+ *   recv_offsets      int64 [R+1] out: first row of source s's block in my
+ *                     receive buffer; [R] = rows I receive
+ *   MD_ERR_DATA for a row that does not start at 0 or decreases.
+ */
+int md_exchange_plan(const int64_t *src_rank_offsets, int R, int me, int64_t *dst_row_base,
+                     int64_t *recv_offsets);
+
+/*
+ * md_dispatch_exchange -- the dispatch all-to-all as one kernel: every
+ * distinct row of each local token (rows shared by slots on one rank, in
+ * an MD_DEDUP layout, travel once) is written bit for bit into its
+ * destination rank's buffer, at peers[d].row_base + (row - rank_offsets[d]),
+ * with its metadata (global token id token_base + t, slot experts, gates).
+ *   x               bf16 [T, H], this rank's tokens
+ *   topk_idx, topk_w  int32 / float [T, k] (topk_w may be NULL: gates 0)
+ *   expert_to_rank  int32 [E]
+ *   row_of_slot, rank_offsets  this rank's md_dispatch_layout of its tokens
+ *   peers           host array of R md_peer_rows (rows required)
+ *   Limits as md_dispatch_layout; H % 8 == 0, 16-byte aligned rows,
+ *   token_base + T <= INT32_MAX.
+ */
+int md_dispatch_exchange(const void *x, int64_t T, int H, int k, const int32_t *topk_idx,
+                         const float *topk_w, const int32_t *expert_to_rank, int E, int R,
+                         const int32_t *row_of_slot, const int32_t *rank_offsets,
+                         int64_t token_base, const md_peer_rows *peers, int32_t *dev_status,
+                         void *stream);
+
+/*
+ * md_combine_partials -- on a receiving rank, the row that returns for each
+ * received row i: z[i] = bf16(sum over the slots j it carries, in ascending
+ * expert id, of slot_w[i][j] * y[y_row[i][j]]), fp32 fused multiply-add
+ * from +0.0f (the first stage of MD_COMBINE_WIRE).
+ *   y          bf16 [y_rows, H]: this rank's expert outputs
+ *   y_row      int32 [n, k]: row of y holding slot j's expert output, or -1
+ *              for a slot this row does not carry
+ *   slot_idx, slot_w  int32 / float [n, k] as received
+ *   z          bf16 [n, H] out
+ */
+int md_combine_partials(const void *y, int64_t y_rows, const int32_t *y_row,
+                        const int32_t *slot_idx, const float *slot_w, int64_t n, int k, int H,
+                        void *z, int32_t *dev_status, void *stream);
+
+/*
+ * md_combine_exchange -- the combine all-to-all as one kernel: for each local
+ * token, the return rows of its ranks are read from the peers' buffers
+ * (peers[d].rows at the same rows md_dispatch_exchange wrote) and
+ * out[t] = bf16(fp32 sum of them in ascending rank) (the second stage of
+ * MD_COMBINE_WIRE).  With an MD_DEDUP layout a token has one row per rank.
+ *   out  bf16 [T, H]; other arguments as md_dispatch_exchange.
+ */
+int md_combine_exchange(const md_peer_rows *peers, int64_t T, int H, int k, const int32_t *topk_idx,
+                        const int32_t *expert_to_rank, int E, int R, const int32_t *row_of_slot,
+                        const int32_t *rank_offsets, void *out, int32_t *dev_status, void *stream);
+
+/*
  * Routing statistics ("Expert Coupling ...").
  *
  * md_rank_stats -- Table I (Offline Placement and Prediction Statistics):

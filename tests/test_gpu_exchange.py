@@ -1,0 +1,146 @@
+"""The EP exchange kernels on one GPU, every rank played in turn.
+
+Each source rank s lays out its own block of T/R tokens (md_dispatch_layout),
+the plan places its block in every destination, md_dispatch_exchange writes
+its rows into R separate destination buffers, every destination forms its
+return rows with md_combine_partials from what it received, and
+md_combine_exchange gathers each source's tokens back from the R buffers.
+On one GPU all R buffers are local allocations; across GPUs they are the
+peers' memory and the kernels are the same.
+
+Expected values come from the oracle's single-GPU layout of all T tokens:
+destination d's buffer must hold, bit for bit, the rows [rank_offsets[d],
+rank_offsets[d+1]) of the oracle's dedup dispatch buffer, with their token
+ids and slot metadata; the return rows must equal the oracle's wire partials
+of those rows, and the combined outputs the oracle's wire combine."""
+import numpy as np
+import pytest
+import torch
+
+import combine_warp_top_router_b200 as md
+import oracle
+from combine_warp_top_router_b200 import synth
+
+from _util import DEV, bits, f32, from_bits, i32, shuffled_placement
+
+pytestmark = pytest.mark.gpu
+
+POISON = 0x7FA1
+
+
+def _run(name, T, R, H, placement, seed=0):
+    w = synth.make_workload(name, seed=seed, T=T, R=R, H=H)
+    E, k = w.E, w.k
+    oi, ow = oracle.route_topk(w.logits.numpy(), k)
+    p = w.expert_to_rank.numpy() if placement == "contiguous" else shuffled_placement(E, R, 4)
+    G = oracle.dispatch_layout(oi, E, R, p, oracle.DEDUP)
+    Tr = T // R
+    x = w.x.to(DEV)
+    y = w.y.to(DEV)
+    pg = i32(p)
+    idx = i32(oi)
+    gates = f32(ow)
+
+    # 1. every source lays out its own tokens
+    local = [md.md_dispatch_layout(idx[s * Tr:(s + 1) * Tr].contiguous(), E, R, pg, md.MD_DEDUP)
+             for s in range(R)]
+    gathered = torch.stack([L.rank_offsets for L in local]).cpu().to(torch.int64)
+    plans = [md.md_exchange_plan(gathered, s) for s in range(R)]
+    caps = [plans[d][1][R] for d in range(R)]
+    # the receive sizes are the global layout's rank blocks
+    assert caps == list(np.diff(G["rank_offsets"]))
+
+    # 2. receive buffers of every destination, poisoned
+    recv = [from_bits(np.full((caps[d] + 2, H), POISON, np.uint16)) for d in range(R)]
+    tok = [torch.full((caps[d] + 2,), -9, dtype=torch.int32, device=DEV) for d in range(R)]
+    sidx = [torch.full((caps[d] + 2, k), -9, dtype=torch.int32, device=DEV) for d in range(R)]
+    sw = [torch.full((caps[d] + 2, k), -9.0, dtype=torch.float32, device=DEV) for d in range(R)]
+    st = md.new_status(DEV)
+    for s in range(R):
+        base = plans[s][0]
+        peers = [md.PeerRows(rows=recv[d], token=tok[d], slot_idx=sidx[d], slot_w=sw[d],
+                             row_base=base[d], rows_cap=caps[d]) for d in range(R)]
+        sl = slice(s * Tr, (s + 1) * Tr)
+        md.md_dispatch_exchange(x[sl], idx[sl].contiguous(), gates[sl].contiguous(), pg, E,
+                                local[s].row_of_slot, local[s].rank_offsets, s * Tr, peers,
+                                dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == md.MD_OK
+    want_rows = oracle.dispatch_permute(bits(w.x), G["row_token"])
+    ro = G["rank_offsets"]
+    for d in range(R):
+        seg = slice(ro[d], ro[d + 1])
+        got = bits(recv[d])
+        assert np.array_equal(got[:caps[d]], want_rows[seg])
+        assert np.all(got[caps[d]:] == POISON)
+        assert np.array_equal(tok[d][:caps[d]].cpu().numpy(), G["row_token"][seg])
+        assert np.all(tok[d][caps[d]:].cpu().numpy() == -9)
+        mask = G["row_mask"][seg]
+        carried = ((mask[:, None] >> np.arange(k)[None, :]) & 1).astype(bool)
+        t_of = G["row_token"][seg]
+        assert np.array_equal(sidx[d][:caps[d]].cpu().numpy(), np.where(carried, oi[t_of], -1))
+        assert np.array_equal(sw[d][:caps[d]].cpu().numpy(), np.where(carried, ow[t_of], 0.0))
+
+    # 3. every destination forms its return rows from what it received; its
+    # expert outputs are the conventional rows of y (identity mapping here)
+    _, want_z = oracle.combine(bits(w.y), G["assign_row"], oi, ow, oracle.COMBINE_WIRE, p,
+                               G["row_of_slot"], G["n_rows"])
+    ret = []
+    for d in range(R):
+        seg = slice(ro[d], ro[d + 1])
+        mask = G["row_mask"][seg]
+        carried = ((mask[:, None] >> np.arange(k)[None, :]) & 1).astype(bool)
+        y_row = np.where(carried, G["assign_row"][G["row_token"][seg]], -1).astype(np.int32)
+        z = md.md_combine_partials(y, i32(y_row), sidx[d][:caps[d]].contiguous(),
+                                   sw[d][:caps[d]].contiguous(), dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == md.MD_OK
+        assert np.array_equal(bits(z), want_z[seg])
+        ret.append(z)
+
+    # 4. every source gathers its tokens' return rows and sums them
+    want_out, _ = oracle.combine(bits(w.y), G["assign_row"], oi, ow, oracle.COMBINE_WIRE, p,
+                                 G["row_of_slot"], G["n_rows"])
+    for s in range(R):
+        base = plans[s][0]
+        peers = [md.PeerRows(rows=ret[d], row_base=base[d], rows_cap=caps[d]) for d in range(R)]
+        sl = slice(s * Tr, (s + 1) * Tr)
+        out = md.md_combine_exchange(peers, idx[sl].contiguous(), pg, E, local[s].row_of_slot,
+                                     local[s].rank_offsets, H, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == md.MD_OK
+        assert np.array_equal(bits(out), want_out[sl])
+
+
+@pytest.mark.parametrize("name,T,R,H,placement", [
+    ("zipf_pairs_e128_k8", 4096, 16, 2048, "contiguous"),
+    ("boost_pairs_e128_k2", 2048, 8, 4096, "shuffled"),
+    ("full_e256_k8", 4096, 64, 256, "shuffled"),
+    ("two_layer_e128_k6", 16 * 48, 16, 264, "shuffled"),   # k = 6 (generic kernel), odd H
+])
+def test_exchange_matches_single_gpu_oracle(name, T, R, H, placement):
+    _run(name, T, R, H, placement)
+
+
+def test_exchange_reports_rows_outside_the_buffers():
+    # a destination buffer one row too small: that row is skipped and reported
+    name, T, R, H = "zipf_pairs_e128_k8", 512, 4, 64
+    w = synth.make_workload(name, T=T, R=R, H=H)
+    E, k = w.E, w.k
+    oi, ow = oracle.route_topk(w.logits.numpy(), k)
+    pg = i32(w.expert_to_rank.numpy())
+    L = md.md_dispatch_layout(i32(oi), E, R, pg, md.MD_DEDUP)
+    ro = L.rank_offsets.cpu().numpy()
+    caps = list(np.diff(ro))
+    bufs = [torch.zeros(max(c, 1), H, dtype=torch.bfloat16, device=DEV) for c in caps]
+    peers = [md.PeerRows(rows=bufs[d], row_base=0, rows_cap=caps[d] - (1 if d == 2 else 0))
+             for d in range(R)]
+    st = md.new_status(DEV)
+    md.md_dispatch_exchange(w.x.to(DEV), i32(oi), f32(ow), pg, E, L.row_of_slot, L.rank_offsets, 0,
+                            peers, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == md.MD_ERR_DATA
+    # every row that fits still landed
+    rows = oracle.dispatch_permute(bits(w.x), L.row_token[:ro[R]].cpu().numpy())
+    assert np.array_equal(bits(bufs[0])[:caps[0]], rows[ro[0]:ro[1]])
+    assert np.array_equal(bits(bufs[2])[:caps[2] - 1], rows[ro[2]:ro[3] - 1])
