@@ -246,14 +246,16 @@ void launch_k(const float *logits, int64_t T, int E, int k, int gate_mode, int32
 // ---------------------------------------------------------------- thread per token
 // E in {64, 128, 256}, k in {1, 2, 4, 6, 8}: one thread per token, so the
 // selection needs no cross-lane steps.  A warp stages its 32 consecutive rows
-// (contiguous in memory) in shared memory with 16-byte async copies.  Lane L
-// reads its row's 16-byte chunks in the order (c + L) mod E/4, which puts the
-// 8 lanes of a shared-memory phase on distinct banks.
+// (contiguous in memory) in shared memory with one bulk copy.  Lane L reads
+// its row's 16-byte chunks in the order (c + L) mod E/4, which puts the 8
+// lanes of a shared-memory phase on distinct banks.
 //   1. Threshold.  Chunk iteration c belongs to group c mod 16; the k-th
 //      largest of the 16 group maxima is at or below the k-th largest logit
 //      (k group maxima are k distinct elements at or above it).
-//   2. Candidates.  Elements at or above the threshold (about 10 for k = 8)
-//      are compacted into a per-lane list of expert indices.
+//   2. Candidates.  Only groups whose maximum reaches the threshold (k or a
+//      few more of the 16) are read again; their elements at or above it
+//      (about 10 for k = 8) are compacted into a per-lane list of expert
+//      indices.
 //   3. Selection.  Candidates become exact 64-bit keys (order-preserving
 //      logit key, then the complement of the expert index, so that equal
 //      logits go to the lower index).  Batches of 8 are sorted by a 19-
@@ -262,14 +264,7 @@ void launch_k(const float *logits, int64_t T, int E, int k, int gate_mode, int32
 //      as a bitonic sequence, which a 12-comparator bitonic merge sorts.
 // The gates are computed as in the warp kernel, one token per thread.
 constexpr int kTptGroups = 16;
-
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(md::smem_addr(dst_smem)), "l"(src)
-                 : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+constexpr long long kTptPolls = 1ll << 22;
 
 // descending compare-exchange
 __device__ __forceinline__ void cx(uint64_t &a, uint64_t &b)
@@ -321,7 +316,8 @@ constexpr size_t tpt_smem() { return (size_t)32 * E * 4 + (size_t)32 * E; }
 template <int E, int KC>
 __global__ void __launch_bounds__(32)
     k_route_topk_tpt(const float *__restrict__ logits, int64_t T, int gate_mode,
-                     int32_t *__restrict__ out_idx, float *__restrict__ out_w, int vec_out)
+                     int32_t *__restrict__ out_idx, float *__restrict__ out_w, int vec_out,
+                     long long polls)
 {
     constexpr int NCH = E / 4;
     constexpr int NG = kTptGroups;
@@ -333,10 +329,30 @@ __global__ void __launch_bounds__(32)
     const int64_t t0 = (int64_t)blockIdx.x * 32;
     const int ntok = (int)(T - t0 < 32 ? T - t0 : 32);
     {
-        const float4 *src = reinterpret_cast<const float4 *>(logits + t0 * E);
-        float4 *dst = reinterpret_cast<float4 *>(rows);
-        for (int i = lane; i < ntok * NCH; i += 32) cp_async16(dst + i, src + i);
-        cp_async_wait_all();
+        // the tile's rows are contiguous: one bulk copy, completing on an
+        // mbarrier every lane waits on (bounded; if the bound runs out, the
+        // lanes copy the same bytes with plain loads, so a late bulk copy can
+        // only rewrite identical values)
+        __shared__ uint64_t bar;
+        const uint32_t bytes = (uint32_t)(ntok * E * 4);
+        if (lane == 0) {
+            md::mbar_init(&bar, 1);
+            md::fence_mbar_init();
+        }
+        __syncwarp();
+        if (lane == 0) {
+            md::mbar_expect_tx(&bar, bytes);
+            md::bulk_load(rows, logits + t0 * E, bytes, &bar);
+        }
+        const bool ok = md::mbar_wait_bounded(&bar, 0u, polls);
+        if (!__all_sync(0xffffffffu, ok)) {
+            const float4 *src = reinterpret_cast<const float4 *>(logits + t0 * E);
+            float4 *dst = reinterpret_cast<float4 *>(rows);
+            for (int i = lane; i < ntok * NCH; i += 32) dst[i] = __ldg(src + i);
+            // let the late copy land (bounded again, at the default limit)
+            // before the rows are read, so it cannot arrive after the CTA
+            md::mbar_wait_bounded(&bar, 0u, kTptPolls);
+        }
         __syncwarp();
     }
     const bool live = lane < ntok;
@@ -366,15 +382,25 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
         for (int i = 1; i < KC; ++i) th = fmaxf(th, fminf(a[i - 1], b[KC - i - 1]));
 
+        // only a group whose maximum reaches the threshold can hold a
+        // candidate: k or a few more of the 16, so about half the chunks
+        uint32_t gmask = 0u;
 #pragma unroll
-        for (int c = 0; c < NCH; ++c) {
-            const int ch = (c + lane) & (NCH - 1);
-            const float4 q = row4[ch];
-            const int e0 = ch * 4;
-            if (q.x >= th) { lst[32 * n] = (uint8_t)e0; ++n; }
-            if (q.y >= th) { lst[32 * n] = (uint8_t)(e0 + 1); ++n; }
-            if (q.z >= th) { lst[32 * n] = (uint8_t)(e0 + 2); ++n; }
-            if (q.w >= th) { lst[32 * n] = (uint8_t)(e0 + 3); ++n; }
+        for (int g = 0; g < NG; ++g)
+            if (gm[g] >= th) gmask |= 1u << g;
+        while (gmask) {
+            const int g = __ffs(gmask) - 1;
+            gmask &= gmask - 1;
+#pragma unroll
+            for (int j = 0; j < NCH / NG; ++j) {  // iterations g, g + 16, ... of the first pass
+                const int ch = (g + NG * j + lane) & (NCH - 1);
+                const float4 q = row4[ch];
+                const int e0 = ch * 4;
+                if (q.x >= th) { lst[32 * n] = (uint8_t)e0; ++n; }
+                if (q.y >= th) { lst[32 * n] = (uint8_t)(e0 + 1); ++n; }
+                if (q.z >= th) { lst[32 * n] = (uint8_t)(e0 + 2); ++n; }
+                if (q.w >= th) { lst[32 * n] = (uint8_t)(e0 + 3); ++n; }
+            }
         }
         // fewer than k candidates happens only with NaN logits (outside the
         // contract): take every element, so the indices stay valid and distinct
@@ -420,7 +446,8 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
     for (int r = 0; r < KC; ++r) {
         sel[r] = (int)(0xffffu - (uint32_t)(best[r] & 0xffffffffu));
-        ex[r] = exp((double)key_float((uint32_t)(best[r] >> 32)) - m);
+        // slot 0 holds the largest logit m itself: exp(0) = 1 exactly
+        ex[r] = r == 0 ? 1.0 : exp((double)key_float((uint32_t)(best[r] >> 32)) - m);
         den += ex[r];
     }
     if (gate_mode == MD_GATE_FULL_SOFTMAX) {
@@ -432,9 +459,12 @@ __global__ void __launch_bounds__(32)
                    exp((double)q.w - m);
         }
     }
+    // one reciprocal; each quotient stays within a double ulp or two of
+    // ex / den before its single rounding to float
+    const double inv = 1.0 / den;
     float w[KC];
 #pragma unroll
-    for (int r = 0; r < KC; ++r) w[r] = (float)(ex[r] / den);
+    for (int r = 0; r < KC; ++r) w[r] = (float)(ex[r] * inv);
     if (vec_out && KC % 4 == 0) {
 #pragma unroll
         for (int q = 0; q < KC / 4; ++q) {
@@ -462,7 +492,8 @@ void launch_tpt(const float *logits, int64_t T, int gate_mode, int32_t *idx, flo
     });
     const int vec = md::aligned16(idx) && md::aligned16(w);
     const int64_t blocks = (T + 31) / 32;
-    k_route_topk_tpt<E, KC><<<(unsigned)blocks, 32, tpt_smem<E>(), s>>>(logits, T, gate_mode, idx, w, vec);
+    k_route_topk_tpt<E, KC><<<(unsigned)blocks, 32, tpt_smem<E>(), s>>>(logits, T, gate_mode, idx, w, vec,
+                                                                       md::hook_poll_limit(kTptPolls));
     md::count_launches(1);
 }
 

@@ -609,7 +609,8 @@ int md_pearson_from_sums(const uint64_t *sums, int64_t n, double *r);
  * md_set_test_hooks -- fault injection for tests; not for production use.
  * Every bounded device-side wait gives up after a poll limit and reports
  * MD_ERR_TIMEOUT.  These hooks make such a wait run out on purpose, with no
- * fault: poll_limit > 0 replaces the default limits; layout_skip_tile >= 0
+ * fault: poll_limit > 0 replaces the default limits (md_route_topk then may
+ * fall back to plain loads for a tile, with the same results); layout_skip_tile >= 0
  * makes that md_dispatch_layout CTA stamp no arrival word, so every CTA
  * waits for it in vain; expand_skip_unit >= 0 makes md_dedup_expand (bulk-copy
  * path) never fill that unit's shared-memory slot.  (0, -1, -1) restores the

@@ -133,3 +133,18 @@ def test_nan_rows_give_valid_distinct_experts(E, k):
     # rows without NaN are unaffected
     oi, _ = oracle.route_topk(lg[4:], k, 0)
     assert np.array_equal(gi[4:], oi)
+
+
+@pytest.mark.parametrize("E,k", [(64, 6), (128, 8), (256, 8), (256, 2)])
+def test_bounded_tile_wait_fallback_is_exact(E, k):
+    # The per-token kernel stages each 32-row tile with one bulk copy and a
+    # bounded wait; when the bound runs out it copies the same bytes with
+    # plain loads.  A poll limit of 1 makes that path likely; either way the
+    # result must be the oracle's.
+    lg = synth.normal_f32(4096 + 17, E, E + k, 1).numpy()
+    md.md_set_test_hooks(poll_limit=1)
+    try:
+        _compare(lg, k, 0)
+    finally:
+        md.md_set_test_hooks()
+    _compare(lg, k, 1)
