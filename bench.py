@@ -382,7 +382,99 @@ def run_rows(args, md, device, stream, peak):
     rows.update(rows_config3(args, md, device, stream, peak))
     rows.update(rows_config4(args, md, device, stream, peak))
     rows.update(rows_config5_planning(args, md, device, stream, peak))
+    rows.update(rows_ep_exchange(args, md, device, stream, peak))
     return rows
+
+
+def rows_ep_exchange(args, md, device, stream, peak):
+    """The EP exchange kernels on one GPU: config 2's workload split into its
+    16 source ranks of 4096 tokens, each laid out on its own; the dispatch
+    exchange writes every source's rows into 16 separate destination buffers,
+    every destination forms its return rows, and the combine exchange reads
+    them back.  Across GPUs the same kernels store to and load from the peers'
+    memory over NVLink; here every buffer is local, so this times the
+    kernels' HBM side."""
+    from combine_warp_top_router_b200 import synth
+    reps = max(3, args.row_reps // 4)
+    w = synth.make_workload("zipf_pairs_e128_k8", seed=args.seed, device=device)
+    T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
+    Tr = T // R
+    idx, gates = md.md_route_topk(w.logits, k)
+    p = w.expert_to_rank
+    local = [md.md_dispatch_layout(idx[s * Tr:(s + 1) * Tr], E, R, p, md.MD_DEDUP) for s in range(R)]
+    gathered = torch.stack([L.rank_offsets for L in local]).cpu().to(torch.int64)
+    plans = [md.md_exchange_plan(gathered, s) for s in range(R)]
+    caps = [plans[d][1][R] for d in range(R)]
+    recv = [torch.empty(max(c, 1), H, dtype=torch.bfloat16, device=device) for c in caps]
+    tok = [torch.empty(max(c, 1), dtype=torch.int32, device=device) for c in caps]
+    sidx = [torch.empty(max(c, 1), k, dtype=torch.int32, device=device) for c in caps]
+    sw = [torch.empty(max(c, 1), k, dtype=torch.float32, device=device) for c in caps]
+    G = md.md_dispatch_layout(idx, E, R, p, md.MD_DEDUP)   # the receivers' expert rows
+    ro = G.rank_offsets.cpu().tolist()
+    y_row = [torch.empty(max(c, 1), k, dtype=torch.int32, device=device) for c in caps]
+    # receiver d's expert-output row of each carried slot (identity mapping
+    # onto y's conventional rows; built once, outside the timing)
+    carried = (G.row_mask[:ro[R]].view(-1, 1) >> torch.arange(k, device=device).view(1, -1)) & 1
+    yr_all = torch.where(carried.bool(), G.assign_row[G.row_token[:ro[R]].long()], -1).to(torch.int32)
+    for d in range(R):
+        y_row[d][:caps[d]].copy_(yr_all[ro[d]:ro[d + 1]])
+    ret = [torch.empty(max(c, 1), H, dtype=torch.bfloat16, device=device) for c in caps]
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=device)
+    dpeers = [[md.PeerRows(rows=recv[d], token=tok[d], slot_idx=sidx[d], slot_w=sw[d],
+                           row_base=plans[s][0][d], rows_cap=caps[d]) for d in range(R)]
+              for s in range(R)]
+    cpeers = [[md.PeerRows(rows=ret[d], row_base=plans[s][0][d], rows_cap=caps[d]) for d in range(R)]
+              for s in range(R)]
+
+    # the calls enqueue on the current stream; each phase's 16 calls are
+    # captured in a CUDA graph and replayed, so host marshalling stays out of
+    # the timed region (16 small launches per phase would otherwise leave the
+    # GPU waiting on the host)
+    def dispatch():
+        for s_ in range(R):
+            sl = slice(s_ * Tr, (s_ + 1) * Tr)
+            md.md_dispatch_exchange(w.x[sl], idx[sl], gates[sl], p, E, local[s_].row_of_slot,
+                                    local[s_].rank_offsets, s_ * Tr, dpeers[s_])
+
+    def partials():
+        for d in range(R):
+            md.md_combine_partials(w.y, y_row[d][:caps[d]], sidx[d][:caps[d]], sw[d][:caps[d]],
+                                   out=ret[d][:caps[d]])
+
+    def combine():
+        for s_ in range(R):
+            sl = slice(s_ * Tr, (s_ + 1) * Tr)
+            md.md_combine_exchange(cpeers[s_], idx[sl], p, E, local[s_].row_of_slot,
+                                   local[s_].rank_offsets, H, out=out[sl])
+
+    def graphed(fn):
+        torch.cuda.synchronize()
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    graphs = [graphed(f) for f in (dispatch, partials, combine)]
+    t_d, t_p, t_c = (_time(g.replay, stream, reps) for g in graphs)
+    del graphs
+    n = sum(caps)
+    # dispatch: x once, each row written once with its metadata (4 + 8k B)
+    db = T * (2 * H + 12 * k) + n * (2 * H + 4 + 8 * k)
+    # partials: the carried slots' expert rows and metadata in, one row out
+    pb = T * k * 2 * H + n * (12 * k + 2 * H)
+    # combine: each return row read once, one row out per token
+    cb = n * 2 * H + T * (2 * H + 8 * k)
+    r = {"T": T, "ranks": R, "tokens_per_rank": Tr, "rows_per_token": round(n / T, 4),
+         "dispatch_exchange_us": round(t_d * 1e3, 1), "dispatch_exchange": gbps(db, t_d, peak),
+         "combine_partials_us": round(t_p * 1e3, 1), "combine_partials": gbps(pb, t_p, peak),
+         "combine_exchange_us": round(t_c * 1e3, 1), "combine_exchange": gbps(cb, t_c, peak),
+         "note": "16 calls of each kernel (one per source or destination rank), replayed from a "
+                 "CUDA graph; all buffers on this GPU"}
+    del w, recv, tok, sidx, sw, ret, out, y_row, local, G
+    torch.cuda.empty_cache()
+    return {"ep_exchange_zipf_pairs_e128_k8": r}
 
 
 def rows_config2(args, md, device, stream, peak):
@@ -439,9 +531,11 @@ def rows_config2(args, md, device, stream, peak):
 
 
 def rows_config1(args, md, device, stream, peak):
-    """iid_e64_k6 (T=4096, 117 MB per kernel, about the size of L2): every
-    step is timed on its own with L2 flushed before it (a write of twice the
-    L2 size), and the median over the steps is reported."""
+    """iid_e64_k6 (T=4096, 117 MB per kernel, about the size of L2): L2 is
+    flushed (a write of twice its size) before every timed launch, and medians
+    are reported.  Each kernel, and the whole step, is captured in a CUDA graph
+    and replayed right after the flush, so the host's marshalling of the four
+    calls does not leave the GPU idle inside the timed region."""
     from combine_warp_top_router_b200 import synth
     w = synth.make_workload("iid_e64_k6", seed=args.seed, device=device)
     T, H, E, k, R = w.T, w.H, w.E, w.k, w.R
@@ -456,40 +550,53 @@ def rows_config1(args, md, device, stream, peak):
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
     parts = ("route_topk", "dispatch_layout", "dispatch_permute", "combine")
     calls = (
-        lambda: md.md_route_topk(w.logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates, stream=stream),
-        lambda: md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp,
-                                      stream=stream),
-        lambda: md.md_dispatch_permute(w.x, L.row_of_slot, out=buf, stream=stream),
-        lambda: md.md_combine(w.y, L.assign_row, idx, gates, out=out, stream=stream),
+        lambda: md.md_route_topk(w.logits, k, md.MD_GATE_TOPK_SOFTMAX, idx, gates),
+        lambda: md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode, out=L, workspace=wsp),
+        lambda: md.md_dispatch_permute(w.x, L.row_of_slot, out=buf),
+        lambda: md.md_combine(w.y, L.assign_row, idx, gates, out=out),
     )
-    torch.cuda.synchronize()
-    times = {n: [] for n in parts + ("step",)}
+
+    def graphed(fns):
+        torch.cuda.synchronize()
+        for f in fns:
+            f()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for f in fns:
+                f()
+        return g
+
+    graphs = {n: graphed([c]) for n, c in zip(parts, calls)}
+    graphs["step"] = graphed(calls)
     n_steps = max(20, args.row_reps)
+    times = {n: [] for n in graphs}
+    torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for i in range(3 + n_steps):
-            flush.fill_(i & 0xff)
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
-            ev[0].record(stream)
-            for j, c in enumerate(calls):
-                c()
-                ev[j + 1].record(stream)
-            stream.synchronize()
-            if i >= 3:
-                for j, n in enumerate(parts):
-                    times[n].append(ev[j].elapsed_time(ev[j + 1]))
-                times["step"].append(ev[0].elapsed_time(ev[-1]))
+            for name, g in graphs.items():
+                flush.fill_(i & 0xff)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                stream.synchronize()
+                if i >= 3:
+                    times[name].append(e0.elapsed_time(e1))
     med = {n: statistics.median(v) for n, v in times.items()}
     n = int(L.n_rows.item())
     ab = algorithmic_bytes(T, H, k, E, n)
     r = {"T": T, "H": H, "E": E, "top_k": k, "ep_ranks": R, "dispatch": "conv",
-         "placement": "contiguous", "l2": f"flushed before every step ({2 * l2 >> 20} MiB write)",
+         "placement": "contiguous", "l2": f"flushed before every timed launch ({2 * l2 >> 20} MiB write)",
+         "timing": "CUDA graph replay per kernel and per step; medians",
          "steps": n_steps, "median_step_us": round(med["step"] * 1e3, 2),
          "Mtokens_per_s": round(T / (med["step"] * 1e-3) / 1e6, 2),
          "dispatch_combine_excl_router": round(
              T / ((med["dispatch_layout"] + med["dispatch_permute"] + med["combine"]) * 1e-3) / 1e6, 2)}
     for nme in parts:
         r[nme] = {"us": round(med[nme] * 1e3, 2), **gbps(ab[nme], med[nme], peak)}
-    del w, idx, gates, L, wsp, buf, out, flush
+    del graphs, w, idx, gates, L, wsp, buf, out, flush
     torch.cuda.empty_cache()
     return {"iid_e64_k6_l2_flushed": r}
 

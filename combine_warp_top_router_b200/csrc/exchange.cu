@@ -23,13 +23,18 @@
 //   dispatch  one warp per token: the token's distinct rows, each written
 //             once into its destination rank's buffer with 16-byte stores,
 //             with the token's global id and, per slot carried by the row,
-//             the expert ID (-1 for slots of other ranks) and its gate.
+//             the expert ID (-1 for slots of other ranks) and its gate; the
+//             next token's row and slot data load while the current token's
+//             rows are stored.
 //   partials  on the receiver, one warp per received row: the gate-weighted
 //             sum of its slots' expert outputs in ascending expert order,
 //             fp32 FMA, one bf16 rounding -- the row that travels back.
 //   combine   one warp per token: the bf16 partial rows of the token's
 //             ranks, read from the peers in ascending rank, summed in fp32,
 //             one bf16 rounding.
+// The combine issues all of a token's return rows before it adds (a token
+// has several), so about 8 16-byte loads per lane are in flight; the partials
+// take the few slots of a received row one after another.
 // No load or store here uses multicast; peers are plain pointers.
 #include <climits>
 
@@ -54,6 +59,11 @@ int grid_warps(int64_t units)
 }
 
 // --------------------------------------------------------------- dispatch
+// One warp per token, the vector permute's pipeline: a pass moves kU 16-byte
+// chunks per lane (4 KiB of the row); while the current token's rows are
+// stored, the next token's chunks and slot data are already in flight.  Rows
+// longer than 4 KiB take one pass over the warp's tokens per 4 KiB block;
+// the metadata is written in the first.
 template <int KC>
 __global__ void __launch_bounds__(kThreads)
     k_dispatch_exchange(const uint4 *__restrict__ x, int64_t T, int C, int k,
@@ -65,38 +75,58 @@ __global__ void __launch_bounds__(kThreads)
 {
     const int K = KC ? KC : k;
     const int lane = threadIdx.x & 31;
+    const int64_t w0 = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
-    for (int64_t t = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; t < T; t += nw) {
-        int r = -1, e = -1, d = -1;
-        float ww = 0.0f;
-        if (lane < K) {
+    if (w0 >= T) return;
+    auto slot = [&](int64_t t, int &r, int &e, float &ww) {
+        r = -1;
+        e = -1;
+        ww = 0.0f;
+        if (t < T && lane < K) {
             r = __ldg(row_of_slot + t * K + lane);
             e = __ldg(idx + t * K + lane);
             ww = w ? __ldg(w + t * K + lane) : 0.0f;
-            d = (e >= 0 && e < E) ? __ldg(p_g + e) : -1;
-            if (d >= R) d = -1;
         }
-        // slots sharing a row travel in it once; the row's slot mask is the group
-        const unsigned g = __match_any_sync(0xffffffffu, lane < K ? (unsigned)r : (0x80000000u | lane));
-        const bool first = lane < K && (g & md::lanemask_lt()) == 0u;
-        int64_t dst = -1;
-        if (first && d >= 0) {
-            const int lo = __ldg(rank_offsets + d), hi = __ldg(rank_offsets + d + 1);
-            if (r >= lo && r < hi) {
-                dst = pt.p[d].row_base + (r - lo);
-                if (dst < 0 || dst >= pt.p[d].rows_cap) dst = -1;
-            }
-        }
-        if (first && dst < 0) md::report(status, MD_ERR_DATA);
-        const unsigned rows = __ballot_sync(0xffffffffu, first && dst >= 0);
-        // the row once from HBM, kU chunks per lane at a time, into every destination
-        for (int c0 = 0; c0 < C; c0 += 32 * kU) {
-            uint4 v[kU];
+    };
+    for (int c0 = 0; c0 < C; c0 += 32 * kU) {
+        int64_t t = w0;
+        uint4 cur[kU];
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const int c = c0 + u * 32 + lane;
-                if (c < C) v[u] = md::ld_stream(x + t * C + c);
+        for (int u = 0; u < kU; ++u) {
+            const int c = c0 + u * 32 + lane;
+            if (c < C) cur[u] = md::ld_stream(x + t * C + c);
+        }
+        int r, e;
+        float ww;
+        slot(t, r, e, ww);
+        for (; t < T; t += nw) {
+            const int64_t tn = t + nw;
+            uint4 nxt[kU];
+            int rn, en;
+            float wn;
+            if (tn < T) {
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    const int c = c0 + u * 32 + lane;
+                    if (c < C) nxt[u] = md::ld_stream(x + tn * C + c);
+                }
             }
+            slot(tn, rn, en, wn);
+            int d = (lane < K && e >= 0 && e < E) ? __ldg(p_g + e) : -1;
+            if (d >= R) d = -1;
+            // slots sharing a row travel in it once; the row's slot mask is the group
+            const unsigned g = __match_any_sync(0xffffffffu, lane < K ? (unsigned)r : (0x80000000u | lane));
+            const bool first = lane < K && (g & md::lanemask_lt()) == 0u;
+            int64_t dst = -1;
+            if (first && d >= 0) {
+                const int lo = __ldg(rank_offsets + d), hi = __ldg(rank_offsets + d + 1);
+                if (r >= lo && r < hi) {
+                    dst = pt.p[d].row_base + (r - lo);
+                    if (dst < 0 || dst >= pt.p[d].rows_cap) dst = -1;
+                }
+            }
+            if (first && dst < 0 && c0 == 0) md::report(status, MD_ERR_DATA);
+            const unsigned rows = __ballot_sync(0xffffffffu, first && dst >= 0);
             unsigned todo = rows;
             while (todo) {
                 const int j = __ffs(todo) - 1;
@@ -107,25 +137,24 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
                 for (int u = 0; u < kU; ++u) {
                     const int c = c0 + u * 32 + lane;
-                    if (c < C) out[c] = v[u];
+                    if (c < C) out[c] = cur[u];
+                }
+                if (c0 == 0) {  // metadata: global token id, expert and gate per slot
+                    const unsigned gm = __shfl_sync(0xffffffffu, g, j);
+                    const md_peer_rows &q = pt.p[dd];
+                    if (lane == 0 && q.token) q.token[drow] = (int32_t)(token_base + t);
+                    if (lane < K) {
+                        const bool mine = (gm >> lane) & 1u;
+                        if (q.slot_idx) q.slot_idx[drow * K + lane] = mine ? e : -1;
+                        if (q.slot_w) q.slot_w[drow * K + lane] = mine ? ww : 0.0f;
+                    }
                 }
             }
-        }
-        // metadata of each row sent: global token id, expert and gate per slot
-        unsigned todo = rows;
-        while (todo) {
-            const int j = __ffs(todo) - 1;
-            todo &= todo - 1;
-            const int dd = __shfl_sync(0xffffffffu, d, j);
-            const int64_t drow = __shfl_sync(0xffffffffu, dst, j);
-            const unsigned gm = __shfl_sync(0xffffffffu, g, j);
-            const md_peer_rows &q = pt.p[dd];
-            if (lane == 0 && q.token) q.token[drow] = (int32_t)(token_base + t);
-            if (lane < K) {
-                const bool mine = (gm >> lane) & 1u;
-                if (q.slot_idx) q.slot_idx[drow * K + lane] = mine ? e : -1;
-                if (q.slot_w) q.slot_w[drow * K + lane] = mine ? ww : 0.0f;
-            }
+#pragma unroll
+            for (int u = 0; u < kU; ++u) cur[u] = nxt[u];
+            r = rn;
+            e = en;
+            ww = wn;
         }
     }
 }
@@ -176,21 +205,27 @@ __device__ __forceinline__ int rank_among(bool live, int key, int n)
 
 // --------------------------------------------------------------- partials
 // z[i] = bf16(sum over slots j carried by received row i, ascending expert,
-// of slot_w[i][j] * y[y_row[i][j]]), fp32 FMA from +0.0f.
+// of slot_w[i][j] * y[y_row[i][j]]), fp32 FMA from +0.0f.  A received dedup
+// row carries few slots (k / rows per token, about 1.2 for top-8 over 16
+// ranks), so the warp takes them one after another, 4 16-byte chunks per
+// lane of each at a time (8 measured slower: twice the registers, half the
+// resident warps; so did a compile-time k, 930 against 780 us).
 __global__ void __launch_bounds__(kThreads)
     k_combine_partials(const uint4 *__restrict__ y, int64_t y_rows, const int32_t *__restrict__ y_row,
                        const int32_t *__restrict__ slot_idx, const float *__restrict__ slot_w,
                        int64_t n, int k, int C, uint4 *__restrict__ z, int32_t *status)
 {
+    constexpr int U = 4;
+    const int K = k;
     const int lane = threadIdx.x & 31;
     const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
     for (int64_t i = ((int64_t)blockIdx.x * kThreads + threadIdx.x) >> 5; i < n; i += nw) {
         int yr = -1, e = INT_MAX;
         float ww = 0.0f;
-        if (lane < k) {
-            yr = __ldg(y_row + i * k + lane);
-            e = __ldg(slot_idx + i * k + lane);
-            ww = __ldg(slot_w + i * k + lane);
+        if (lane < K) {
+            yr = __ldg(y_row + i * K + lane);
+            e = __ldg(slot_idx + i * K + lane);
+            ww = __ldg(slot_w + i * K + lane);
             if (yr >= y_rows) {
                 md::report(status, MD_ERR_DATA);
                 yr = -1;
@@ -198,28 +233,28 @@ __global__ void __launch_bounds__(kThreads)
         }
         const bool live = yr >= 0;
         const int nv = __popc(__ballot_sync(0xffffffffu, live));
-        const int rank = rank_among(live, e, k);
-        for (int c0 = 0; c0 < C; c0 += 32 * 4) {
-            float acc[4][8];
+        const int rank = rank_among(live, e, K);
+        for (int c0 = 0; c0 < C; c0 += 32 * U) {
+            float acc[U][8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
             for (int q = 0; q < nv; ++q) {
                 const int j = __ffs(__ballot_sync(0xffffffffu, live && rank == q)) - 1;
                 const int64_t r = __shfl_sync(0xffffffffu, yr, j);
                 const float wt = __shfl_sync(0xffffffffu, ww, j);
-                uint4 v[4];
+                uint4 v[U];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < U; ++u) {
                     const int c = c0 + u * 32 + lane;
                     v[u] = c < C ? md::ld_stream(y + r * C + c) : make_uint4(0, 0, 0, 0);
                 }
 #pragma unroll
-                for (int u = 0; u < 4; ++u) fma_row8(acc[u], wt, v[u]);
+                for (int u = 0; u < U; ++u) fma_row8(acc[u], wt, v[u]);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int c = c0 + u * 32 + lane;
                 if (c < C) md::st_stream(z + i * C + c, pack8(acc[u]));
             }
@@ -229,7 +264,8 @@ __global__ void __launch_bounds__(kThreads)
 
 // ---------------------------------------------------------------- combine
 // out[t] = bf16(fp32 sum over t's distinct rows, in ascending destination
-// rank, of the bf16 return row held by that rank).
+// rank, of the bf16 return row held by that rank).  With a compile-time k the
+// warp issues the loads of all the token's return rows before the adds.
 template <int KC>
 __global__ void __launch_bounds__(kThreads)
     k_combine_exchange(int64_t T, int C, int k, const int32_t *__restrict__ idx,
@@ -238,6 +274,8 @@ __global__ void __launch_bounds__(kThreads)
                        const int32_t *__restrict__ rank_offsets, PeerTable pt,
                        uint4 *__restrict__ out, int32_t *status)
 {
+    constexpr int KB = KC ? KC : 1;
+    constexpr int U = KC ? (KC >= 8 ? 1 : 8 / KC) : 4;
     const int K = KC ? KC : k;
     const int lane = threadIdx.x & 31;
     const int64_t nw = ((int64_t)gridDim.x * kThreads) >> 5;
@@ -263,28 +301,55 @@ __global__ void __launch_bounds__(kThreads)
         const bool live = first && src >= 0;
         const int nv = __popc(__ballot_sync(0xffffffffu, live));
         const int rank = rank_among(live, d, K);
-        for (int c0 = 0; c0 < C; c0 += 32 * 4) {
-            float acc[4][8];
+        // the token's return rows in ascending rank
+        const uint4 *zr[KB];
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+        for (int q = 0; q < KB; ++q) {
+            const unsigned bal = KC ? __ballot_sync(0xffffffffu, live && rank == q) : 0u;
+            const int j = bal ? __ffs(bal) - 1 : 0;
+            const int dd = __shfl_sync(0xffffffffu, d, j);
+            const int64_t sr = __shfl_sync(0xffffffffu, src, j);
+            zr[q] = bal ? static_cast<const uint4 *>(pt.p[dd].rows) + sr * C : nullptr;
+        }
+        for (int c0 = 0; c0 < C; c0 += 32 * U) {
+            float acc[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[u][q] = 0.0f;
-            for (int q = 0; q < nv; ++q) {
-                const int j = __ffs(__ballot_sync(0xffffffffu, live && rank == q)) - 1;
-                const int dd = __shfl_sync(0xffffffffu, d, j);
-                const int64_t sr = __shfl_sync(0xffffffffu, src, j);
-                const uint4 *zr = static_cast<const uint4 *>(pt.p[dd].rows) + sr * C;
-                uint4 v[4];
+            if (KC) {
+                uint4 v[KB][U];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + u * 32 + lane;
-                    v[u] = c < C ? __ldcg(zr + c) : make_uint4(0, 0, 0, 0);
+                for (int q = 0; q < KB; ++q)
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + u * 32 + lane;
+                        v[q][u] = (zr[q] && c < C) ? __ldcg(zr[q] + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                for (int q = 0; q < KB; ++q)
+                    if (zr[q]) {
+#pragma unroll
+                        for (int u = 0; u < U; ++u) add_row8(acc[u], v[q][u]);
+                    }
+            } else {
+                for (int q = 0; q < nv; ++q) {
+                    const int j = __ffs(__ballot_sync(0xffffffffu, live && rank == q)) - 1;
+                    const int dd = __shfl_sync(0xffffffffu, d, j);
+                    const int64_t sr = __shfl_sync(0xffffffffu, src, j);
+                    const uint4 *row = static_cast<const uint4 *>(pt.p[dd].rows) + sr * C;
+                    uint4 v[U];
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int c = c0 + u * 32 + lane;
+                        v[u] = c < C ? __ldcg(row + c) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int u = 0; u < U; ++u) add_row8(acc[u], v[u]);
                 }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) add_row8(acc[u], v[u]);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int c = c0 + u * 32 + lane;
                 if (c < C) md::st_stream(out + t * C + c, pack8(acc[u]));
             }
@@ -371,6 +436,8 @@ extern "C" int md_dispatch_exchange(const void *x, int64_t T, int H, int k, cons
                                                       dev_status)
     switch (k) {
     case 2: MD_DX(2); break;
+    case 4: MD_DX(4); break;
+    case 6: MD_DX(6); break;
     case 8: MD_DX(8); break;
     default: MD_DX(0); break;
     }
@@ -418,6 +485,8 @@ extern "C" int md_combine_exchange(const md_peer_rows *peers, int64_t T, int H, 
                                                      static_cast<uint4 *>(out), dev_status)
     switch (k) {
     case 2: MD_CX(2); break;
+    case 4: MD_CX(4); break;
+    case 6: MD_CX(6); break;
     case 8: MD_CX(8); break;
     default: MD_CX(0); break;
     }

@@ -33,7 +33,8 @@
 
 namespace {
 
-constexpr int kRankThreads = 512;  // one token per thread
+// one token per thread; 256-thread CTAs, two per SM, measured no faster
+constexpr int kRankThreads = 512;
 constexpr int kRankWarps = kRankThreads / 32;
 constexpr int kStageRows = 4096;   // output rows a tile can stage
 constexpr int kMaxCtas = 256;      // CTAs of one launch; the workspace is sized for it
@@ -571,28 +572,31 @@ int check_layout_args(int64_t T, int E, int k, int R, int mode)
 constexpr size_t kLayoutSmemMax = (size_t)(2 * 1024 + (2 * kRankWarps + 4) * (1024 + 64) +
                                            3 * kStageRows + 32 * 64) * sizeof(int);
 
-// CTAs of k_layout<KC> resident per SM with the largest shared-memory size
-// (set once per device)
+// CTAs of k_layout<KC> resident per SM with `smem` bytes of dynamic shared
+// memory (the limit is raised to the largest size once per device; the
+// occupancy query is host arithmetic, so it runs per call)
 template <int KC>
-int layout_per_sm()
+int layout_per_sm(size_t smem)
 {
     static std::atomic<uint64_t> done{0};
-    static int per_sm[64];
+    static std::atomic<int> attr_ok[64];
     md::once_per_device(done, [] {
-        int dev = 0, nb = 0;
+        int dev = 0;
         cudaGetDevice(&dev);
-        if (cudaFuncSetAttribute(k_layout<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kLayoutSmemMax) != cudaSuccess ||
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_layout<KC>, kRankThreads,
-                                                          kLayoutSmemMax) != cudaSuccess) {
-            cudaGetLastError();
-            nb = 0;
-        }
-        per_sm[dev & 63] = nb;
+        const bool ok = cudaFuncSetAttribute(k_layout<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)kLayoutSmemMax) == cudaSuccess;
+        if (!ok) cudaGetLastError();
+        attr_ok[dev & 63].store(ok ? 1 : 0);
     });
     int dev = 0;
     cudaGetDevice(&dev);
-    return per_sm[dev & 63];
+    if (!attr_ok[dev & 63].load()) return 0;
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_layout<KC>, kRankThreads, smem) != cudaSuccess) {
+        cudaGetLastError();
+        nb = 0;
+    }
+    return nb;
 }
 
 template <int KC>
@@ -604,7 +608,7 @@ int launch_layout(const int32_t *topk_idx, int64_t T, int E, int k, int R,
                   int32_t *dev_status, cudaStream_t s)
 {
     const size_t smem = layout_smem(E, R, mode);
-    const int per_sm = layout_per_sm<KC>();
+    const int per_sm = layout_per_sm<KC>(smem);
     if (per_sm < 1 || smem > kLayoutSmemMax) return MD_ERR_UNSUPPORTED;
     // every CTA waits for all the others: the grid must be resident at once
     int resident = md::sm_count() * per_sm;

@@ -28,8 +28,19 @@ pytestmark = pytest.mark.gpu
 POISON = 0x7FA1
 
 
-def _run(name, T, R, H, placement, seed=0):
-    w = synth.make_workload(name, seed=seed, T=T, R=R, H=H)
+class _Generic:
+    """A small workload with a k that has no specialised kernel."""
+
+    def __init__(self, T, E, k, R, H, seed):
+        self.T, self.E, self.k, self.R, self.H = T, E, k, R, H
+        self.logits = synth.normal_f32(T, E, seed, 1)
+        self.x = synth.normal_bf16(T, H, seed, 3)
+        self.y = synth.normal_bf16(T * k, H, seed, 4)
+        self.expert_to_rank = synth.contiguous_placement(E, R)
+
+
+def _run(name, T, R, H, placement, seed=0, w=None):
+    w = w or synth.make_workload(name, seed=seed, T=T, R=R, H=H)
     E, k = w.E, w.k
     oi, ow = oracle.route_topk(w.logits.numpy(), k)
     p = w.expert_to_rank.numpy() if placement == "contiguous" else shuffled_placement(E, R, 4)
@@ -120,6 +131,14 @@ def _run(name, T, R, H, placement, seed=0):
 ])
 def test_exchange_matches_single_gpu_oracle(name, T, R, H, placement):
     _run(name, T, R, H, placement)
+
+
+@pytest.mark.parametrize("k,E,R", [(3, 32, 4), (12, 64, 8)])
+def test_exchange_generic_k(k, E, R):
+    # k without a specialised kernel: the reading kernels take a token's rows
+    # one after another
+    T, H = 64 * R, 40
+    _run(None, T, R, H, "shuffled", w=_Generic(T, E, k, R, H, seed=k))
 
 
 def test_exchange_reports_rows_outside_the_buffers():
