@@ -42,14 +42,19 @@ inline int clear_status(int32_t *dev_status, cudaStream_t s)
     return cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) == cudaSuccess ? MD_OK : MD_ERR_CUDA;
 }
 
+// SMs of the current device (cached per device)
 inline int sm_count()
 {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    int n = cache[dev & 63].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+            cudaGetLastError();
+            n = 148;
+        }
+        cache[dev & 63].store(n, std::memory_order_relaxed);
     }
     return n;
 }

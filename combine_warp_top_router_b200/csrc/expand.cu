@@ -183,7 +183,12 @@ extern "C" int md_dedup_expand(const void *wire, int64_t n_wire, int H, const in
     if (rowbytes >= kMinRowBytes) {
         const int pieces = (rowbytes + kPiece - 1) / kPiece;
         const size_t smem = (size_t)kWarps * kStages * kPiece;
-        cudaFuncSetAttribute(k_expand_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        static std::atomic<uint64_t> attr_done{0};
+        md::once_per_device(attr_done, [smem] {
+            if (cudaFuncSetAttribute(k_expand_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                cudaSuccess)
+                cudaGetLastError();  // the launch then fails and reports MD_ERR_CUDA
+        });
         int64_t blocks = (n_slots * pieces + kWarps - 1) / kWarps;
         if (blocks > md::sm_count()) blocks = md::sm_count();
         k_expand_tma<<<(unsigned)(blocks < 1 ? 1 : blocks), kWarps * 32, smem, s>>>(

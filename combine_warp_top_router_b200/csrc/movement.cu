@@ -446,10 +446,24 @@ void launch_permute(const void *x, int64_t T, int C, int k, const int32_t *rs, i
     bool bulk = rowbytes >= kTmaMinRowBytes && path != MD_PERMUTE_VECTOR;
     if (bulk && path == MD_PERMUTE_AUTO)
         bulk = k > 4 && units >= (int64_t)8 * md::sm_count() * kTmaWarps;
+    // once per device: the ring's shared-memory limit and the vector
+    // kernel's resident CTAs per SM
+    static std::atomic<uint64_t> setup{0};
+    static std::atomic<int> vec_per_sm[64];
+    const size_t smem = (size_t)kTmaWarps * kTmaStages * kTmaPiece;
+    md::once_per_device(setup, [smem] {
+        int dev = 0, nb = 0;
+        cudaGetDevice(&dev);
+        if (cudaFuncSetAttribute(k_permute_tma<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            cudaGetLastError();  // the launch then fails and reports MD_ERR_CUDA
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_permute<KC>, kThreads, 0) != cudaSuccess) {
+            cudaGetLastError();
+            nb = 1;
+        }
+        vec_per_sm[dev & 63].store(nb < 1 ? 1 : nb);
+    });
     if (bulk) {
-        const size_t smem = (size_t)kTmaWarps * kTmaStages * kTmaPiece;
-        cudaFuncSetAttribute(k_permute_tma<KC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
         int64_t blocks = (units + kTmaWarps - 1) / kTmaWarps;
         const int64_t cap = md::sm_count();
         if (blocks > cap) blocks = cap;
@@ -458,11 +472,9 @@ void launch_permute(const void *x, int64_t T, int C, int k, const int32_t *rs, i
             st);
         return;
     }
-    static int per_sm = 0;
-    if (per_sm == 0) {
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_permute<KC>, kThreads, 0);
-        if (per_sm < 1) per_sm = 1;
-    }
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int per_sm = vec_per_sm[dev & 63].load();
     int64_t blocks = (T + kThreads / 32 - 1) / (kThreads / 32);
     const int64_t cap = (int64_t)md::sm_count() * per_sm;
     if (blocks > cap) blocks = cap;

@@ -2,7 +2,8 @@
 device memory (for example a plug-in whose host framework owns all GPU memory
 through its own pool).  It must give exactly what md_dispatch_layout gives with
 a caller-allocated workspace, call after call, although every call reuses the
-same fixed scratch array inside the library.
+same fixed scratch array inside the library (and, for the smaller shapes,
+exactly the oracle's layout).
 
 Called through the C ABI with ctypes.  This file is collected last on purpose;
 it also passes when run alone in a fresh process."""
@@ -88,6 +89,14 @@ def test_noalloc_matches_workspace_entry_point_twice(name, T, mode):
         torch.cuda.synchronize()
         assert int(status.item()) == md.MD_OK
         _same(got, want)
+        if T <= 65536:  # and the oracle's layout of the same top-k lists
+            import oracle
+            O = oracle.dispatch_layout(idx.cpu().numpy(), E, R, p.cpu().numpy(), mode)
+            n = O["n_rows"]
+            assert int(got.n_rows.item()) == n
+            for name_ in ("row_of_slot", "assign_row", "send_counts", "rank_offsets"):
+                assert np.array_equal(getattr(got, name_).cpu().numpy(), O[name_]), name_
+            assert np.array_equal(got.row_token[:n].cpu().numpy(), O["row_token"])
 
 
 def test_noalloc_takes_sizes_whose_old_scratch_need_was_larger():
