@@ -21,7 +21,7 @@
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kGroup = 8;  // tokens per CTA iteration (one warp per token when sorting)
+constexpr int kGroup = 8;  // tokens per CTA iteration: one of the 8 warps sorts each token's slots
 
 int grid_for(int64_t units, int per_block)
 {
@@ -487,7 +487,7 @@ void launch_combine(const void *y, int64_t y_rows, const int32_t *ar, const int3
                     const float *w, int64_t T, int k, int C, const int32_t *rs, int64_t z_rows,
                     void *z, void *out, int32_t *st, cudaStream_t s)
 {
-    if (KC > 0 && !WIRE) {
+    if (KC > 0 && !WIRE) {  // 4, 6 or 16 CTAs per SM measured no better than 8
         k_combine_fused<KC ? KC : 1><<<grid_for(T, kGroup), kThreads, 0, s>>>(
             static_cast<const uint4 *>(y), y_rows, ar, idx, w, T, C, static_cast<uint4 *>(out), st);
         return;
