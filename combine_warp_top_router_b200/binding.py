@@ -26,6 +26,7 @@ MD_COMBINE_FUSED, MD_COMBINE_WIRE = 0, 1
 MD_SEED_CONTIGUOUS, MD_SEED_GREEDY_PAIRS = 0, 1
 MD_REFINE_NONE, MD_REFINE_SWAPS, MD_REFINE_KL = 0, 1, 2
 MD_PERMUTE_AUTO, MD_PERMUTE_BULK, MD_PERMUTE_VECTOR = 0, 1, 2
+MD_LAYOUT_AUTO, MD_LAYOUT_COOPERATIVE, MD_LAYOUT_SPLIT = 0, 1, 2
 
 _lock = threading.Lock()
 _lib = None
@@ -44,6 +45,7 @@ _SIGNATURES = {
                                     _P, _P, _P], _I),
     "md_dispatch_permute": ([_P, _L, _I, _I, _P, _L, _P, _P, _P], _I),
     "md_set_permute_path": ([_I], _I),
+    "md_set_layout_path": ([_I], _I),
     "md_exchange_plan": ([_P, _I, _I, _P, _P], _I),
     "md_dispatch_exchange": ([_P, _L, _I, _I, _P, _P, _P, _I, _I, _P, _P, _L, _P, _P, _P], _I),
     "md_combine_partials": ([_P, _L, _P, _P, _P, _L, _I, _I, _P, _P, _P], _I),
@@ -304,6 +306,11 @@ def md_dispatch_permute(x, row_of_slot, out_rows=None, out=None, dev_status=None
 def md_set_permute_path(path=MD_PERMUTE_AUTO):
     """Choose md_dispatch_permute's kernel (tests and tuning; same bits either way)."""
     _check(lib().md_set_permute_path(int(path)), "md_set_permute_path")
+
+
+def md_set_layout_path(path=MD_LAYOUT_AUTO):
+    """Choose md_dispatch_layout's launch form (tests; same results either way)."""
+    _check(lib().md_set_layout_path(int(path)), "md_set_layout_path")
 
 
 def md_dedup_expand(wire, row_of_slot, assign_row, out_rows=None, out=None, dev_status=None,

@@ -22,7 +22,17 @@ long long hook_expand_skip_unit() { return g_expand_skip_unit.load(std::memory_o
 
 static std::atomic<int> g_permute_path{MD_PERMUTE_AUTO};
 int permute_path() { return g_permute_path.load(std::memory_order_relaxed); }
+static std::atomic<int> g_layout_path{MD_LAYOUT_AUTO};
+int layout_path() { return g_layout_path.load(std::memory_order_relaxed); }
 }  // namespace md
+
+extern "C" int md_set_layout_path(int path)
+{
+    if (path != MD_LAYOUT_AUTO && path != MD_LAYOUT_COOPERATIVE && path != MD_LAYOUT_SPLIT)
+        return MD_ERR_ARG;
+    md::g_layout_path.store(path, std::memory_order_relaxed);
+    return MD_OK;
+}
 
 extern "C" int md_set_permute_path(int path)
 {

@@ -21,8 +21,10 @@ long long hook_poll_limit(long long dflt);
 int hook_layout_skip_tile();        // -1: none
 long long hook_expand_skip_unit();  // -1: none
 
-// Kernel choice of md_dispatch_permute (md_set_permute_path).
+// Kernel choice of md_dispatch_permute (md_set_permute_path) and launch form
+// of md_dispatch_layout (md_set_layout_path).
 int permute_path();
+int layout_path();
 
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 

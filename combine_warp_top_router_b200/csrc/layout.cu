@@ -24,6 +24,10 @@
 //      32-bit set per bucket, built with shared atomicOr), so a pair's rank
 //      among the warp's earlier tokens is a popcount; rows are staged in
 //      shared memory in bucket order and written out in runs.
+// When a cooperative launch is refused (its CTAs cannot all be resident, e.g.
+// while other work holds SMs), the same kernel runs split in two launches:
+// A, then B and C; the second launch starts after every CTA's counts, so no
+// arrival wait is needed.
 // Nothing in the workspace has to start at zero: every call first clears the
 // arrival words on its stream (a 1 KiB memset, recorded too when the stream is
 // capturing), so a word left over from an earlier call, or from whatever the
@@ -39,6 +43,7 @@ constexpr int kRankWarps = kRankThreads / 32;
 constexpr int kStageRows = 4096;   // output rows a tile can stage
 constexpr int kMaxCtas = 256;      // CTAs of one launch; the workspace is sized for it
 constexpr long long kPollLimit = 1ll << 22;
+constexpr int kPhaseCounts = 1, kPhaseWait = 2, kPhaseRanks = 4;
 
 struct Ws {
     long long poll_limit;         // bound of the arrival wait
@@ -149,8 +154,14 @@ __global__ void __launch_bounds__(kRankThreads, 1)
              int32_t *__restrict__ row_token, uint32_t *__restrict__ row_mask, int64_t row_cap,
              int32_t *__restrict__ expert_counts, int32_t *__restrict__ send_counts,
              int32_t *__restrict__ expert_offsets, int32_t *__restrict__ rank_offsets,
-             int32_t *__restrict__ n_rows, int32_t *status)
+             int32_t *__restrict__ n_rows, int32_t *status, int phases)
 {
+    // phases: kPhaseCounts (A, publish the counts), kPhaseWait (the arrival
+    // wait: all CTAs resident), kPhaseRanks (B, bases, C).  One cooperative
+    // launch runs all three; the split form runs counts, then ranks in a
+    // second launch whose start orders it after every CTA's counts.
+    const bool do_counts = phases & kPhaseCounts, do_wait = phases & kPhaseWait;
+    const bool do_ranks = phases & kPhaseRanks;
     constexpr int KM = KC ? KC : MD_MAX_TOPK;
     const int K = KC ? KC : k;
     extern __shared__ int smem[];
@@ -206,7 +217,7 @@ __global__ void __launch_bounds__(kRankThreads, 1)
 
     // ---- A. bucket counts and send rows of this CTA's tokens
     bool bad = false;
-    for (int tile = tile_lo; tile < tile_hi; ++tile) {
+    for (int tile = tile_lo; do_counts && tile < tile_hi; ++tile) {
         const int64_t t = (int64_t)tile * tile_tok + tid;
         if (tid >= tile_tok || t >= T) continue;
         int e[KM], d[KM];
@@ -238,7 +249,7 @@ __global__ void __launch_bounds__(kRankThreads, 1)
         }
     }
     __syncthreads();
-    if (one_src) {
+    if (do_counts && one_src) {
         if (dedup) {
             for (int dd = tid; dd < R; dd += kRankThreads) s_send[s_lo * R + dd] = s_acnt[E + dd];
         } else {
@@ -249,19 +260,25 @@ __global__ void __launch_bounds__(kRankThreads, 1)
         }
         __syncthreads();
     }
-    for (int b = tid; b < NB; b += kRankThreads) ws.cnt[(size_t)b * kMaxCtas + cta] = s_acnt[b];
-    for (int i = tid; i < (s_hi - s_lo + 1) * R; i += kRankThreads) {
-        const int s = s_lo + i / R, dd = i % R;
-        ws.part[(size_t)(cta + s) * R + dd] = s_send[s * R + dd];
+    if (do_counts) {
+        for (int b = tid; b < NB; b += kRankThreads) ws.cnt[(size_t)b * kMaxCtas + cta] = s_acnt[b];
+        for (int i = tid; i < (s_hi - s_lo + 1) * R; i += kRankThreads) {
+            const int s = s_lo + i / R, dd = i % R;
+            ws.part[(size_t)(cta + s) * R + dd] = s_send[s * R + dd];
+        }
+        __syncthreads();
+        if (do_wait && tid == 0 && cta != ws.skip_cta) {
+            __threadfence();
+            st_relaxed_u32(ws.flags + cta, ws.epoch);
+        }
     }
-    __syncthreads();
-    if (tid == 0 && cta != ws.skip_cta) {
-        __threadfence();
-        st_relaxed_u32(ws.flags + cta, ws.epoch);
+    if (!do_ranks) {  // the split form's first launch ends here
+        if (bad) md::report(status, MD_ERR_DATA);
+        return;
     }
     // every CTA's counts are in once its arrival word is stamped; one
     // warp reads all stamps, four per 16-byte load
-    if (w == 0) {
+    if (do_wait && w == 0) {
         long long polls = 0;
         for (;;) {
             bool ok = true;
@@ -618,19 +635,34 @@ int launch_layout(const int32_t *topk_idx, int64_t T, int E, int k, int R,
     int tile_tok = pl.tile_tok, n_tiles = pl.n_tiles, mode_ = mode, k_ = k, E_ = E, R_ = R;
     int64_t T_ = T, cap_ = cap;
     Ws ws_ = ws;
-    void *args[] = {(void *)&topk_idx, &T_,          &E_,         &k_,          &R_,
-                    (void *)&expert_to_rank, &mode_, &tile_tok,  &n_tiles,     (void *)&tpc,
-                    &ws_,        (void *)&row_of_slot, (void *)&assign_row, (void *)&row_token,
-                    (void *)&row_mask, &cap_, (void *)&expert_counts, (void *)&send_counts,
-                    (void *)&expert_offsets, (void *)&rank_offsets, (void *)&n_rows,
-                    (void *)&dev_status};
-    md::count_launches(1);
-    if (cudaLaunchCooperativeKernel((const void *)k_layout<KC>, dim3((unsigned)G), dim3(kRankThreads),
-                                    args, smem, s) != cudaSuccess) {
-        cudaGetLastError();
-        return MD_ERR_CUDA;
+    const int path = md::layout_path();
+    if (path != MD_LAYOUT_SPLIT) {
+        int phases = kPhaseCounts | kPhaseWait | kPhaseRanks;
+        void *args[] = {(void *)&topk_idx, &T_,          &E_,         &k_,          &R_,
+                        (void *)&expert_to_rank, &mode_, &tile_tok,  &n_tiles,     (void *)&tpc,
+                        &ws_,        (void *)&row_of_slot, (void *)&assign_row, (void *)&row_token,
+                        (void *)&row_mask, &cap_, (void *)&expert_counts, (void *)&send_counts,
+                        (void *)&expert_offsets, (void *)&rank_offsets, (void *)&n_rows,
+                        (void *)&dev_status, &phases};
+        md::count_launches(1);
+        if (cudaLaunchCooperativeKernel((const void *)k_layout<KC>, dim3((unsigned)G), dim3(kRankThreads),
+                                        args, smem, s) == cudaSuccess)
+            return MD_OK;
+        cudaGetLastError();  // refused (e.g. SMs held by other work): split, unless forbidden
+        if (path == MD_LAYOUT_COOPERATIVE) return MD_ERR_CUDA;
     }
-    return MD_OK;
+    // split form: the counts of every CTA, then the ranks in a second launch;
+    // no CTA waits on another, so the grid need not be resident at once
+    md::count_launches(2);
+    k_layout<KC><<<(unsigned)G, kRankThreads, smem, s>>>(
+        topk_idx, T, E, k, R, expert_to_rank, mode, tile_tok, n_tiles, tpc, ws, row_of_slot,
+        assign_row, row_token, row_mask, cap, expert_counts, send_counts, expert_offsets, rank_offsets,
+        n_rows, dev_status, kPhaseCounts);
+    k_layout<KC><<<(unsigned)G, kRankThreads, smem, s>>>(
+        topk_idx, T, E, k, R, expert_to_rank, mode, tile_tok, n_tiles, tpc, ws, row_of_slot,
+        assign_row, row_token, row_mask, cap, expert_counts, send_counts, expert_offsets, rank_offsets,
+        n_rows, dev_status, kPhaseRanks);
+    return md::launch_status();
 }
 
 }  // namespace
@@ -666,10 +698,12 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
     // memsets, so every replay waits for its own counts).  Stale arrival words
     // can therefore never let a CTA pass the wait early.
     if ((rc = md::clear_status(dev_status, s)) != MD_OK) return rc;
-    md::count_launches(1);
-    if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 4, s) != cudaSuccess) {
-        cudaGetLastError();
-        return MD_ERR_CUDA;
+    if (md::layout_path() != MD_LAYOUT_SPLIT) {  // the split form has no arrival wait
+        md::count_launches(1);
+        if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 4, s) != cudaSuccess) {
+            cudaGetLastError();
+            return MD_ERR_CUDA;
+        }
     }
 
     const int64_t cap = mode == MD_CONV ? T * k : T * (int64_t)(k < R ? k : R);

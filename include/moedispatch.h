@@ -140,11 +140,13 @@ int md_route_topk(const float *logits, int64_t T, int E, int k, int gate_mode,
  *                   size does not grow with T (at most about 1.2 MiB, at
  *                   E=1024, R=64).
  *   One cooperative launch: all its CTAs (at most one per SM) must be
- *   resident at once, so a GPU shared with a running kernel that holds SMs
- *   may delay it; MD_ERR_CUDA if the launch is refused.  Every CTA waits for
- *   the others' counts with a bounded wait (MD_ERR_TIMEOUT in dev_status if
- *   it runs out; the outputs are then not written).  Safe in CUDA graph
- *   capture: the graph records the clear of the arrival words with the kernel.
+ *   resident at once, and every CTA waits for the others' counts with a
+ *   bounded wait (MD_ERR_TIMEOUT in dev_status if it runs out; the outputs
+ *   are then not written).  If the cooperative launch is refused (other work
+ *   holds SMs), the call runs the same kernel split in two ordinary launches,
+ *   counts then ranks, with identical results (md_set_layout_path).  Safe in
+ *   CUDA graph capture: the graph records the clear of the arrival words
+ *   with the kernel (a launch refused during capture ends the capture).
  *   Limits: T % R == 0, E % R == 0, 1 <= k <= min(E, 32), E <= 1024,
  *   R <= 64, T*k < 2^31.
  */
@@ -227,6 +229,23 @@ int md_dispatch_permute(const void *x, int64_t T, int H, int k,
 #define MD_PERMUTE_VECTOR 2
 
 int md_set_permute_path(int path);
+
+/*
+ * md_set_layout_path -- the launch form of md_dispatch_layout (for tests and
+ * for GPUs shared with other work; the results are the same either way).
+ *   MD_LAYOUT_AUTO         one cooperative launch; if it is refused, the
+ *                          split form (default)
+ *   MD_LAYOUT_COOPERATIVE  one cooperative launch; MD_ERR_CUDA if refused
+ *   MD_LAYOUT_SPLIT        always two launches: every CTA's counts, then the
+ *                          ranks; no CTA waits on another
+ * Process-wide; MD_ERR_ARG for another value.  Set it only while no
+ * md_dispatch_layout call is being enqueued.
+ */
+#define MD_LAYOUT_AUTO 0
+#define MD_LAYOUT_COOPERATIVE 1
+#define MD_LAYOUT_SPLIT 2
+
+int md_set_layout_path(int path);
 
 /*
  * md_dedup_expand -- receiver-side expand of deduplicated rows.

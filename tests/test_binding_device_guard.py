@@ -63,5 +63,5 @@ def test_every_compute_entry_point_goes_through_the_guard():
               if "lib().md_" in ln and "workspace_size" not in ln and "status_string" not in ln
               and "launch_count" not in ln and "set_test_hooks" not in ln
               and "md_table1_row" not in ln and "md_pearson_from_sums" not in ln
-              and "set_permute_path" not in ln and "md_exchange_plan" not in ln]
+              and "set_permute_path" not in ln and "set_layout_path" not in ln and "md_exchange_plan" not in ln]
     assert direct == []

@@ -17,6 +17,15 @@ pytestmark = pytest.mark.gpu
 POISON = -7
 
 
+@pytest.fixture(params=[md.MD_LAYOUT_COOPERATIVE, md.MD_LAYOUT_SPLIT], ids=["coop", "split"])
+def layout_path(request):
+    """Run a layout test with each launch form: one cooperative launch with
+    the arrival wait, and the split form (counts, then ranks)."""
+    md.md_set_layout_path(request.param)
+    yield request.param
+    md.md_set_layout_path(md.MD_LAYOUT_AUTO)
+
+
 def gpu_layout(idx_np, E, R, p_np, mode):
     idx = i32(idx_np)
     T, k = idx_np.shape
@@ -65,7 +74,7 @@ CASES = [
 
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("name,T,R,pl", CASES)
-def test_layout_matches_oracle(name, T, R, pl, mode):
+def test_layout_matches_oracle(name, T, R, pl, mode, layout_path):
     idx = _routes(name, T)
     E = synth.SPECS[name]["E"]
     p = synth.contiguous_placement(E, R).numpy() if pl == "contiguous" else shuffled_placement(E, R, 3)
@@ -77,7 +86,7 @@ def test_layout_matches_oracle(name, T, R, pl, mode):
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("E,k,R,T", [(8, 1, 2, 100), (8, 8, 8, 64), (16, 3, 1, 48), (12, 5, 3, 99),
                                      (1024, 32, 64, 128), (256, 16, 4, 256), (64, 6, 64, 4096)])
-def test_layout_edge_shapes(E, k, R, T, mode):
+def test_layout_edge_shapes(E, k, R, T, mode, layout_path):
     lg = synth.normal_f32(T, E, 11, 1).numpy()
     idx = oracle.route_topk(lg, k)[0]
     p = shuffled_placement(E, R, 5)
@@ -86,7 +95,7 @@ def test_layout_edge_shapes(E, k, R, T, mode):
     assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), T, k)
 
 
-def test_layout_empty():
+def test_layout_empty(layout_path):
     E, k, R = 16, 2, 4
     L, st = gpu_layout(np.zeros((0, k), np.int32), E, R, synth.contiguous_placement(E, R).numpy(), 1)
     assert st == md.MD_OK and int(L.n_rows.item()) == 0
@@ -94,7 +103,7 @@ def test_layout_empty():
     assert L.rank_offsets.cpu().tolist() == [0] * (R + 1)
 
 
-def test_layout_reports_bad_data():
+def test_layout_reports_bad_data(layout_path):
     E, k, R, T = 16, 3, 4, 64
     idx = oracle.route_topk(synth.normal_f32(T, E, 1, 1).numpy(), k)[0]
     p = synth.contiguous_placement(E, R).numpy()
@@ -125,7 +134,7 @@ def test_layout_rejects_bad_arguments():
 
 
 @pytest.mark.parametrize("mode", [0, 1])
-def test_layout_full_size(mode):
+def test_layout_full_size(mode, layout_path):
     # the full-pipeline workload at full size: T=262144, E=256, k=8, R=64
     w = synth.make_workload("full_e256_k8", device=DEV, with_rows=False)
     idx_g, _ = md.md_route_topk(w.logits, 8)
@@ -157,7 +166,7 @@ def test_layout_unaligned_outputs(mode):
     assert_layout_equal(L, oracle.dispatch_layout(idx, E, R, p, mode), T, k)
 
 
-def test_layout_replays_in_cuda_graph():
+def test_layout_replays_in_cuda_graph(layout_path):
     # A captured layout replays with new inputs: the capture also records the
     # clear of the arrival words, so every replay waits for its own counts.
     from combine_warp_top_router_b200 import binding
@@ -186,7 +195,7 @@ def test_layout_replays_in_cuda_graph():
 
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("T", [512 * 148 * 3 + 64, 512 * 300, 512 * 148, 512 * 149])
-def test_layout_several_tiles_per_cta(T, mode):
+def test_layout_several_tiles_per_cta(T, mode, layout_path):
     # more tiles than resident CTAs: each CTA walks a run of tiles and carries
     # its bucket starts from one tile to the next (T = 512*148*3 + 64 leaves a
     # short last tile).  512*148 tiles launch one CTA per SM, so the arrival
@@ -203,7 +212,7 @@ def test_layout_several_tiles_per_cta(T, mode):
 
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("fill", ["stamp", "ones_bits", "random"])
-def test_layout_ignores_stale_workspace(fill, mode):
+def test_layout_ignores_stale_workspace(fill, mode, layout_path):
     # Whatever the workspace holds on entry -- every 32-bit word equal to the
     # value a CTA stamps on arrival (1), all bits set, or random words such as
     # a recycled allocation holds -- the layout is the oracle's: the call
@@ -235,3 +244,9 @@ def test_layout_ignores_stale_workspace(fill, mode):
         torch.cuda.synchronize()
         assert int(st.item()) == md.MD_OK
         assert_layout_equal(L, O, T, k)
+
+
+def test_layout_path_selector_rejects_unknown_values():
+    with pytest.raises(md.MoeDispatchError):
+        md.md_set_layout_path(5)
+    md.md_set_layout_path(md.MD_LAYOUT_AUTO)
