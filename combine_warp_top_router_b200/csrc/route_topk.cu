@@ -255,7 +255,9 @@ void launch_k(const float *logits, int64_t T, int E, int k, int gate_mode, int32
 //   2. Candidates.  Only groups whose maximum reaches the threshold (k or a
 //      few more of the 16) are read again; their elements at or above it
 //      (about 10 for k = 8) are compacted into a per-lane list of expert
-//      indices.
+//      indices (64 entries, so a sixth warp fits an SM at E = 256; appends
+//      past the end land on the last entry without a branch, and a lane
+//      with more candidates ranks them by insertion over its row instead).
 //   3. Selection.  Candidates become exact 64-bit keys (order-preserving
 //      logit key, then the complement of the expert index, so that equal
 //      logits go to the lower index).  Batches of 8 are sorted by a 19-
@@ -310,7 +312,9 @@ __device__ __forceinline__ uint64_t cand_key(float v, int e)
 }
 
 template <int E>
-constexpr size_t tpt_smem() { return (size_t)32 * E * 4 + (size_t)32 * E; }
+constexpr int tpt_cap() { return E > 64 ? 64 : E; }  // candidate list entries per lane
+template <int E>
+constexpr size_t tpt_smem() { return (size_t)32 * E * 4 + (size_t)32 * tpt_cap<E>(); }
 
 // One warp per CTA, one tile of 32 consecutive tokens (one per lane).
 template <int E, int KC>
@@ -321,6 +325,8 @@ __global__ void __launch_bounds__(32)
 {
     constexpr int NCH = E / 4;
     constexpr int NG = kTptGroups;
+    constexpr int CAP = tpt_cap<E>();
+    __shared__ float s_th[32];
     static_assert(KC >= 1 && KC <= 8 && NCH >= NG && (NCH & (NCH - 1)) == 0, "shape");
     extern __shared__ __align__(16) unsigned char smem[];
     float *rows = reinterpret_cast<float *>(smem);                      // [32][E]
@@ -396,22 +402,24 @@ __global__ void __launch_bounds__(32)
                 const int ch = (g + NG * j + lane) & (NCH - 1);
                 const float4 q = row4[ch];
                 const int e0 = ch * 4;
-                if (q.x >= th) { lst[32 * n] = (uint8_t)e0; ++n; }
-                if (q.y >= th) { lst[32 * n] = (uint8_t)(e0 + 1); ++n; }
-                if (q.z >= th) { lst[32 * n] = (uint8_t)(e0 + 2); ++n; }
-                if (q.w >= th) { lst[32 * n] = (uint8_t)(e0 + 3); ++n; }
+                if (q.x >= th) { lst[32 * min(n, CAP - 1)] = (uint8_t)e0; ++n; }
+                if (q.y >= th) { lst[32 * min(n, CAP - 1)] = (uint8_t)(e0 + 1); ++n; }
+                if (q.z >= th) { lst[32 * min(n, CAP - 1)] = (uint8_t)(e0 + 2); ++n; }
+                if (q.w >= th) { lst[32 * min(n, CAP - 1)] = (uint8_t)(e0 + 3); ++n; }
             }
         }
-        // fewer than k candidates happens only with NaN logits (outside the
-        // contract): take every element, so the indices stay valid and distinct
+        s_th[lane] = th;  // for the overflow path below
         if (n < KC) {
-            for (int e = 0; e < E; ++e) lst[32 * e] = (uint8_t)e;
-            n = E;
+            // fewer than k candidates happens only with NaN logits (outside
+            // the contract): every element becomes a candidate, through the
+            // overflow path, so the indices stay valid and distinct
+            n = E + 1;
         }
     }
 
     // 3. sorted top 8 of the candidates, batches of 8
-    const int nmax = (int)__reduce_max_sync(0xffffffffu, (unsigned)n);
+    const int nb = n > CAP ? 0 : n;
+    const int nmax = (int)__reduce_max_sync(0xffffffffu, (unsigned)nb);
     uint64_t best[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) best[i] = 0ull;
@@ -420,7 +428,7 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             uint64_t key = 0ull;  // below every logit's key
-            if (s + j < n) {
+            if (s + j < nb) {
                 const int e = lst[32 * (s + j)];
                 key = cand_key(row[e], e);
             }
@@ -434,6 +442,25 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
             for (int i = 0; i < 8; ++i) best[i] = best[i] > bt[7 - i] ? best[i] : bt[7 - i];
             bitonic8(best);
+        }
+    }
+    // a lane with more candidates than its list holds (heavy ties, NaN rows)
+    // inserts them into its sorted top 8 straight from the row; the loop is
+    // kept compact so that it costs the common path nothing
+    if (__any_sync(0xffffffffu, n > CAP) && n > CAP) {
+        const float th = s_th[lane];
+        const bool all = n > E;  // NaN row: every element
+#pragma unroll 1
+        for (int e = 0; e < E; ++e) {
+            const float v = row[e];
+            if (!(all || v >= th)) continue;
+            uint64_t key = cand_key(v, e);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint64_t hi = best[i] > key ? best[i] : key;
+                key = best[i] > key ? key : best[i];
+                best[i] = hi;
+            }
         }
     }
     if (!live) return;
