@@ -16,7 +16,9 @@ torch.distributed steps around them:
      address -- torch symmetric memory, whose peer pointers map the other
      GPUs' buffers over NVLink -- or plain local tensors when the group has
      one rank (or for tests that play every rank on one GPU);
-  5. dispatch, a barrier, the receiver's partial sums, a barrier, combine.
+  5. ``dispatch``: the rows into the destinations, then a barrier; the
+     receiver's experts and ``md_combine_partials``; ``combine``: a barrier,
+     then the return rows read back and summed.
 
 No step here computes anything of the method: the counts, offsets, rows and
 sums all come from the library.  The data path has no library collective
@@ -55,22 +57,27 @@ class ExchangeBuffers:
     dispatch sends a token at most one row per rank, so the group's token
     count bounds it)."""
 
-    def __init__(self, rows_cap: int, H: int, k: int, device, group=None):
+    def __init__(self, rows_cap: int, H: int, k: int, device, group=None, symmetric=None):
         import torch.distributed as dist
         self.rows_cap, self.H, self.k = int(rows_cap), int(H), int(k)
-        self.world = dist.get_world_size(group) if dist.is_available() and dist.is_initialized() else 1
-        self.rank = dist.get_rank(group) if self.world > 1 else 0
+        self.group = group
+        on = dist.is_available() and dist.is_initialized()
+        self.world = dist.get_world_size(group) if on else 1
+        self.rank = dist.get_rank(group) if on else 0
+        # symmetric memory whenever other ranks must reach these buffers (and
+        # on request, e.g. to exercise it with a one-rank group)
+        self.symmetric = (self.world > 1) if symmetric is None else bool(symmetric)
         shapes = {"rows": ((self.rows_cap, H), torch.bfloat16), "token": ((self.rows_cap,), torch.int32),
                   "slot_idx": ((self.rows_cap, k), torch.int32),
                   "slot_w": ((self.rows_cap, k), torch.float32),
                   "ret": ((self.rows_cap, H), torch.bfloat16)}
         self.local = {}
         self.ptrs = {}
-        if self.world > 1:
+        if self.symmetric:
             import torch.distributed._symmetric_memory as symm
             for name, (shape, dtype) in shapes.items():
                 t = symm.empty(*shape, dtype=dtype, device=device)
-                h = symm.rendezvous(t, group)
+                h = symm.rendezvous(t, group if group is not None else dist.group.WORLD)
                 self.local[name] = t
                 self.ptrs[name] = list(h.buffer_ptrs)
         else:
@@ -93,6 +100,40 @@ class ExchangeBuffers:
                 out.append(md.PeerRows(rows=self.ptrs["ret"][d], row_base=dst_row_base[d],
                                        rows_cap=caps[d]))
         return out
+
+
+def dispatch(x, topk_idx, topk_w, expert_to_rank, E, bufs: ExchangeBuffers, dev_status=None):
+    """This rank's side of the dispatch all-to-all.
+
+    x bf16 [T, H] and topk_idx / topk_w [T, k] are this rank's T tokens (the
+    group's tokens are the ranks' blocks in rank order, so token t here is
+    global token rank*T + t).  Lays the tokens out (dedup), exchanges the
+    layout offsets, writes every row into its destination rank's buffers and
+    waits for the group.  Returns (layout, rows received): bufs.local["rows"]
+    [:rows], ["token"], ["slot_idx"], ["slot_w"] then hold what this rank's
+    experts must process, in (source rank, token) order."""
+    R, me = bufs.world, bufs.rank
+    T = x.shape[0]
+    L = md.md_dispatch_layout(topk_idx, E, R, expert_to_rank, md.MD_DEDUP, dev_status=dev_status)
+    gathered = gather_rank_offsets(L.rank_offsets, bufs.group)
+    base, recv = plan(gathered, me)
+    md.md_dispatch_exchange(x, topk_idx, topk_w, expert_to_rank, E, L.row_of_slot, L.rank_offsets,
+                            me * T, bufs.peers(base, [bufs.rows_cap] * R), dev_status=dev_status)
+    L.exchange_base = base  # where this rank's blocks sit on every destination
+    barrier(bufs.group)
+    return L, int(recv[R])
+
+
+def combine(L, topk_idx, expert_to_rank, E, bufs: ExchangeBuffers, out=None, dev_status=None):
+    """This rank's side of the combine all-to-all: once every rank has written
+    its return rows (bufs.local["ret"], one per received row, e.g. with
+    md_combine_partials) and the group has met, read the return rows of this
+    rank's tokens from their ranks and sum them."""
+    barrier(bufs.group)
+    R = bufs.world
+    return md.md_combine_exchange(bufs.peers(L.exchange_base, [bufs.rows_cap] * R, which="combine"),
+                                  topk_idx, expert_to_rank, E, L.row_of_slot, L.rank_offsets,
+                                  bufs.H, out=out, dev_status=dev_status)
 
 
 def barrier(group=None):
