@@ -189,6 +189,31 @@ __global__ void __launch_bounds__(256)
     for (int b = threadIdx.x; b < nbk; b += 256) tile_hist[(int64_t)blockIdx.x * nbk + b] = h[b];
 }
 
+// LSD radix sort of the 64-bit confidence keys (pair form of the shuffle):
+// 11-bit digits, at most six passes.
+constexpr int kRadixBits = 11;
+constexpr int kRadixBuckets = 1 << kRadixBits;
+constexpr int kRadixPasses = (64 + kRadixBits - 1) / kRadixBits;
+
+// Fewer digits suffice when the row totals are small.  With every total below
+// 2^b, two different fractions differ by more than 2^-2b, so
+// floor(num * 2^S / den) with S = 2b + 1 still orders them exactly and keeps
+// equal ones equal; it is key >> (63 - S) (a floor of a floor), and it needs
+// S + 1 bits.  The passes above those bits would see one constant digit, an
+// identity for a stable sort, and are skipped.
+struct RadixPlan {
+    int r;      // right shift of the 63-bit key
+    int passes; // LSD passes needed
+};
+
+__device__ __forceinline__ RadixPlan radix_plan(const uint32_t *maxden)
+{
+    const uint32_t d = *maxden;
+    const int b = d ? 32 - __clz(d) : 0;
+    const int S = 2 * b + 1 < 63 ? 2 * b + 1 : 63;
+    return {63 - S, (S + 1 + kRadixBits - 1) / kRadixBits};
+}
+
 // tile_hist[tile][b] <- items of bucket b in the tiles before `tile` (column
 // scan), and row n_tiles <- the first output position of bucket b (scan of
 // the bucket totals); a scatter starts bucket b of a tile at the sum of the
@@ -315,8 +340,14 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
     k_shuf_greedy(const int32_t *__restrict__ order, const int32_t *__restrict__ idx_l, int k,
                   ShufWs ws, const unsigned char *__restrict__ tpref,
                   const unsigned long long *__restrict__ tconf, int64_t T, int E, int R, int64_t Tr,
-                  int32_t *__restrict__ pred, int32_t *status)
+                  int32_t *__restrict__ pred, int32_t *status,
+                  const int32_t *__restrict__ order_even = nullptr,
+                  const uint32_t *__restrict__ maxden = nullptr)
 {
+    // pair form: the radix sort ran radix_plan(maxden).passes passes, which
+    // alternate between two buffers starting with `order`; an even count ends
+    // in `order_even`
+    if (PAIR && maxden && (radix_plan(maxden).passes & 1) == 0) order = order_even;
     extern __shared__ __align__(16) unsigned char g_raw[];
     int *s_first = reinterpret_cast<int *>(g_raw);                    // [E]
     unsigned char *s_pref = g_raw + (size_t)E * sizeof(int);          // [E*R]
@@ -533,9 +564,6 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
 // confidences exactly and equal confidences get equal keys.  Tokens are then
 // sorted by (key desc, t asc) with a stable LSD radix sort (11-bit digits),
 // and the greedy walks each token's own preference list.
-constexpr int kRadixBits = 11;
-constexpr int kRadixBuckets = 1 << kRadixBits;
-constexpr int kRadixPasses = (64 + kRadixBits - 1) / kRadixBits;
 constexpr int kPairWarps = 8;
 
 struct PairWs {
@@ -544,6 +572,8 @@ struct PairWs {
     int32_t *seq_a, *seq_b;    // [T]   radix sort ping-pong
     int32_t *keys;             // [T]   bucket of each token in the final partition
     int32_t *tile_hist;        // [(n_tiles + 1) * max(2^11, R)]
+    uint32_t *maxden;          // [1]   largest row total used by a token
+    uint32_t *ticket;          // [1]   CTAs done in the current radix scan
 };
 
 size_t pair_layout(int64_t T, int R, PairWs *w, void *base)
@@ -565,41 +595,58 @@ size_t pair_layout(int64_t T, int R, PairWs *w, void *base)
     x.keys = reinterpret_cast<int32_t *>(take((size_t)Tn * 4));
     const int nbk = kRadixBuckets > R ? kRadixBuckets : R;
     x.tile_hist = reinterpret_cast<int32_t *>(take((size_t)(n_tiles + 1) * nbk * 4));
+    x.maxden = reinterpret_cast<uint32_t *>(take(8));
+    x.ticket = x.maxden ? x.maxden + 1 : nullptr;
     if (w) *w = x;
     return o;
 }
 
-__global__ void __launch_bounds__(kPairWarps * 32)
+// floor(num * 2^63 / den) for num <= den < 2^31, exactly, in two 64-bit
+// long-division steps: num * 2^63 = (num * 2^32) * 2^31, and the remainder
+// of the first step (< den) shifted by 31 still fits in 64 bits.
+__device__ __forceinline__ unsigned long long conf_key(uint64_t num, uint64_t den)
+{
+    const uint64_t a = num << 32;
+    const uint64_t q1 = a / den, r1 = a - q1 * den;
+    const uint64_t q2 = (r1 << 31) / den;
+    return (q1 << 31) + q2;
+}
+
+// One warp per token.  Lane j holds the row entries of experts j, j+32, ...
+// (E <= 256: at most 8), so the row is read once; the per-rank sums are
+// shared-memory atomics of those entries, and the preference order compares
+// one 64-bit key per rank, (sum << 7) | (127 - rank): larger sum first, lower
+// rank on ties.
+constexpr int kPairPerLane = MD_MAX_PAIR_EXPERTS / 32;
+
+__global__ void __launch_bounds__(kPairWarps * 32, 4)
     k_pair_rows(const int32_t *__restrict__ idx_p, const int32_t *__restrict__ idx_l, int k,
                 const uint32_t *__restrict__ C, const uint32_t *__restrict__ C2,
                 const int32_t *__restrict__ p_next, int64_t T, int E, int R, uint32_t min_obs,
                 PairWs ws, int32_t *__restrict__ use_pair, int32_t *status)
 {
     __shared__ unsigned long long s_sig[kPairWarps][MD_MAX_RANKS];
-    __shared__ int s_rmem[MD_MAX_PAIR_EXPERTS];   // experts grouped by next-layer rank
-    __shared__ int s_rstart[MD_MAX_RANKS + 1];
     const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
     unsigned long long *sig = s_sig[wl];
-    if (threadIdx.x == 0) {
-        // counting sort of the experts by rank; an out-of-range rank is
-        // reported and the expert left out of every rank's sum
-        for (int d = 0; d <= R; ++d) s_rstart[d] = 0;
-        for (int e = 0; e < E; ++e) {
-            const int d = p_next[e];
-            if (d >= 0 && d < R) ++s_rstart[d + 1];
-            else md::report(status, MD_ERR_DATA);
+    // next-layer rank of each of this lane's experts; an out-of-range rank is
+    // reported and the expert left out of every rank's sum
+    int rk[kPairPerLane];
+#pragma unroll
+    for (int j = 0; j < kPairPerLane; ++j) {
+        const int e = lane + 32 * j;
+        int d = -1;
+        if (e < E) {
+            d = __ldg(p_next + e);
+            if (d < 0 || d >= R) {
+                if (blockIdx.x == 0 && wl == 0) md::report(status, MD_ERR_DATA);
+                d = -1;
+            }
         }
-        for (int d = 0; d < R; ++d) s_rstart[d + 1] += s_rstart[d];
-        int fill[MD_MAX_RANKS];
-        for (int d = 0; d < R; ++d) fill[d] = s_rstart[d];
-        for (int e = 0; e < E; ++e) {
-            const int d = p_next[e];
-            if (d >= 0 && d < R) s_rmem[fill[d]++] = e;
-        }
+        rk[j] = d;
     }
-    __syncthreads();
     const int64_t w0 = (int64_t)blockIdx.x * kPairWarps + wl;
     const int64_t nw = (int64_t)gridDim.x * kPairWarps;
+    uint32_t maxden = 0;  // lane 0: the largest row total of this warp's tokens
     for (int64_t t = w0; t < T; t += nw) {
         int a = __ldg(idx_p + t * k), b = __ldg(idx_l + t * k);
         if (a < 0 || a >= E || b < 0 || b >= E) {
@@ -608,123 +655,256 @@ __global__ void __launch_bounds__(kPairWarps * 32)
             b = b < 0 || b >= E ? 0 : b;
         }
         const uint32_t *prow = C2 + ((int64_t)a * E + b) * E;
+        uint32_t v[kPairPerLane];
         unsigned long long psum = 0;
-        for (int e = lane; e < E; e += 32) psum += __ldg(prow + e);
+#pragma unroll
+        for (int j = 0; j < kPairPerLane; ++j) {
+            v[j] = lane + 32 * j < E ? __ldg(prow + lane + 32 * j) : 0u;
+            psum += v[j];
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, o);
         const bool use = psum >= min_obs;
-        const uint32_t *row = use ? prow : C + (int64_t)b * E;
-        // per-rank sums: lane d adds its rank's experts
-        for (int d = lane; d < R; d += 32) {
-            unsigned long long sd = 0;
-            for (int i = s_rstart[d]; i < s_rstart[d + 1]; ++i) sd += __ldg(row + s_rmem[i]);
-            sig[d] = sd;
+        if (!use) {
+            const uint32_t *row = C + (int64_t)b * E;
+#pragma unroll
+            for (int j = 0; j < kPairPerLane; ++j)
+                v[j] = lane + 32 * j < E ? __ldg(row + lane + 32 * j) : 0u;
         }
-        // total and arg-max (lowest index on ties)
-        unsigned long long tot = 0;
-        uint32_t bv = 0;
-        int be = INT_MAX;
-        for (int e = lane; e < E; e += 32) {
-            const uint32_t v = __ldg(row + e);
-            tot += v;
-            if (v > bv || (v == bv && e < be)) {
-                bv = v;
-                be = e;
-            }
+        for (int d = lane; d < R; d += 32) sig[d] = 0ull;
+        __syncwarp();
+        // per-rank sums, total and arg-max (lowest expert on ties)
+        unsigned long long tot = 0, best = 0;
+#pragma unroll
+        for (int j = 0; j < kPairPerLane; ++j) {
+            const int e = lane + 32 * j;
+            if (e >= E) continue;
+            if (rk[j] >= 0 && v[j]) atomicAdd(&sig[rk[j]], (unsigned long long)v[j]);
+            tot += v[j];
+            const unsigned long long c = ((unsigned long long)v[j] << 32) | (0xffffffffu - (unsigned)e);
+            best = c > best ? c : best;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             tot += __shfl_xor_sync(0xffffffffu, tot, o);
-            const uint32_t v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int e2 = __shfl_xor_sync(0xffffffffu, be, o);
-            if (v2 > bv || (v2 == bv && e2 < be)) {
-                bv = v2;
-                be = e2;
-            }
+            const unsigned long long c = __shfl_xor_sync(0xffffffffu, best, o);
+            best = c > best ? c : best;
+        }
+        const uint32_t bv = (uint32_t)(best >> 32);
+        const int be = (int)(0xffffffffu - (uint32_t)best);
+        __syncwarp();
+        for (int d = lane; d < R; d += 32) {
+            const unsigned long long sd = sig[d];
+            sig[d] = ((sd < (1ull << 56) ? sd : (1ull << 56) - 1) << 7) | (unsigned)(127 - d);
         }
         __syncwarp();
         int first = __ldg(p_next + be);
         if (first < 0 || first >= R) first = 0;
         unsigned char *pl = ws.tpref + t * pref_stride(R);
-        for (int d = lane; d < R; d += 32) {
-            int pos = 0;
-            if (d != first) {
-                pos = 1;
-                for (int d2 = 0; d2 < R; ++d2)
-                    if (d2 != first && d2 != d && (sig[d2] > sig[d] || (sig[d2] == sig[d] && d2 < d)))
-                        ++pos;
+        // position of rank d: 0 for `first`; else 1 + the ranks other than
+        // `first` whose key is larger.  With R <= 16 the two half-warps each
+        // count half of the ranks.
+        if (R <= 16) {
+            const int d = lane & 15, half = lane >> 4;
+            int n = 0;
+            if (d < R) {
+                const unsigned long long kd = sig[d];
+                const int lo = half * 8, hi = min(R, lo + 8);
+                for (int d2 = lo; d2 < hi; ++d2) n += d2 != first && sig[d2] > kd;
             }
-            pl[pos] = (unsigned char)d;
+            n += __shfl_xor_sync(0xffffffffu, n, 16);
+            if (half == 0 && d < R) pl[d == first ? 0 : 1 + n] = (unsigned char)d;
+        } else {
+            for (int d = lane; d < R; d += 32) {
+                const unsigned long long kd = sig[d];
+                int n = 0;
+                for (int d2 = 0; d2 < R; ++d2) n += d2 != first && sig[d2] > kd;
+                pl[d == first ? 0 : 1 + n] = (unsigned char)d;
+            }
         }
         if (lane == 0) {
             unsigned long long key = 0ull;
             if (tot > 0) {
-                if (tot >= (1ull << 31)) md::report(status, MD_ERR_UNSUPPORTED);
-                key = (unsigned long long)(((unsigned __int128)bv << 63) / tot);
+                if (tot >= (1ull << 31)) {
+                    md::report(status, MD_ERR_UNSUPPORTED);
+                } else {
+                    key = conf_key(bv, tot);
+                    maxden = (uint32_t)tot > maxden ? (uint32_t)tot : maxden;
+                }
             }
             ws.conf[t] = key;
             if (use_pair) use_pair[t] = use ? 1 : 0;
         }
         __syncwarp();
     }
+    if (lane == 0 && maxden) atomicMax(ws.maxden, maxden);
 }
 
 // digit of the sort key for one LSD pass: confidence descending
-__device__ __forceinline__ int radix_digit(const unsigned long long *conf, int32_t tok, int shift)
+__device__ __forceinline__ int radix_digit(const unsigned long long *conf, int32_t tok, int shift, int r)
 {
-    return (int)((~conf[tok] >> shift) & (kRadixBuckets - 1));
+    return (int)((~(conf[tok] >> r) >> shift) & (kRadixBuckets - 1));
 }
 
 __global__ void __launch_bounds__(256)
     k_radix_hist(const int32_t *__restrict__ seq, const unsigned long long *__restrict__ conf,
-                 int64_t T, int shift, int32_t *__restrict__ tile_hist)
+                 int64_t T, int pass, const uint32_t *__restrict__ maxden,
+                 int32_t *__restrict__ tile_hist)
 {
+    const RadixPlan pl = radix_plan(maxden);
+    if (pass >= pl.passes) return;
+    const int shift = pass * kRadixBits;
     __shared__ int h[kRadixBuckets];
     for (int b = threadIdx.x; b < kRadixBuckets; b += 256) h[b] = 0;
     __syncthreads();
     const int64_t t0 = (int64_t)blockIdx.x * kTile;
     for (int i = threadIdx.x; i < kTile; i += 256) {
         const int64_t pos = t0 + i;
-        if (pos < T) atomicAdd(&h[radix_digit(conf, seq ? seq[pos] : (int32_t)pos, shift)], 1);
+        if (pos < T) atomicAdd(&h[radix_digit(conf, seq ? seq[pos] : (int32_t)pos, shift, pl.r)], 1);
     }
     __syncthreads();
     for (int b = threadIdx.x; b < kRadixBuckets; b += 256)
         tile_hist[(int64_t)blockIdx.x * kRadixBuckets + b] = h[b];
 }
 
-// One warp per tile, items in sequence order, stable within each digit.
-__global__ void __launch_bounds__(32)
-    k_radix_scatter(const int32_t *__restrict__ seq, const unsigned long long *__restrict__ conf,
-                    int64_t T, int shift, const int32_t *__restrict__ tile_hist,
-                    int32_t *__restrict__ seq_out)
+// Column scan of the radix histogram, spread over the GPU: CTA c takes
+// digits [32c, 32c+32) (a lane each, so every tile row is read in 128-byte
+// pieces) and its 8 warps split the tiles into 8 runs; a run's sum goes
+// through shared memory to the runs after it.  tile_hist[tile][b] becomes
+// the items of digit b in the tiles before `tile`; the last warp leaves the
+// column total in row n_tiles.  The last CTA to finish (a ticket, no wait)
+// turns that row into the exclusive scan over the digits and puts the ticket
+// back to 0 for the next pass.
+constexpr int kRsWarps = 8;
+
+__global__ void __launch_bounds__(kRsWarps * 32)
+    k_radix_scan(int32_t *__restrict__ tile_hist, int n_tiles, int pass,
+                 const uint32_t *__restrict__ maxden, uint32_t *__restrict__ ticket)
 {
-    __shared__ int cnt[kRadixBuckets];
-    const int lane = threadIdx.x;
-    const int32_t *base = tile_hist + (int64_t)gridDim.x * kRadixBuckets;
-    for (int b = lane; b < kRadixBuckets; b += 32)
-        cnt[b] = tile_hist[(int64_t)blockIdx.x * kRadixBuckets + b] + base[b];
-    const int64_t t0 = (int64_t)blockIdx.x * kTile;
-    int tok[kTile / 32], dg[kTile / 32];
+    if (pass >= radix_plan(maxden).passes) return;
+    __shared__ int s_seg[kRsWarps][32];
+    __shared__ int s_warp[kRsWarps];
+    __shared__ int s_last;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    const int b = blockIdx.x * 32 + lane;
+    const int per = (n_tiles + kRsWarps - 1) / kRsWarps;
+    const int lo = min(n_tiles, wp * per), hi = min(n_tiles, lo + per);
+    int sum = 0;
+    for (int i0 = lo; i0 < hi; i0 += 8) {
+        int v[8];
 #pragma unroll
-    for (int c = 0; c < kTile / 32; ++c) {
+        for (int u = 0; u < 8; ++u)
+            v[u] = i0 + u < hi ? tile_hist[(int64_t)(i0 + u) * kRadixBuckets + b] : 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sum += v[u];
+    }
+    s_seg[wp][lane] = sum;
+    __syncthreads();
+    int run = 0;
+    for (int w = 0; w < wp; ++w) run += s_seg[w][lane];
+    for (int i0 = lo; i0 < hi; i0 += 8) {
+        int v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            v[u] = i0 + u < hi ? tile_hist[(int64_t)(i0 + u) * kRadixBuckets + b] : 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (i0 + u < hi) {
+                tile_hist[(int64_t)(i0 + u) * kRadixBuckets + b] = run;
+                run += v[u];
+            }
+    }
+    int32_t *totals = tile_hist + (int64_t)n_tiles * kRadixBuckets;
+    if (wp == kRsWarps - 1) totals[b] = run;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    constexpr int kPer = kRadixBuckets / (kRsWarps * 32);
+    int t[kPer];
+    int own = 0;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        t[j] = __ldcg(totals + tid * kPer + j);
+        own += t[j];
+    }
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_warp[wp] = incl;
+    __syncthreads();
+    int acc = incl - own;
+    for (int w = 0; w < wp; ++w) acc += s_warp[w];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        totals[tid * kPer + j] = acc;
+        acc += t[j];
+    }
+    if (tid == 0) *ticket = 0u;
+}
+
+// One tile per CTA, items in sequence order, stable within each digit.  The
+// tile's four warps take a quarter each: a warp ranks its items per digit
+// (__match_any_sync, 8 rounds of 32), then every digit's start is laid out
+// over the warps in order, and each item goes to its warp's start plus its
+// rank.
+constexpr int kScatWarps = 4;
+constexpr int kScatItems = kTile / (kScatWarps * 32);
+
+__global__ void __launch_bounds__(kScatWarps * 32)
+    k_radix_scatter(const int32_t *__restrict__ seq, const unsigned long long *__restrict__ conf,
+                    int64_t T, int pass, const uint32_t *__restrict__ maxden,
+                    const int32_t *__restrict__ tile_hist, int32_t *__restrict__ seq_out)
+{
+    __shared__ int wcnt[kScatWarps][kRadixBuckets];
+    const RadixPlan pl = radix_plan(maxden);
+    if (pass >= pl.passes) return;  // identity: the reader takes the last pass's buffer
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    const int shift = pass * kRadixBits;
+    for (int i = tid; i < kScatWarps * kRadixBuckets; i += kScatWarps * 32) (&wcnt[0][0])[i] = 0;
+    const int64_t t0 = (int64_t)blockIdx.x * kTile + wp * (kTile / kScatWarps);
+    int tok[kScatItems], dg[kScatItems], rk[kScatItems];
+#pragma unroll
+    for (int c = 0; c < kScatItems; ++c) {
         const int64_t pos = t0 + c * 32 + lane;
         tok[c] = pos < T ? (seq ? seq[pos] : (int32_t)pos) : -1;
     }
 #pragma unroll
-    for (int c = 0; c < kTile / 32; ++c) dg[c] = tok[c] >= 0 ? radix_digit(conf, tok[c], shift) : -1;
-    __syncwarp();
+    for (int c = 0; c < kScatItems; ++c)
+        dg[c] = tok[c] >= 0 ? radix_digit(conf, tok[c], shift, pl.r) : -1;
+    __syncthreads();
+    int *cw = wcnt[wp];
 #pragma unroll
-    for (int c = 0; c < kTile / 32; ++c) {
+    for (int c = 0; c < kScatItems; ++c) {
         const int key = dg[c];
         const bool in = key >= 0;
         const unsigned g = __match_any_sync(0xffffffffu, in ? (unsigned)key : (0x80000000u | lane));
-        int pos = 0;
-        if (in) pos = cnt[key] + __popc(g & md::lanemask_lt());
+        rk[c] = in ? cw[key] + __popc(g & md::lanemask_lt()) : 0;
         __syncwarp();
-        if (in && (g >> lane) == 1u) cnt[key] += __popc(g);
+        if (in && (g >> lane) == 1u) cw[key] += __popc(g);
         __syncwarp();
-        if (in) seq_out[pos] = tok[c];
     }
+    __syncthreads();
+    const int32_t *row = tile_hist + (int64_t)blockIdx.x * kRadixBuckets;
+    const int32_t *base = tile_hist + (int64_t)gridDim.x * kRadixBuckets;
+    for (int b = tid; b < kRadixBuckets; b += kScatWarps * 32) {
+        int run = row[b] + base[b];
+#pragma unroll
+        for (int w = 0; w < kScatWarps; ++w) {
+            const int c = wcnt[w][b];
+            wcnt[w][b] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < kScatItems; ++c)
+        if (dg[c] >= 0) seq_out[cw[dg[c]] + rk[c]] = tok[c];
 }
 
 // ------------------------------------------------------ rounds assignment
@@ -1052,22 +1232,24 @@ extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx
     pair_layout(T, R, &pw, workspace);
     const int n_tiles = (int)((T + kTile - 1) / kTile);
     const int64_t Tr = T / R;
+    if (cudaMemsetAsync(pw.maxden, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return MD_ERR_CUDA;
 
     int64_t blocks = (T + kPairWarps - 1) / kPairWarps;
-    const int64_t cap = (int64_t)md::sm_count() * 8;
+    const int64_t cap = (int64_t)md::sm_count() * 4;  // one wave: 4 CTAs per SM
     if (blocks > cap) blocks = cap;
     k_pair_rows<<<(unsigned)blocks, kPairWarps * 32, 0, s>>>(idx_prev, idx_l, k, C, C2,
                                                              expert_to_rank_next, T, E, R, min_obs,
                                                              pw, use_pair, dev_status);
-    // visit order: stable LSD radix sort by (confidence key desc), from t ascending
+    // visit order: stable LSD radix sort by (confidence key desc), from t
+    // ascending; the passes above the key's significant digits do nothing
     const int32_t *in = nullptr;
     int32_t *out = pw.seq_a;
     for (int pass = 0; pass < kRadixPasses; ++pass) {
-        const int shift = pass * kRadixBits;
-        k_radix_hist<<<n_tiles, 256, 0, s>>>(in, pw.conf, T, shift, pw.tile_hist);
-        k_bucket_scan<<<1, kScanThreads, kRadixBuckets * sizeof(int), s>>>(pw.tile_hist, n_tiles,
-                                                                  kRadixBuckets);
-        k_radix_scatter<<<n_tiles, 32, 0, s>>>(in, pw.conf, T, shift, pw.tile_hist, out);
+        k_radix_hist<<<n_tiles, 256, 0, s>>>(in, pw.conf, T, pass, pw.maxden, pw.tile_hist);
+        k_radix_scan<<<kRadixBuckets / 32, kRsWarps * 32, 0, s>>>(pw.tile_hist, n_tiles, pass,
+                                                                  pw.maxden, pw.ticket);
+        k_radix_scatter<<<n_tiles, kScatWarps * 32, 0, s>>>(in, pw.conf, T, pass, pw.maxden,
+                                                            pw.tile_hist, out);
         in = out;
         out = out == pw.seq_a ? pw.seq_b : pw.seq_a;
     }
@@ -1076,8 +1258,9 @@ extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx
     if (cudaFuncSetAttribute(k_shuf_greedy<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)lsm) != cudaSuccess)
         return MD_ERR_CUDA;
-    k_shuf_greedy<true><<<1, kGreedyThreads, lsm, s>>>(in, nullptr, k, none, pw.tpref, pw.conf, T, E,
-                                                       R, Tr, pred_rank, dev_status);
+    k_shuf_greedy<true><<<1, kGreedyThreads, lsm, s>>>(pw.seq_a, nullptr, k, none, pw.tpref, pw.conf,
+                                                       T, E, R, Tr, pred_rank, dev_status, pw.seq_b,
+                                                       pw.maxden);
     // new positions: stable partition by assigned rank
     k_bucket_hist<<<n_tiles, 256, R * sizeof(int), s>>>(1, T, nullptr, k, nullptr, E, pred_rank, R,
                                                        pw.keys, pw.tile_hist);
