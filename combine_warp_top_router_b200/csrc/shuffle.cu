@@ -562,8 +562,9 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
 // For den < 2^31, two different fractions num/den <= 1 differ by at least
 // 2^-62, i.e. by at least 2 after scaling, so the keys order the
 // confidences exactly and equal confidences get equal keys.  Tokens are then
-// sorted by (key desc, t asc) with a stable LSD radix sort (11-bit digits),
-// and the greedy walks each token's own preference list.
+// sorted by (key desc, t asc) with a stable LSD radix sort (11-bit digits,
+// only as many passes as the largest row total calls for: radix_plan), and
+// the greedy walks each token's own preference list.
 constexpr int kPairWarps = 8;
 
 struct PairWs {
