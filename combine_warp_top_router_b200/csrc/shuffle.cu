@@ -327,6 +327,9 @@ __global__ void __launch_bounds__(32)
 //   rank reaches T/R is found from per-warp counts, the chunk is committed up
 //   to it, that rank is marked full, first[] is recomputed and the rest of
 //   the chunk is re-evaluated: exactly the sequential visit.
+// A chunk with no fill event crosses a single block barrier: the per-rank
+// totals go to one of three buffers and the loads to one of two, and every
+// warp reads them back after the barrier and reaches the same decision.
 constexpr int kGreedyThreads = 1024;
 constexpr int kGreedyWarps = kGreedyThreads / 32;
 
@@ -351,29 +354,43 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
     extern __shared__ __align__(16) unsigned char g_raw[];
     int *s_first = reinterpret_cast<int *>(g_raw);                    // [E]
     unsigned char *s_pref = g_raw + (size_t)E * sizeof(int);          // [E*R]
-    __shared__ long long s_load[MD_MAX_RANKS];
-    __shared__ int s_tot[MD_MAX_RANKS];
+    // per-rank loads (two buffers) and per-rank totals of an evaluation (three
+    // buffers): a chunk with no fill event crosses one block barrier, so each
+    // buffer is rewritten only once no thread can still read it
+    __shared__ long long s_load[2][MD_MAX_RANKS];
+    __shared__ int s_tot[3][MD_MAX_RANKS];
     __shared__ int s_cnt[kGreedyWarps][MD_MAX_RANKS];
     __shared__ unsigned s_msk[kGreedyWarps][MD_MAX_RANKS];
-    __shared__ unsigned long long s_full;
-    __shared__ int s_first_any, s_over, s_pmin;
+    __shared__ int s_pmin;
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
 
     if (!PAIR)
         for (int i = tid; i < E * R; i += kGreedyThreads) s_pref[i] = (unsigned char)ws.pref[i];
-    for (int d = tid; d < R; d += kGreedyThreads) {
-        s_load[d] = 0;
-        s_tot[d] = 0;
-    }
-    if (tid == 0) {
-        s_full = 0ull;
-        s_first_any = 0;
-    }
+    for (int i = tid; i < 2 * MD_MAX_RANKS; i += kGreedyThreads) (&s_load[0][0])[i] = 0;
+    for (int i = tid; i < 3 * MD_MAX_RANKS; i += kGreedyThreads) (&s_tot[0][0])[i] = 0;
     __syncthreads();
     if (!PAIR)
         for (int e = tid; e < E; e += kGreedyThreads)
             s_first[e] = ws.den[e] == 0ull ? -1 : (int)s_pref[(size_t)e * R];
     __syncthreads();
+
+    // The set of full ranks: every thread keeps the same copy, derived from
+    // the same shared words after a barrier, so every branch on it is uniform.
+    unsigned long long full = 0ull;
+    const unsigned long long all_ranks = R == 64 ? ~0ull : (1ull << R) - 1ull;
+    int first_any = 0;  // the lowest rank that is not full (0 once all are)
+    int lb = 0, tb = 0;  // current load and total buffers
+    auto refresh_first = [&]() {
+        const unsigned long long open = ~full & all_ranks;
+        first_any = open ? __ffsll((long long)open) - 1 : 0;
+        for (int e = tid; !PAIR && e < E; e += kGreedyThreads) {
+            if (s_first[e] < 0) continue;
+            const unsigned char *pl = s_pref + (size_t)e * R;
+            int n = 0;
+            while (n < R && ((full >> pl[n]) & 1ull)) ++n;
+            s_first[e] = n < R ? (int)pl[n] : 0;
+        }
+    };
 
     // token ids are fetched two chunks ahead and their top-1 experts one chunk
     // ahead, so neither load is waited on in the chunk that uses it
@@ -433,7 +450,6 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
                     f = -1;
                     if (!e1) {
                         const unsigned char *pl = my_list;
-                        const unsigned long long full = s_full;
                         int n = 0;
                         while (n < R && ((full >> pl[n]) & 1ull)) ++n;
                         f = n < R ? (int)pl[n] : 0;
@@ -441,47 +457,38 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
                 } else {
                     f = s_first[e1];
                 }
-                ch = f >= 0 ? f : (((s_full >> src_rank) & 1ull) ? s_first_any : src_rank);
+                ch = f >= 0 ? f : (((full >> src_rank) & 1ull) ? first_any : src_rank);
             }
             const unsigned g =
                 __match_any_sync(0xffffffffu, ch >= 0 ? (unsigned)ch : (0x80000000u | lane));
             const bool leader = ch >= 0 && (g & md::lanemask_lt()) == 0u;
-            if (leader) atomicAdd(&s_tot[ch], __popc(g));
-            if (tid == 0) s_over = 0;
+            if (leader) atomicAdd(&s_tot[tb][ch], __popc(g));
             __syncthreads();
-            for (int d = tid; d < R; d += kGreedyThreads)
-                if (s_load[d] + s_tot[d] > Tr) s_over = 1;
-            __syncthreads();
-            if (!s_over) {
-                // no rank goes past T/R: commit the whole chunk
+            // every warp reads the loads and this evaluation's totals: does a
+            // rank go past T/R, and which ranks end exactly at T/R
+            bool over = false;
+            unsigned long long at_cap = 0ull;
+            for (int d0 = 0; d0 < R; d0 += 32) {
+                const int d = d0 + lane;
+                const long long nl = d < R ? s_load[lb][d] + s_tot[tb][d] : 0;
+                over |= __any_sync(0xffffffffu, d < R && nl > Tr);
+                at_cap |= (unsigned long long)__ballot_sync(0xffffffffu, d < R && nl == Tr) << d0;
+            }
+            if (!over) {
+                // no rank goes past T/R: commit the rest of the chunk at once
                 if (ch >= 0) pred[t] = ch;
-                int newly_full = 0;
                 for (int d = tid; d < R; d += kGreedyThreads) {
-                    s_load[d] += s_tot[d];
-                    s_tot[d] = 0;
-                    if (s_load[d] == Tr && !((s_full >> d) & 1ull)) newly_full = 1;
+                    s_load[lb ^ 1][d] = s_load[lb][d] + s_tot[tb][d];
+                    s_tot[tb == 0 ? 2 : tb - 1][d] = 0;  // the previous evaluation's buffer
                 }
-                if (__syncthreads_or(newly_full)) {
-                    if (tid == 0) {
-                        unsigned long long f = s_full;
-                        for (int d = 0; d < R; ++d)
-                            if (s_load[d] == Tr) f |= 1ull << d;
-                        s_full = f;
-                    }
-                    __syncthreads();
-                    for (int e = tid; !PAIR && e < E; e += kGreedyThreads) {
-                        if (s_first[e] < 0) continue;
-                        const unsigned char *pl = s_pref + (size_t)e * R;
-                        int n = 0;
-                        while (n < R && ((s_full >> pl[n]) & 1ull)) ++n;
-                        s_first[e] = n < R ? (int)pl[n] : 0;
-                    }
-                    if (tid == 0) {
-                        int d = 0;
-                        while (d < R && ((s_full >> d) & 1ull)) ++d;
-                        s_first_any = d < R ? d : 0;
-                    }
-                    __syncthreads();
+                lb ^= 1;
+                tb = tb == 2 ? 0 : tb + 1;
+                if (at_cap & ~full) {
+                    full |= at_cap;
+                    // every thread chose before the barrier above, so the
+                    // per-expert choices can be rewritten now
+                    refresh_first();
+                    if (!PAIR) __syncthreads();
                 }
                 break;
             }
@@ -497,8 +504,8 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
             __syncthreads();
             for (int d = wp; d < R; d += kGreedyWarps) {
                 // ranks that fill inside this chunk (full ranks get no tokens)
-                if (s_tot[d] == 0 || s_load[d] + s_tot[d] < Tr) continue;
-                const long long need = Tr - s_load[d];  // tokens rank d still takes
+                if (s_tot[tb][d] == 0 || s_load[lb][d] + s_tot[tb][d] < Tr) continue;
+                const long long need = Tr - s_load[lb][d];  // tokens rank d still takes
                 int c = s_cnt[lane][d];
                 int incl = c;
 #pragma unroll
@@ -523,29 +530,16 @@ __global__ void __launch_bounds__(kGreedyThreads, 1)
             const unsigned g2 =
                 __match_any_sync(0xffffffffu, commit ? (unsigned)ch : (0x80000000u | lane));
             if (commit && (g2 & md::lanemask_lt()) == 0u)
-                atomicAdd(reinterpret_cast<unsigned long long *>(&s_load[ch]),
+                atomicAdd(reinterpret_cast<unsigned long long *>(&s_load[lb][ch]),
                           (unsigned long long)__popc(g2));
-            for (int d = tid; d < R; d += kGreedyThreads) s_tot[d] = 0;
+            for (int i = tid; i < 3 * MD_MAX_RANKS; i += kGreedyThreads) (&s_tot[0][0])[i] = 0;
             __syncthreads();
-            if (tid == 0) {
-                unsigned long long f = s_full;
-                for (int d = 0; d < R; ++d)
-                    if (s_load[d] == Tr) f |= 1ull << d;
-                s_full = f;
+            for (int d0 = 0; d0 < R; d0 += 32) {
+                const int d = d0 + lane;
+                full |= (unsigned long long)__ballot_sync(0xffffffffu, d < R && s_load[lb][d] == Tr)
+                        << d0;
             }
-            __syncthreads();
-            for (int e = tid; !PAIR && e < E; e += kGreedyThreads) {
-                if (s_first[e] < 0) continue;
-                const unsigned char *pl = s_pref + (size_t)e * R;
-                int n = 0;
-                while (n < R && ((s_full >> pl[n]) & 1ull)) ++n;
-                s_first[e] = n < R ? (int)pl[n] : 0;
-            }
-            if (tid == 0) {
-                int d = 0;
-                while (d < R && ((s_full >> d) & 1ull)) ++d;
-                s_first_any = d < R ? d : 0;
-            }
+            refresh_first();
             __syncthreads();
             if (pmin >= kGreedyThreads - 1) break;
             start = pmin + 1;
