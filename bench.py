@@ -349,16 +349,35 @@ def run_native(args):
     return line
 
 
-def _time(fn, stream, reps):
-    """Average device time (ms) of fn() over reps launches on `stream`, after a warm-up.
-    Inputs are produced on the default stream, which the (non-blocking) timing
-    stream does not wait for: synchronise the device first."""
+def _time(fn, stream, reps, graph=True):
+    """Average device time (ms) of fn() over reps calls on `stream`, after a warm-up.
+    With graph=True the reps calls are captured in one CUDA graph and replayed, so
+    the host's marshalling of each call does not leave the GPU idle between them
+    (a short kernel would otherwise measure the Python call, not the kernel);
+    graph=False times an eager loop, for calls that cannot be captured.  Inputs
+    are produced on the default stream, which the (non-blocking) timing stream
+    does not wait for: synchronise the device first."""
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         fn()
     stream.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(reps):
+                fn()
+        with torch.cuda.stream(stream):
+            g.replay()  # warm replay, on the timing stream like the timed one
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        stream.synchronize()
+        del g
+        return e0.elapsed_time(e1) / reps
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(reps):
@@ -457,7 +476,7 @@ def rows_ep_exchange(args, md, device, stream, peak):
         return g
 
     graphs = [graphed(f) for f in (dispatch, partials, combine)]
-    t_d, t_p, t_c = (_time(g.replay, stream, reps) for g in graphs)
+    t_d, t_p, t_c = (_time(g.replay, stream, reps, graph=False) for g in graphs)
     del graphs
     n = sum(caps)
     # dispatch: x once, each row written once with its metadata (4 + 8k B)
@@ -809,7 +828,7 @@ def rows_config5_planning(args, md, device, stream, peak):
         q = torch.empty(E, dtype=torch.int32, device=device)
         qws = md.alloc_workspace(int(md.lib().md_place_two_level_workspace_size(E, R, nodes)), device)
         t_q = _time(lambda: md.md_place_two_level(W, R, nodes, md.MD_SEED_CONTIGUOUS, refine, out=q,
-                                                  workspace=qws, stream=stream), stream, 3)
+                                                  workspace=qws, stream=stream), stream, 3, graph=False)
         torch.cuda.synchronize()
         Lq = md.md_dispatch_layout(a, E, R, q, md.MD_DEDUP)
         modes[label] = {"us": round(t_q * 1e3, 1),
