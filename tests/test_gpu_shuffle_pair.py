@@ -112,3 +112,28 @@ def test_pair_shuffle_full_size():
     want = oracle.token_shuffle_pair(o[0], o[1], oC, oC2, w.expert_to_rank.cpu().numpy(), w.R, 8 * w.k)
     for gv, ov in zip((pred, perm, inv, use), want):
         assert np.array_equal(gv.cpu().numpy(), ov)
+
+
+# Row totals up to 2^b: the visit order's sort keys then need 2b+2 bits, so the
+# cases run one (all rows empty) to six radix passes; every
+# confidence is distinct at high precision, so a dropped pass or a wrong shift
+# changes the order.
+@pytest.mark.parametrize("bits", [0, 8, 15, 18, 22, 30])
+def test_pair_shuffle_wide_keys(bits):
+    E, k, R, T, min_obs = 64, 2, 16, 16 * 160, 1
+    rng = np.random.default_rng(100 + bits)
+    a, b, _ = (oracle.route_topk(synth.normal_f32(T, E, s, 11).numpy(), k)[0] for s in (4, 5, 6))
+    if bits == 0:
+        C2 = np.zeros((E, E, E), dtype=np.uint32)
+        C = np.zeros((E, E), dtype=np.uint32)
+    else:
+        top = 1 << max(0, bits - 6)  # 64 entries per row: totals below 2^bits
+        C2 = rng.integers(0, top, size=(E, E, E), dtype=np.uint64).astype(np.uint32)
+        C = rng.integers(0, top, size=(E, E), dtype=np.uint64).astype(np.uint32)
+        C2[:, :, 0] = top - 1         # no empty pair rows at the top of the range
+        C2[rng.choice(E, size=8, replace=False), :, :] = 0  # some tokens fall back to C
+    p = shuffled_placement(E, R, 5)
+    got = _gpu_shuffle(a, b, C, C2, p, R, min_obs)
+    want = oracle.token_shuffle_pair(a, b, C, C2, p, R, min_obs)
+    for g, o in zip(got, want):
+        assert np.array_equal(g, o)
