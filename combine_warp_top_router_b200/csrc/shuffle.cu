@@ -1152,6 +1152,35 @@ extern "C" size_t md_token_shuffle_workspace_size(int64_t T, int E, int R)
     return shuf_layout(T, E, R, nullptr, nullptr);
 }
 
+namespace {
+
+// Raises the greedy's shared-memory limit once per device, to the largest size
+// either form asks for (single: E first ranks and E*R preferences; pair: two
+// chunks of per-token lists); false if CUDA refuses.
+bool greedy_smem_ready()
+{
+    static std::atomic<uint64_t> done{0};
+    static std::atomic<int> ok_dev[64];
+    md::once_per_device(done, [] {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const int single = MD_MAX_EXPERTS * (int)sizeof(int) + MD_MAX_EXPERTS * MD_MAX_RANKS;
+        const int pair = 2 * kGreedyThreads * pref_stride(MD_MAX_RANKS);
+        const bool ok =
+            cudaFuncSetAttribute(k_shuf_greedy<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, single) ==
+                cudaSuccess &&
+            cudaFuncSetAttribute(k_shuf_greedy<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, pair) ==
+                cudaSuccess;
+        if (!ok) cudaGetLastError();
+        ok_dev[dev & 63].store(ok ? 1 : 0);
+    });
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return ok_dev[dev & 63].load() != 0;
+}
+
+}  // namespace
+
 extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
                                 const int32_t *expert_to_rank_next, int64_t T, int E, int R,
                                 int32_t *pred_rank, int32_t *perm, int32_t *inv, void *workspace,
@@ -1183,9 +1212,7 @@ extern "C" int md_token_shuffle(const int32_t *idx_l, int k, const uint32_t *C,
     k_bucket_scatter<<<n_tiles, 32, nbk0 * sizeof(int), s>>>(0, T, nbk0, ws.keys, ws.tile_hist,
                                                             ws.order, nullptr, nullptr);
     const size_t gsm = (size_t)E * sizeof(int) + (size_t)E * R;
-    if (cudaFuncSetAttribute(k_shuf_greedy<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsm) !=
-        cudaSuccess)
-        return MD_ERR_CUDA;
+    if (!greedy_smem_ready()) return MD_ERR_CUDA;
     k_shuf_greedy<false><<<1, kGreedyThreads, gsm, s>>>(ws.order, idx_l, k, ws, nullptr, nullptr, T,
                                                         E, R, Tr, pred_rank, dev_status);
     // new positions: stable partition by assigned rank
@@ -1250,9 +1277,7 @@ extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx
     }
     ShufWs none{};
     const size_t lsm = (size_t)2 * kGreedyThreads * pref_stride(R);
-    if (cudaFuncSetAttribute(k_shuf_greedy<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)lsm) != cudaSuccess)
-        return MD_ERR_CUDA;
+    if (!greedy_smem_ready()) return MD_ERR_CUDA;
     k_shuf_greedy<true><<<1, kGreedyThreads, lsm, s>>>(pw.seq_a, nullptr, k, none, pw.tpref, pw.conf,
                                                        T, E, R, Tr, pred_rank, dev_status, pw.seq_b,
                                                        pw.maxden);
