@@ -273,13 +273,14 @@ def run_native(args):
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     barrier(dist, device)
     torch.cuda.synchronize()
-    launches0 = md.launch_count()
+    launches0, memsets0 = md.launch_count(), md.memset_count()
     with ClockSampler(device.index if device.index is not None else 0) as clk:
         with torch.cuda.stream(stream):
             for i in range(args.steps):
                 step(events[i])
         stream.synchronize()
     launches = md.launch_count() - launches0
+    memsets = md.memset_count() - memsets0
     torch.cuda.synchronize()
     barrier(dist, device)
 
@@ -336,6 +337,7 @@ def run_native(args):
                           "frac": round(sum(ab.values()) / (total_ms_max / args.steps * 1e-3) / 1e9 / peak, 4)},
         "kernels": kernels,
         "gpu_launches": int(launches),
+        "device_memsets": int(memsets),
         "e2e": e2e,
         "clocks": clk.summary(),
     }

@@ -36,6 +36,7 @@ _SIGNATURES = {
     "md_status_string": ([_I], ctypes.c_char_p),
     "md_version": ([], _I),
     "md_launch_count": ([], ctypes.c_uint64),
+    "md_memset_count": ([], ctypes.c_uint64),
     "md_route_topk": ([_P, _L, _I, _I, _I, _P, _P, _P], _I),
     "md_dispatch_layout_workspace_size": ([_L, _I, _I, _I, _I], _S),
     "md_dispatch_layout": ([_P, _L, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -104,7 +105,13 @@ def status_string(code: int) -> str:
 
 
 def launch_count() -> int:
+    """Kernels the library has launched in this process."""
     return int(lib().md_launch_count())
+
+
+def memset_count() -> int:
+    """Device memsets and device-to-device copies the library has enqueued."""
+    return int(lib().md_memset_count())
 
 
 def _check(rc: int, what: str):

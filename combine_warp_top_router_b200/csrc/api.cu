@@ -5,7 +5,9 @@
 
 namespace md {
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<uint64_t> g_memsets{0};
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+void count_memsets(int n) { g_memsets.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
 // Fault injection for tests (md_set_test_hooks): a short poll limit and one
 // publish / one copy left out, so that a bounded wait runs out.
@@ -67,3 +69,5 @@ extern "C" const char *md_status_string(int status)
 extern "C" int md_version(void) { return 100; }
 
 extern "C" uint64_t md_launch_count(void) { return md::g_launches.load(std::memory_order_relaxed); }
+
+extern "C" uint64_t md_memset_count(void) { return md::g_memsets.load(std::memory_order_relaxed); }

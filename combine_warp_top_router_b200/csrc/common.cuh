@@ -14,7 +14,8 @@ namespace md {
 // ---------------------------------------------------------------- host side
 
 // Host-side count of enqueued kernels / memsets (md_launch_count).
-void count_launches(int n);
+void count_launches(int n);   // kernels enqueued
+void count_memsets(int n);    // device memsets and device-to-device copies enqueued
 
 // Test hooks (md_set_test_hooks); the defaults leave every kernel unchanged.
 long long hook_poll_limit(long long dflt);
@@ -40,7 +41,7 @@ inline int launch_status()
 inline int clear_status(int32_t *dev_status, cudaStream_t s)
 {
     if (!dev_status) return MD_OK;
-    count_launches(1);
+    count_memsets(1);
     return cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s) == cudaSuccess ? MD_OK : MD_ERR_CUDA;
 }
 

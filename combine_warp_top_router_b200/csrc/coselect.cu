@@ -139,11 +139,11 @@ extern "C" int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, 
     const size_t table = (size_t)E * E * sizeof(uint32_t);
     if (!accumulate) {
         if (W) {
-            md::count_launches(1);
+            md::count_memsets(1);
             if (cudaMemsetAsync(W, 0, table, s) != cudaSuccess) return MD_ERR_CUDA;
         }
         if (C) {
-            md::count_launches(1);
+            md::count_memsets(1);
             if (cudaMemsetAsync(C, 0, table, s) != cudaSuccess) return MD_ERR_CUDA;
         }
     }
@@ -184,7 +184,7 @@ extern "C" int md_coselect_pair_stats(const int32_t *idx_prev, const int32_t *id
     int rc = md::clear_status(dev_status, s);
     if (rc != MD_OK) return rc;
     if (!accumulate) {
-        md::count_launches(1);
+        md::count_memsets(1);
         if (cudaMemsetAsync(C2, 0, (size_t)E * E * E * sizeof(uint32_t), s) != cudaSuccess)
             return MD_ERR_CUDA;
     }

@@ -699,7 +699,7 @@ extern "C" int md_dispatch_layout(const int32_t *topk_idx, int64_t T, int E, int
     // can therefore never let a CTA pass the wait early.
     if ((rc = md::clear_status(dev_status, s)) != MD_OK) return rc;
     if (md::layout_path() != MD_LAYOUT_SPLIT) {  // the split form has no arrival wait
-        md::count_launches(1);
+        md::count_memsets(1);
         if (cudaMemsetAsync(ws.flags, 0, (size_t)kMaxCtas * 4, s) != cudaSuccess) {
             cudaGetLastError();
             return MD_ERR_CUDA;

@@ -1254,6 +1254,7 @@ extern "C" int md_token_shuffle_pair(const int32_t *idx_prev, const int32_t *idx
     pair_layout(T, R, &pw, workspace);
     const int n_tiles = (int)((T + kTile - 1) / kTile);
     const int64_t Tr = T / R;
+    md::count_memsets(1);
     if (cudaMemsetAsync(pw.maxden, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return MD_ERR_CUDA;
 
     int64_t blocks = (T + kPairWarps - 1) / kPairWarps;
@@ -1358,11 +1359,11 @@ extern "C" int md_token_shuffle_rounds(const int32_t *idx_l, int k, const uint32
     shuf_layout(T, E, R, &ws, workspace);
     RoundWs rw;
     round_layout(T, R, &rw, static_cast<char *>(workspace) + need_s);
-    md::count_launches(1);
+    md::count_memsets(1);
     if (cudaMemsetAsync(rw.bar, 0, 256 * 3, s) != cudaSuccess) return MD_ERR_CUDA;  // bar, abort, rounds
     if (T == 0) {
         if (rounds) {
-            md::count_launches(1);
+            md::count_memsets(1);
             if (cudaMemsetAsync(rounds, 0, sizeof(int32_t), s) != cudaSuccess) return MD_ERR_CUDA;
         }
         return MD_OK;
@@ -1395,7 +1396,7 @@ extern "C" int md_token_shuffle_rounds(const int32_t *idx_l, int k, const uint32
                                                          perm, inv);
     md::count_launches(9);
     if (rounds) {
-        md::count_launches(1);
+        md::count_memsets(1);
         if (cudaMemcpyAsync(rounds, rw.rounds, sizeof(int32_t), cudaMemcpyDeviceToDevice, s) !=
             cudaSuccess)
             return MD_ERR_CUDA;

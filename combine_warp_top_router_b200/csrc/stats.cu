@@ -122,7 +122,7 @@ extern "C" int md_rank_stats(const int32_t *topk_idx, int64_t T, int E, int k, i
     cudaStream_t s = md::as_stream(stream);
     int rc = md::clear_status(dev_status, s);
     if (rc != MD_OK) return rc;
-    md::count_launches(1);
+    md::count_memsets(1);
     if (cudaMemsetAsync(hist, 0, sizeof(int64_t) * (size_t)(k + 1), s) != cudaSuccess)
         return MD_ERR_CUDA;
     if (T == 0) return MD_OK;

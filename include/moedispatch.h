@@ -80,9 +80,14 @@ const char *md_status_string(int status);
 /* Library version, major*10000 + minor*100 + patch. */
 int md_version(void);
 
-/* Number of kernels (and device memsets) this library has enqueued in this
- * process so far; a host-side counter for launch accounting. */
+/* Number of kernels this library has launched in this process so far; a
+ * host-side counter for launch accounting. */
 uint64_t md_launch_count(void);
+
+/* Number of device memsets and device-to-device copies this library has
+ * enqueued in this process so far (status words, arrival words, tables it
+ * zeroes before accumulating); counted apart from the kernels. */
+uint64_t md_memset_count(void);
 
 /*
  * md_route_topk -- router top-k selection and gate weights.
