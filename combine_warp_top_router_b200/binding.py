@@ -404,6 +404,8 @@ def md_coselect_stats(idx_l, idx_next, E, T_fit=None, W=None, C=None, accumulate
         W = torch.empty(E, E, dtype=torch.int32, device=dev)
     if C is None and want_C and idx_next is not None:
         C = torch.empty(E, E, dtype=torch.int32, device=dev)
+    if C is not None and idx_next is None:
+        raise ValueError("C needs idx_next (the layer-l+1 top-k)")
     if idx_next is not None and idx_next.shape[1] != k:
         raise ValueError("idx_l and idx_next differ in k")
     if idx_next is not None and idx_next.shape[0] < T_fit:

@@ -130,9 +130,8 @@ extern "C" int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, 
 {
     if (T_fit < 0 || E < 1 || k < 1 || k > MD_MAX_TOPK) return MD_ERR_ARG;
     if (E > MD_MAX_EXPERTS) return MD_ERR_UNSUPPORTED;
-    if (!idx_next) C = nullptr;
     if (!W && !C) return MD_ERR_ARG;
-    if (T_fit > 0 && !idx_l) return MD_ERR_ARG;
+    if (T_fit > 0 && (!idx_l || (C && !idx_next))) return MD_ERR_ARG;
     cudaStream_t s = md::as_stream(stream);
     int rc = md::clear_status(dev_status, s);
     if (rc != MD_OK) return rc;

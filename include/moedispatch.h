@@ -304,11 +304,13 @@ int md_combine(const void *y, int64_t y_rows, const int32_t *assign_row,
  * correlation: experts chosen at layer l predict those at layer l+1.
  *
  *   idx_l     int32 [>= T_fit, k]  layer-l top-k
- *   idx_next  int32 [>= T_fit, k]  layer-l+1 top-k, or NULL (then C unused)
+ *   idx_next  int32 [>= T_fit, k]  layer-l+1 top-k; may be NULL when C is NULL
+ *             or T_fit is 0 (else MD_ERR_ARG)
  *   W         uint32 [E, E] or NULL: W[e][e'] += #{t < T_fit : e, e' in S_l(t)}
  *   C         uint32 [E, E] or NULL: C[e][e'] += #{(t,i,j) : S_l(t)_i = e,
  *                                                     S_l+1(t)_j = e'}
- *   accumulate  0: W and C are cleared first; 1: counts are added.
+ *   accumulate  0: each table given is cleared first (T_fit = 0 leaves it
+ *               zero); 1: counts are added.  At least one of W, C.
  *   Limits: E <= 1024, k <= 32.
  */
 int md_coselect_stats(const int32_t *idx_l, const int32_t *idx_next, int64_t T_fit, int E,
