@@ -73,3 +73,31 @@ def test_shuffles_with_no_tokens():
                 md.md_token_shuffle_pair(none, none, C, C2, p, R, 8, dev_status=st)):
         _ok(st)
         assert all(o.numel() == 0 for o in out[:3])
+
+
+def test_exchange_with_no_tokens():
+    st = md.new_status(DEV)
+    Rx = 2
+    none = torch.empty(0, k, dtype=torch.int32, device=DEV)
+    x = torch.empty(0, H, dtype=torch.bfloat16, device=DEV)
+    p = torch.arange(E, dtype=torch.int32, device=DEV) // (E // Rx)
+    ro = torch.zeros(Rx + 1, dtype=torch.int32, device=DEV)
+    cap = 4
+    bufs = [dict(rows=torch.full((cap, H), 2.0, dtype=torch.bfloat16, device=DEV),
+                 token=_i32(cap), slot_idx=_i32(cap, k),
+                 slot_w=torch.zeros(cap, k, dtype=torch.float32, device=DEV)) for _ in range(Rx)]
+    peers = [md.PeerRows(rows=b["rows"], row_base=0, rows_cap=cap, token=b["token"],
+                         slot_idx=b["slot_idx"], slot_w=b["slot_w"]) for b in bufs]
+    md.md_dispatch_exchange(x, none, torch.empty(0, k, dtype=torch.float32, device=DEV), p, E,
+                            none, ro, 0, peers, dev_status=st)
+    _ok(st)
+    for b in bufs:
+        assert bool((b["rows"] == 2.0).all()) and bool((b["token"] == CANARY).all())
+    z = md.md_combine_partials(torch.ones(4, H, dtype=torch.bfloat16, device=DEV), none, none,
+                               torch.empty(0, k, dtype=torch.float32, device=DEV), dev_status=st)
+    _ok(st)
+    assert z.shape == (0, H)
+    ret = [md.PeerRows(rows=b["rows"], row_base=0, rows_cap=cap) for b in bufs]
+    out = md.md_combine_exchange(ret, none, p, E, none, ro, H, dev_status=st)
+    _ok(st)
+    assert out.shape == (0, H)
