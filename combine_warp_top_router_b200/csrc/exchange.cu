@@ -50,10 +50,36 @@ struct PeerTable {
     md_peer_rows p[MD_MAX_RANKS];
 };
 
-int grid_warps(int64_t units)
+// CTAs of kernel K (kThreads threads, no dynamic shared memory) resident per
+// SM, queried once per device (8 if the query fails).  A grid of at most that
+// many per SM runs in one wave: every CTA walks its share of the units from the
+// start, with no second wave left to finish alone.  The dispatch (over 100
+// registers, two CTAs per SM) gained from it (391 -> 374 us for the 16 calls
+// of the E=128 exchange row); the partials and the combine, four CTAs per SM,
+// did better with 8 CTAs per SM launched (783 against 833 us for the partials).
+template <auto K>
+int resident_per_sm()
+{
+    static std::atomic<uint64_t> done{0};
+    static std::atomic<int> per[64];
+    md::once_per_device(done, [] {
+        int dev = 0, n = 0;
+        cudaGetDevice(&dev);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, K, kThreads, 0) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = 8;
+        }
+        per[dev & 63].store(n);
+    });
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return per[dev & 63].load();
+}
+
+int grid_warps(int64_t units, int per_sm)
 {
     int64_t b = (units + kWarps - 1) / kWarps;
-    const int64_t cap = (int64_t)md::sm_count() * 8;
+    const int64_t cap = (int64_t)md::sm_count() * per_sm;
     if (b > cap) b = cap;
     return b < 1 ? 1 : (int)b;
 }
@@ -428,12 +454,11 @@ extern "C" int md_dispatch_exchange(const void *x, int64_t T, int H, int k, cons
     cudaStream_t s = md::as_stream(stream);
     if ((rc = md::clear_status(dev_status, s)) != MD_OK || T == 0) return rc;
     const int C = H / 8;
-    const unsigned grid = (unsigned)grid_warps(T);
 #define MD_DX(KC)                                                                                  \
-    k_dispatch_exchange<KC><<<grid, kThreads, 0, s>>>(static_cast<const uint4 *>(x), T, C, k,       \
-                                                      topk_idx, topk_w, expert_to_rank, E, R,        \
-                                                      row_of_slot, rank_offsets, token_base, pt,     \
-                                                      dev_status)
+    k_dispatch_exchange<KC><<<(unsigned)grid_warps(T, resident_per_sm<k_dispatch_exchange<KC>>()),  \
+                              kThreads, 0, s>>>(                                                    \
+        static_cast<const uint4 *>(x), T, C, k, topk_idx, topk_w, expert_to_rank, E, R, row_of_slot, \
+        rank_offsets, token_base, pt, dev_status)
     switch (k) {
     case 2: MD_DX(2); break;
     case 4: MD_DX(4); break;
@@ -456,7 +481,7 @@ extern "C" int md_combine_partials(const void *y, int64_t y_rows, const int32_t 
     cudaStream_t s = md::as_stream(stream);
     int rc = md::clear_status(dev_status, s);
     if (rc != MD_OK || n == 0) return rc;
-    k_combine_partials<<<(unsigned)grid_warps(n), kThreads, 0, s>>>(
+    k_combine_partials<<<(unsigned)grid_warps(n, 8), kThreads, 0, s>>>(
         static_cast<const uint4 *>(y), y_rows, y_row, slot_idx, slot_w, n, k, H / 8,
         static_cast<uint4 *>(z), dev_status);
     md::count_launches(1);
@@ -478,11 +503,10 @@ extern "C" int md_combine_exchange(const md_peer_rows *peers, int64_t T, int H, 
     cudaStream_t s = md::as_stream(stream);
     if ((rc = md::clear_status(dev_status, s)) != MD_OK || T == 0) return rc;
     const int C = H / 8;
-    const unsigned grid = (unsigned)grid_warps(T);
 #define MD_CX(KC)                                                                                  \
-    k_combine_exchange<KC><<<grid, kThreads, 0, s>>>(T, C, k, topk_idx, expert_to_rank, E, R,      \
-                                                     row_of_slot, rank_offsets, pt,                \
-                                                     static_cast<uint4 *>(out), dev_status)
+    k_combine_exchange<KC><<<(unsigned)grid_warps(T, 8), kThreads, 0, s>>>(                        \
+        T, C, k, topk_idx, expert_to_rank, E, R, row_of_slot, rank_offsets, pt,                     \
+        static_cast<uint4 *>(out), dev_status)
     switch (k) {
     case 2: MD_CX(2); break;
     case 4: MD_CX(4); break;
