@@ -6,6 +6,9 @@ configuration it times them.
   rows, the combine;
 * the E=256 workload (T=262144, H=2048, R=64) with the correlated placement
   fitted on all tokens: the same, with rows of 4 KiB (the bulk-copy permute);
+* the E=128, top-8 workload (T=65536, H=2048, R=16, contiguous placement) in
+  both dispatch modes, with the two-stage ("wire") combine and the dedup
+  expand the benchmark also times;
 * the token shuffle followed by the dedup layout of the next layer in the
   shuffled order (single-expert and pair-based prediction).
 
@@ -114,6 +117,49 @@ def test_full_e256_k8_full_size():
     OL = oracle.dispatch_layout(oi, E, R, op, oracle.DEDUP)
     _check_layout(L, OL)
     _check_rows_and_combine(w, idx, gates, L, OL, oi, ow, buf, out, 8192, 1024)
+
+
+@pytest.mark.parametrize("mode", [0, 1])
+def test_zipf_pairs_e128_k8_full_size(mode):
+    # T=65536, H=2048, E=128, k=8, R=16, contiguous placement
+    w = synth.make_workload("zipf_pairs_e128_k8", device=DEV)
+    E, k, R = w.E, w.k, w.R
+    idx, gates = md.md_route_topk(w.logits, k)
+    L = md.md_dispatch_layout(idx, E, R, w.expert_to_rank, mode)
+    buf = md.md_dispatch_permute(w.x, L.row_of_slot, out_rows=L.row_capacity)
+    out = md.md_combine(w.y, L.assign_row, idx, gates)
+    torch.cuda.synchronize()
+    oi, ow = oracle.route_topk(w.logits.cpu().numpy(), k)
+    assert np.array_equal(idx.cpu().numpy(), oi)
+    p = w.expert_to_rank.cpu().numpy()
+    OL = oracle.dispatch_layout(oi, E, R, p, mode)
+    _check_layout(L, OL)
+    _check_rows_and_combine(w, idx, gates, L, OL, oi, ow, buf, out, 8192, 1024)
+    if mode != md.MD_DEDUP:
+        return
+    # the expand: every (token, expert) row holds the token's x row
+    xe = md.md_dedup_expand(buf, L.row_of_slot, L.assign_row)
+    torch.cuda.synchronize()
+    assert _inverse_identity(xe, w.x, L.assign_row)
+    del xe
+    # the two-stage combine on sampled tokens: a token's stage-1 rows are its
+    # own, so the oracle runs on the sample with its rows renumbered
+    n = OL["n_rows"]
+    z = torch.empty(n, w.H, dtype=torch.bfloat16, device=DEV)
+    wire = md.md_combine(w.y, L.assign_row, idx, gates, md.MD_COMBINE_WIRE,
+                         row_of_slot=L.row_of_slot, z=z)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(2)
+    toks = np.sort(rng.choice(w.T, 1024, replace=False))
+    ar = OL["assign_row"][toks]
+    rs = OL["row_of_slot"][toks]
+    uniq, local = np.unique(rs, return_inverse=True)
+    ysub = bits(w.y[torch.from_numpy(ar.ravel()).long().to(DEV)])
+    want_out, want_z = oracle.combine(ysub, np.arange(ar.size, dtype=np.int32).reshape(ar.shape),
+                                      oi[toks], ow[toks], oracle.COMBINE_WIRE, p,
+                                      local.reshape(rs.shape).astype(np.int32), len(uniq))
+    assert np.array_equal(bits(wire[torch.from_numpy(toks).long().to(DEV)]), want_out)
+    assert np.array_equal(bits(z[torch.from_numpy(uniq).long().to(DEV)]), want_z)
 
 
 def _chain_gpu(idx_next, inv, E, R, p):
