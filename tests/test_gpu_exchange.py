@@ -128,6 +128,8 @@ def _run(name, T, R, H, placement, seed=0, w=None):
     ("boost_pairs_e128_k2", 2048, 8, 4096, "shuffled"),
     ("full_e256_k8", 4096, 64, 256, "shuffled"),
     ("two_layer_e128_k6", 16 * 48, 16, 264, "shuffled"),   # k = 6 (generic kernel), odd H
+    # the benchmark's size: 16 ranks of 4096 tokens each, rows of 4 KiB
+    ("zipf_pairs_e128_k8", 65536, 16, 2048, "contiguous"),
 ])
 def test_exchange_matches_single_gpu_oracle(name, T, R, H, placement):
     _run(name, T, R, H, placement)
