@@ -15,10 +15,11 @@ in HBM, and each step moves ~17 GB, far more than the 126 MB L2.
 Under torchrun each rank runs an independent replica on its own GPU (the
 virtual EP ranks live inside one GPU; nothing is sharded), times K steps with
 CUDA events, and rank 0 prints one JSON line with the max over ranks.  The
-`rows` object times every other workload of the path on its own (config-2
-conventional and dedup dispatch, the L2-flushed small config, the top-2
-H=4096 config at EP 8 and 32, the token shuffle and the dedup dispatch after
-it, placement modes, routing statistics, the full E=256 pipeline).
+`rows` object times every other workload of the path on its own (the E=128
+top-8 workload in conventional and dedup dispatch, the L2-flushed T=4096 E=64
+workload, the top-2 H=4096 workload at EP 8 and 32, the token shuffle and the
+dedup dispatch after it, placement modes, routing statistics, the full E=256
+pipeline, the EP exchange on one GPU).
 --impl reference times the CPU oracle on the host instead (bounded samples).
 """
 from __future__ import annotations
@@ -398,17 +399,17 @@ def _remote_rows(send_counts):
 def run_rows(args, md, device, stream, peak):
     """Every other workload of the path, each on its own (one GPU)."""
     rows = {}
-    rows.update(rows_config2(args, md, device, stream, peak))
-    rows.update(rows_config1(args, md, device, stream, peak))
-    rows.update(rows_config3(args, md, device, stream, peak))
-    rows.update(rows_config4(args, md, device, stream, peak))
-    rows.update(rows_config5_planning(args, md, device, stream, peak))
+    rows.update(rows_e128_k8(args, md, device, stream, peak))
+    rows.update(rows_e64_k6_l2_flushed(args, md, device, stream, peak))
+    rows.update(rows_e128_k2_fitted(args, md, device, stream, peak))
+    rows.update(rows_token_shuffle(args, md, device, stream, peak))
+    rows.update(rows_e256_k8_planning(args, md, device, stream, peak))
     rows.update(rows_ep_exchange(args, md, device, stream, peak))
     return rows
 
 
 def rows_ep_exchange(args, md, device, stream, peak):
-    """The EP exchange kernels on one GPU: config 2's workload split into its
+    """The EP exchange kernels on one GPU: the E=128 top-8 workload split into its
     16 source ranks of 4096 tokens, each laid out on its own; the dispatch
     exchange writes every source's rows into 16 separate destination buffers,
     every destination forms its return rows, and the combine exchange reads
@@ -498,7 +499,7 @@ def rows_ep_exchange(args, md, device, stream, peak):
     return {"ep_exchange_zipf_pairs_e128_k8": r}
 
 
-def rows_config2(args, md, device, stream, peak):
+def rows_e128_k8(args, md, device, stream, peak):
     """zipf_pairs_e128_k8: conventional and dedup dispatch, wire combine, expand."""
     from combine_warp_top_router_b200 import synth
     rows = {}
@@ -551,7 +552,7 @@ def rows_config2(args, md, device, stream, peak):
     return rows
 
 
-def rows_config1(args, md, device, stream, peak):
+def rows_e64_k6_l2_flushed(args, md, device, stream, peak):
     """iid_e64_k6 (T=4096, 117 MB per kernel, about the size of L2): L2 is
     flushed (a write of twice its size) before every timed launch, and medians
     are reported.  Each kernel, and the whole step, is captured in a CUDA graph
@@ -622,7 +623,7 @@ def rows_config1(args, md, device, stream, peak):
     return {"iid_e64_k6_l2_flushed": r}
 
 
-def rows_config3(args, md, device, stream, peak):
+def rows_e128_k2_fitted(args, md, device, stream, peak):
     """boost_pairs_e128_k2 (T=65536, H=4096, top-2) at EP 8 and 32: placement
     fitted on tokens [0, 4096) (greedy pair seed, then best single swaps),
     dedup dispatch and fused combine; rows per token against contiguous."""
@@ -663,7 +664,7 @@ def rows_config3(args, md, device, stream, peak):
     return rows
 
 
-def rows_config4(args, md, device, stream, peak):
+def rows_token_shuffle(args, md, device, stream, peak):
     """The token shuffle and the dedup dispatch after it.  Single form on
     two_layer_e128_k6, pair form on three_layer_e128_k6; counts fitted on
     tokens [0, 4096); contiguous placement at layer l+1.  After the shuffle the
@@ -758,7 +759,7 @@ def rows_config4(args, md, device, stream, peak):
     return rows
 
 
-def rows_config5_planning(args, md, device, stream, peak):
+def rows_e256_k8_planning(args, md, device, stream, peak):
     """The E=256 workload's planning steps: the full pipeline with co-selection
     counts and placement inside every step, placement modes, routing statistics."""
     from combine_warp_top_router_b200 import synth
