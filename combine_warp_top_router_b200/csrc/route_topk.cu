@@ -246,8 +246,8 @@ void launch_k(const float *logits, int64_t T, int E, int k, int gate_mode, int32
 // ---------------------------------------------------------------- thread per token
 // E in {64, 128, 256}, k in {1, 2, 4, 6, 8}: one thread per token, so the
 // selection needs no cross-lane steps.  A warp stages its 32 consecutive rows
-// (contiguous in memory) in shared memory with one bulk copy.  Lane L reads
-// its row's 16-byte chunks in the order (c + L) mod E/4, which puts the 8
+// (contiguous in memory) in shared memory with one bulk copy.  At iteration c
+// lane L reads its row's 16-byte chunk c xor (L mod 8), which puts the 8
 // lanes of a shared-memory phase on distinct banks.
 //   1. Threshold.  Chunk iteration c belongs to group c mod 16; the k-th
 //      largest of the 16 group maxima is at or below the k-th largest logit
@@ -368,10 +368,17 @@ __global__ void __launch_bounds__(32)
     // 1-2. threshold and candidate list
     int n = 0;
     if (live) {
+        // iteration c reads chunk c ^ (lane & 7): the 8 lanes of a shared-
+        // memory phase hit distinct banks, and with the 8 row pointers below
+        // each read is one load at a constant offset
+        const int sw = lane & 7;
+        const float4 *rb[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) rb[q] = row4 + (q ^ sw);
         float gm[NG];
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
-            const float4 q = row4[(c + lane) & (NCH - 1)];
+            const float4 q = rb[c & 7][c & ~7];
             const float m = fmaxf(fmaxf(q.x, q.y), fmaxf(q.z, q.w));
             gm[c % NG] = c < NG ? m : fmaxf(gm[c % NG], m);
         }
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(32)
             gmask &= gmask - 1;
 #pragma unroll
             for (int j = 0; j < NCH / NG; ++j) {  // iterations g, g + 16, ... of the first pass
-                const int ch = (g + NG * j + lane) & (NCH - 1);
+                const int ch = (g + NG * j) ^ sw;
                 const float4 q = row4[ch];
                 const int e0 = ch * 4;
                 if (q.x >= th) { lst[32 * min(n, CAP - 1)] = (uint8_t)e0; ++n; }
